@@ -1,0 +1,320 @@
+// Warp-level online-softmax attention of the RLT path.
+//
+// One warp owns one (sequence, head[, key chunk]) work item.  Lanes are grouped so that
+// LPK lanes hold one key row with 16-byte loads (LPK = head_dim * sizeof(T) / 16); the
+// KPI = 32 / LPK groups walk interleaved keys, keep their own running (max, sum, acc)
+// and are merged by shuffles at the end.  Keys and values are streamed with coalesced
+// 16-byte loads, several rounds in flight per lane.  Used for
+//   - decoder sliding-window self-attention over the ring cache plus the current token,
+//   - decoder cross-attention over the causal encoder memory M_{<=t} (split along keys
+//     when there are too few (sequence, head) pairs to fill the GPU),
+//   - the encoder's causal self-attention (one query per warp).
+#include "kernels.cuh"
+
+namespace rlt {
+
+namespace {
+
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float NEG_BIG = -1e30f;
+constexpr int WARPS = 4;
+
+template <typename T, int HD>
+struct Geom {
+    static constexpr int EPL = 16 / (int)sizeof(T);   // elements per lane
+    static constexpr int LPK = HD / EPL;               // lanes per key row
+    static constexpr int KPI = 32 / LPK;               // keys per warp round
+    static_assert(LPK >= 1 && LPK <= 32 && 32 % LPK == 0, "head_dim not supported");
+};
+
+template <int LPK>
+__device__ __forceinline__ float group_sum(float v) {
+#pragma unroll
+    for (int o = LPK / 2; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Accumulate keys [0, n) of K/V (row stride HD) into this lane group's running softmax.
+// q is pre-scaled by log2(e)/sqrt(hd).  n must be warp-uniform.
+template <typename T, int HD, int U, bool STREAM>
+__device__ __forceinline__ void attend(const float* q, const T* __restrict__ K, const T* __restrict__ V,
+                                       int n, int g, int li, float& m, float& l, float* acc) {
+    using G = Geom<T, HD>;
+    constexpr int EPL = G::EPL, LPK = G::LPK, KPI = G::KPI;
+    for (int base = 0; base < n; base += KPI * U) {
+        uint4 kr[U], vr[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            int j = base + u * KPI + g;
+            if (j < n) {
+                const T* kp = K + (long long)j * HD + li * EPL;
+                const T* vp = V + (long long)j * HD + li * EPL;
+                kr[u] = STREAM ? ld16_stream(kp) : ld16(kp);
+                vr[u] = STREAM ? ld16_stream(vp) : ld16(vp);
+            } else {
+                kr[u] = make_uint4(0, 0, 0, 0);
+                vr[u] = make_uint4(0, 0, 0, 0);
+            }
+        }
+        float s[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            float kf[EPL];
+            Vec16<T>::unpack(kr[u], kf);
+            float dot = 0.f;
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) dot = fmaf(q[i], kf[i], dot);
+            dot = group_sum<LPK>(dot);
+            s[u] = (base + u * KPI + g < n) ? dot : NEG_BIG;
+        }
+        float mx = m;
+#pragma unroll
+        for (int u = 0; u < U; ++u) mx = fmaxf(mx, s[u]);
+        float corr = exp2f(m - mx);
+        l *= corr;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) acc[i] *= corr;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            float p = (base + u * KPI + g < n) ? exp2f(s[u] - mx) : 0.f;
+            l += p;
+            float vf[EPL];
+            Vec16<T>::unpack(vr[u], vf);
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) acc[i] = fmaf(p, vf[i], acc[i]);
+        }
+        m = mx;
+    }
+}
+
+// Merge the KPI lane groups' running softmax states; afterwards every group holds the total.
+template <typename T, int HD>
+__device__ __forceinline__ void merge_groups(float& m, float& l, float* acc) {
+    using G = Geom<T, HD>;
+#pragma unroll
+    for (int o = G::LPK; o < 32; o <<= 1) {
+        float mo = __shfl_xor_sync(0xffffffffu, m, o);
+        float lo = __shfl_xor_sync(0xffffffffu, l, o);
+        float mx = fmaxf(m, mo);
+        float c1 = exp2f(m - mx), c2 = exp2f(mo - mx);
+        l = l * c1 + lo * c2;
+#pragma unroll
+        for (int i = 0; i < G::EPL; ++i) {
+            float ao = __shfl_xor_sync(0xffffffffu, acc[i], o);
+            acc[i] = acc[i] * c1 + ao * c2;
+        }
+        m = mx;
+    }
+}
+
+template <typename T, int HD>
+__global__ void __launch_bounds__(WARPS * 32) k_swa_decode(const float* __restrict__ qkv,
+                                                           const float2* __restrict__ rope_row,
+                                                           T* __restrict__ ring, T* __restrict__ o,
+                                                           int B, int H, int W, int t, float qscale) {
+    using G = Geom<T, HD>;
+    constexpr int EPL = G::EPL, LPK = G::LPK;
+    int item = blockIdx.x * WARPS + (threadIdx.x >> 5);
+    if (item >= B * H) return;
+    int lane = threadIdx.x & 31, g = lane / LPK, li = lane % LPK;
+    int b = item / H, h = item % H;
+    const int d = H * HD, half = HD / 2;
+    const float* row = qkv + (long long)b * 3 * d + h * HD;
+    float q[EPL], k[EPL], v[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        int c = li * EPL + i;
+        int cp = c < half ? c + half : c - half;
+        float2 cs = rope_row[c % half];
+        float qa = row[c], qp = row[cp];
+        float ka = row[d + c], kp = row[d + cp];
+        q[i] = (c < half ? qa * cs.x - qp * cs.y : qp * cs.y + qa * cs.x) * qscale;
+        k[i] = round_to<T>(c < half ? ka * cs.x - kp * cs.y : kp * cs.y + ka * cs.x);
+        v[i] = round_to<T>(row[2 * d + c]);
+    }
+    float sc = 0.f;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) sc = fmaf(q[i], k[i], sc);
+    sc = group_sum<LPK>(sc);
+    float m, l, acc[EPL];
+    if (g == 0) {
+        m = sc; l = 1.f;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) acc[i] = v[i];
+    } else {
+        m = NEG_BIG; l = 0.f;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) acc[i] = 0.f;
+    }
+    T* Kr = nullptr;
+    T* Vr = nullptr;
+    if (W > 1) {
+        Kr = ring + (((long long)b * 2 + 0) * H + h) * (long long)(W - 1) * HD;
+        Vr = ring + (((long long)b * 2 + 1) * H + h) * (long long)(W - 1) * HD;
+        int n = min(t - 1, W - 1);
+        attend<T, HD, 4, true>(q, Kr, Vr, n, g, li, m, l, acc);
+    }
+    merge_groups<T, HD>(m, l, acc);
+    __syncwarp();
+    if (g == 0) {
+        if (W > 1) {
+            int slot = (t - 1) % (W - 1);
+            st16(Kr + (long long)slot * HD + li * EPL, Vec16<T>::pack(k));
+            st16(Vr + (long long)slot * HD + li * EPL, Vec16<T>::pack(v));
+        }
+        float inv = 1.0f / l, out[EPL];
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) out[i] = acc[i] * inv;
+        st16(o + (long long)b * d + h * HD + li * EPL, Vec16<T>::pack(out));
+    }
+}
+
+template <typename T, int HD>
+__global__ void __launch_bounds__(WARPS * 32) k_xattn_decode(const float* __restrict__ qc,
+                                                             const T* __restrict__ Mg, int T_alloc, int t,
+                                                             T* __restrict__ o, int B, int H, int n_splits,
+                                                             int chunk, float* __restrict__ part, float qscale) {
+    using G = Geom<T, HD>;
+    constexpr int EPL = G::EPL, LPK = G::LPK;
+    int item = blockIdx.x * WARPS + (threadIdx.x >> 5);
+    if (item >= B * H * n_splits) return;
+    int lane = threadIdx.x & 31, g = lane / LPK, li = lane % LPK;
+    int bh = item / n_splits, sp = item % n_splits;
+    int b = bh / H, h = bh % H;
+    const int d = H * HD;
+    float q[EPL];
+    const float* qr = qc + (long long)b * d + h * HD + li * EPL;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) q[i] = qr[i] * qscale;
+    long long plane = (long long)B * H * T_alloc * HD;
+    const T* K = Mg + (long long)bh * T_alloc * HD;
+    const T* V = K + plane;
+    int j0 = sp * chunk;
+    int n = max(0, min(t, j0 + chunk) - j0);
+    float m = NEG_BIG, l = 0.f, acc[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) acc[i] = 0.f;
+    attend<T, HD, 4, true>(q, K + (long long)j0 * HD, V + (long long)j0 * HD, n, g, li, m, l, acc);
+    merge_groups<T, HD>(m, l, acc);
+    if (g != 0) return;
+    if (n_splits == 1) {
+        float inv = 1.0f / l, out[EPL];
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) out[i] = acc[i] * inv;
+        st16(o + (long long)b * d + h * HD + li * EPL, Vec16<T>::pack(out));
+    } else {
+        float* pp = part + (long long)item * (HD + 2);
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) pp[li * EPL + i] = acc[i];
+        if (li == 0) { pp[HD] = m; pp[HD + 1] = l; }
+    }
+}
+
+// Combine key-split partials: one block per (b, h), one thread per output element.
+template <typename T>
+__global__ void k_attn_combine(const float* __restrict__ part, int n_splits, int HD, int H,
+                               T* __restrict__ o) {
+    int bh = blockIdx.x, c = threadIdx.x;
+    if (c >= HD) return;
+    const float* p = part + (long long)bh * n_splits * (HD + 2);
+    float mx = NEG_BIG;
+    for (int s = 0; s < n_splits; ++s) mx = fmaxf(mx, p[s * (HD + 2) + HD]);
+    float L = 0.f, A = 0.f;
+    for (int s = 0; s < n_splits; ++s) {
+        float w = exp2f(p[s * (HD + 2) + HD] - mx);
+        L += p[s * (HD + 2) + HD + 1] * w;
+        A += p[s * (HD + 2) + c] * w;
+    }
+    int b = bh / H, h = bh % H;
+    o[(long long)b * H * HD + h * HD + c] = from_f<T>(A / L);
+}
+
+template <typename T, int HD>
+__global__ void __launch_bounds__(WARPS * 32) k_enc_attn(const T* __restrict__ planes, T* __restrict__ o,
+                                                         int B, int Tn, int H, float qscale) {
+    using G = Geom<T, HD>;
+    constexpr int EPL = G::EPL, LPK = G::LPK;
+    long long item = (long long)blockIdx.x * WARPS + (threadIdx.x >> 5);
+    if (item >= (long long)B * H * Tn) return;
+    int lane = threadIdx.x & 31, g = lane / LPK, li = lane % LPK;
+    long long bh = item / Tn;
+    int i = (int)(item % Tn);
+    long long plane = (long long)B * H * Tn * HD;
+    const T* Q = planes + bh * Tn * HD;
+    const T* K = planes + plane + bh * Tn * HD;
+    const T* V = planes + 2 * plane + bh * Tn * HD;
+    float q[EPL];
+    Vec16<T>::unpack(ld16(Q + (long long)i * HD + li * EPL), q);
+#pragma unroll
+    for (int x = 0; x < EPL; ++x) q[x] *= qscale;
+    float m = NEG_BIG, l = 0.f, acc[EPL];
+#pragma unroll
+    for (int x = 0; x < EPL; ++x) acc[x] = 0.f;
+    attend<T, HD, 4, false>(q, K, V, i + 1, g, li, m, l, acc);
+    merge_groups<T, HD>(m, l, acc);
+    if (g != 0) return;
+    int b = (int)(bh / H), h = (int)(bh % H);
+    float inv = 1.0f / l, out[EPL];
+#pragma unroll
+    for (int x = 0; x < EPL; ++x) out[x] = acc[x] * inv;
+    st16(o + ((long long)b * Tn + i) * H * HD + h * HD + li * EPL, Vec16<T>::pack(out));
+}
+
+inline float qscale_for(int hd) { return LOG2E / sqrtf((float)hd); }
+inline unsigned blocks_for(long long items) { return (unsigned)((items + WARPS - 1) / WARPS); }
+
+}  // namespace
+
+#define RLT_HD_SWITCH(hd, KERNEL_CALL)          \
+    switch (hd) {                               \
+        case 16: { constexpr int HD = 16; KERNEL_CALL; break; }   \
+        case 32: { constexpr int HD = 32; KERNEL_CALL; break; }   \
+        case 64: { constexpr int HD = 64; KERNEL_CALL; break; }   \
+        case 128: { constexpr int HD = 128; KERNEL_CALL; break; } \
+        default: return cudaErrorInvalidValue;  \
+    }
+
+template <typename T>
+cudaError_t launch_swa_decode(Launch L, const float* qkv, const float2* rope_row, T* ring, T* o, int B,
+                              int H, int hd, int W, int t) {
+    RLT_HD_SWITCH(hd, (k_swa_decode<T, HD><<<blocks_for((long long)B * H), WARPS * 32, 0, L.stream>>>(
+                           qkv, rope_row, ring, o, B, H, W, t, qscale_for(hd))));
+    *L.count += 1;
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_xattn_decode(Launch L, const float* qc, const T* Mg, int T_alloc, int t, T* o, int B,
+                                int H, int hd, int n_splits, float* part) {
+    if (n_splits < 1) n_splits = 1;
+    int chunk = (t + n_splits - 1) / n_splits;
+    RLT_HD_SWITCH(hd, (k_xattn_decode<T, HD><<<blocks_for((long long)B * H * n_splits), WARPS * 32, 0,
+                                               L.stream>>>(qc, Mg, T_alloc, t, o, B, H, n_splits, chunk,
+                                                           part, qscale_for(hd))));
+    *L.count += 1;
+    if (n_splits > 1) {
+        k_attn_combine<T><<<B * H, hd, 0, L.stream>>>(part, n_splits, hd, H, o);
+        *L.count += 1;
+    }
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_enc_attention(Launch L, const T* planes, T* o, int B, int Tn, int H, int hd) {
+    RLT_HD_SWITCH(hd, (k_enc_attn<T, HD><<<blocks_for((long long)B * H * Tn), WARPS * 32, 0, L.stream>>>(
+                           planes, o, B, Tn, H, qscale_for(hd))));
+    *L.count += 1;
+    return cudaGetLastError();
+}
+
+#define RLT_INST(T)                                                                                    \
+    template cudaError_t launch_swa_decode<T>(Launch, const float*, const float2*, T*, T*, int, int,   \
+                                              int, int, int);                                          \
+    template cudaError_t launch_xattn_decode<T>(Launch, const float*, const T*, int, int, T*, int, int, \
+                                                int, int, float*);                                     \
+    template cudaError_t launch_enc_attention<T>(Launch, const T*, T*, int, int, int, int);
+RLT_INST(float)
+RLT_INST(bf16)
+#undef RLT_INST
+
+}  // namespace rlt

@@ -1,0 +1,326 @@
+// Bandwidth-bound elementwise kernels of the RLT path: weight packing, rotary table,
+// embedding gather, RMSNorm, merge input assembly, final norm, fused log-softmax gather,
+// and the layout kernels of the encoder.
+#include "kernels.cuh"
+
+namespace rlt {
+
+namespace {
+
+inline unsigned cdiv(long long a, long long b) { return (unsigned)((a + b - 1) / b); }
+
+template <typename T>
+__global__ void k_pack_rows(const float* __restrict__ src, T* __restrict__ dst, int rows, int cols,
+                            int dst_ld, int row_mult, int row_off, int col_off) {
+    long long n = (long long)rows * cols;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+         i += (long long)gridDim.x * blockDim.x) {
+        int r = (int)(i / cols), c = (int)(i % cols);
+        dst[((long long)r * row_mult + row_off) * dst_ld + col_off + c] = from_f<T>(src[i]);
+    }
+}
+
+__global__ void k_rope_table(float2* table, int max_pos, int half, int hd, double base) {
+    long long n = (long long)max_pos * half;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+         i += (long long)gridDim.x * blockDim.x) {
+        int p = (int)(i / half), f = (int)(i % half);
+        double inv = pow(base, -2.0 * f / hd);
+        double s, c;
+        sincos((double)p * inv, &s, &c);
+        table[i] = make_float2((float)c, (float)s);
+    }
+}
+
+template <typename T>
+__global__ void k_embed(const int32_t* __restrict__ tok, int N, const T* __restrict__ embed, int V,
+                        int d, float* __restrict__ h, DevHeader* hdr) {
+    int n = blockIdx.x;
+    if (n >= N) return;
+    int id = tok[n];
+    if (id < 0 || id >= V) {
+        if (threadIdx.x == 0) raise_flag(hdr, ERR_BAD_TOKEN);
+        id = 0;
+    }
+    const T* row = embed + (long long)id * d;
+    float* out = h + (long long)n * d;
+    for (int c = threadIdx.x; c < d; c += blockDim.x) out[c] = to_f(row[c]);
+}
+
+// One warp per row.  d is a multiple of 8, so float4 loads cover the row exactly.
+template <typename T>
+__global__ void k_rmsnorm(const float* __restrict__ x, int N, int d, const float* __restrict__ gain,
+                          float eps, T* __restrict__ out, int out_ld, int rows_per_seq,
+                          int out_rows_per_seq, T* __restrict__ out2) {
+    int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    int lane = threadIdx.x & 31;
+    if (warp >= N) return;
+    const float4* xr = reinterpret_cast<const float4*>(x + (long long)warp * d);
+    float ss = 0.f;
+    for (int c = lane; c < d / 4; c += 32) {
+        float4 v = xr[c];
+        ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+    }
+    ss = warp_sum(ss);
+    float r = 1.0f / sqrtf(ss / d + eps);
+    long long orow = (long long)(warp / rows_per_seq) * out_rows_per_seq + warp % rows_per_seq;
+    T* o = out + orow * out_ld;
+    T* o2 = out2 ? out2 + (long long)warp * d : nullptr;
+    for (int c = lane; c < d / 4; c += 32) {
+        float4 v = xr[c];
+        float4 g = reinterpret_cast<const float4*>(gain)[c];
+        float y[4] = {v.x * r * g.x, v.y * r * g.y, v.z * r * g.z, v.w * r * g.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            o[4 * c + i] = from_f<T>(y[i]);
+            if (o2) o2[4 * c + i] = from_f<T>(y[i]);
+        }
+    }
+}
+
+template <typename T>
+__global__ void k_merge_prep(const T* __restrict__ e, int T_alloc, int t, const float* __restrict__ s,
+                             T* __restrict__ A, int B, int d, const StateHeader* sh, uint64_t version,
+                             DevHeader* hdr) {
+    int b = blockIdx.x;
+    if (b == 0 && threadIdx.x == 0 && sh) {
+        if (sh->magic != STATE_MAGIC || sh->t != t - 1 || sh->version != version)
+            raise_flag(hdr, ERR_STATE_MISMATCH);
+    }
+    const T* er = e + ((long long)b * T_alloc + (t - 1)) * d;
+    T* ar = A + (long long)b * 2 * d;
+    const float* sr = s + (long long)b * d;
+    for (int c = threadIdx.x; c < d; c += blockDim.x) {
+        ar[c] = er[c];
+        ar[d + c] = from_f<T>(sr[c]);
+    }
+}
+
+template <typename T>
+__global__ void k_final_norm(const float* __restrict__ x, int B, int d, const float* __restrict__ gain,
+                             float eps, float* __restrict__ s, T* __restrict__ hs, StateHeader* sh, int t) {
+    int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    int lane = threadIdx.x & 31;
+    if (warp == 0 && lane == 0 && sh) sh->t = t;
+    if (warp >= B) return;
+    const float* xr = x + (long long)warp * d;
+    float ss = 0.f;
+    for (int c = lane; c < d; c += 32) ss += xr[c] * xr[c];
+    ss = warp_sum(ss);
+    float r = 1.0f / sqrtf(ss / d + eps);
+    for (int c = lane; c < d; c += 32) {
+        float y = xr[c] * r * gain[c];
+        s[(long long)warp * d + c] = y;
+        hs[(long long)warp * d + c] = from_f<T>(y);
+    }
+}
+
+// One block per row.  Online (max, sum) per thread, then a block reduction.
+__global__ void k_lse_gather(const float* __restrict__ logits, int B, int V, float tau,
+                             const int32_t* __restrict__ tok, int tok_stride, float* logp_tok,
+                             int lp_stride, float* lse_out, float* logp_full, float* score,
+                             const int32_t* prompt_len, int t, DevHeader* hdr) {
+    int b = blockIdx.x;
+    const float* z = logits + (long long)b * V;
+    float m = -INFINITY, l = 0.f;
+    for (int i = threadIdx.x; i < V; i += blockDim.x) {
+        float v = z[i] / tau;
+        if (v > m) { l = l * expf(m - v) + 1.f; m = v; }
+        else l += expf(v - m);
+    }
+    __shared__ float sm[32], sl[32];
+    int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    float mw = warp_max(m);
+    l = (m == -INFINITY) ? 0.f : l * expf(m - mw);
+    l = warp_sum(l);
+    if (lane == 0) { sm[wid] = mw; sl[wid] = l; }
+    __syncthreads();
+    if (wid == 0) {
+        float mm = lane < nw ? sm[lane] : -INFINITY;
+        float ll = lane < nw ? sl[lane] : 0.f;
+        float mx = warp_max(mm);
+        ll = (mm == -INFINITY) ? 0.f : ll * expf(mm - mx);
+        ll = warp_sum(ll);
+        if (lane == 0) { sm[0] = mx; sl[0] = ll; }
+    }
+    __syncthreads();
+    float lse = sm[0] + logf(sl[0]);
+    if (threadIdx.x == 0) {
+        if (lse_out) lse_out[b] = lse;
+        if (tok) {
+            int id = tok[(long long)b * tok_stride];
+            if (id < 0 || id >= V) { raise_flag(hdr, ERR_BAD_TOKEN); id = 0; }
+            float lp = z[id] / tau - lse;
+            if (logp_tok) logp_tok[(long long)b * lp_stride] = lp;
+            if (score && t >= prompt_len[b]) score[b] += lp;
+        }
+    }
+    if (logp_full) {
+        float* out = logp_full + (long long)b * V;
+        for (int i = threadIdx.x; i < V; i += blockDim.x) out[i] = z[i] / tau - lse;
+    }
+}
+
+// thread per (n, h, i < hd/2): rotate the pair (i, i + hd/2) of q and k, round q, k, v.
+template <typename T>
+__global__ void k_enc_qkv_layout(const float* __restrict__ qkv, int B, int Tn, int H, int hd,
+                                 const float2* __restrict__ rope, T* __restrict__ planes) {
+    int half = hd / 2;
+    int d = H * hd;
+    long long total = (long long)B * Tn * H * half;
+    long long plane = (long long)B * H * Tn * hd;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        int f = (int)(i % half);
+        long long r = i / half;
+        int h = (int)(r % H);
+        long long n = r / H;
+        int b = (int)(n / Tn), p = (int)(n % Tn);
+        const float* row = qkv + n * 3 * d + h * hd;
+        float2 cs = rope[(long long)p * half + f];
+        long long o = (((long long)b * H + h) * Tn + p) * hd;
+        float qa = row[f], qb = row[f + half];
+        float ka = row[d + f], kb = row[d + f + half];
+        planes[o + f] = from_f<T>(qa * cs.x - qb * cs.y);
+        planes[o + f + half] = from_f<T>(qa * cs.y + qb * cs.x);
+        planes[plane + o + f] = from_f<T>(ka * cs.x - kb * cs.y);
+        planes[plane + o + f + half] = from_f<T>(ka * cs.y + kb * cs.x);
+        planes[2 * plane + o + f] = from_f<T>(row[2 * d + f]);
+        planes[2 * plane + o + f + half] = from_f<T>(row[2 * d + f + half]);
+    }
+}
+
+template <typename T>
+__global__ void k_mem_layout(const float* __restrict__ kv, int B, int Tn, int T_alloc, int H, int hd,
+                             T* __restrict__ Mg) {
+    int d = H * hd;
+    long long total = (long long)B * Tn * 2 * d;
+    long long plane = (long long)B * H * T_alloc * hd;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        int c = (int)(i % (2 * d));
+        long long n = i / (2 * d);
+        int b = (int)(n / Tn), p = (int)(n % Tn);
+        int kvsel = c / d, h = (c % d) / hd, x = c % hd;
+        Mg[kvsel * plane + (((long long)b * H + h) * T_alloc + p) * hd + x] = from_f<T>(kv[i]);
+    }
+}
+
+__global__ void k_state_init(const float* __restrict__ s_star, int B, int d, float* __restrict__ s,
+                             StateHeader* sh, uint64_t version) {
+    long long n = (long long)B * d;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+         i += (long long)gridDim.x * blockDim.x)
+        s[i] = s_star[i % d];
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        sh->magic = STATE_MAGIC;
+        sh->t = 0;
+        sh->version = version;
+        sh->B = B;
+    }
+}
+
+inline unsigned grid_for(long long n, int threads) {
+    long long g = (n + threads - 1) / threads;
+    return (unsigned)(g > 148LL * 64 ? 148LL * 64 : (g < 1 ? 1 : g));
+}
+
+inline cudaError_t done(Launch L, int n = 1) {
+    *L.count += n;
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+template <typename T>
+cudaError_t launch_pack_rows(Launch L, const float* src, T* dst, int rows, int cols, int dst_ld,
+                             int row_mult, int row_off, int col_off) {
+    k_pack_rows<T><<<grid_for((long long)rows * cols, 256), 256, 0, L.stream>>>(
+        src, dst, rows, cols, dst_ld, row_mult, row_off, col_off);
+    return done(L);
+}
+
+cudaError_t launch_rope_table(Launch L, float2* table, int max_pos, int head_dim, float base) {
+    int half = head_dim / 2;
+    k_rope_table<<<grid_for((long long)max_pos * half, 256), 256, 0, L.stream>>>(
+        table, max_pos, half, head_dim, (double)base);
+    return done(L);
+}
+
+template <typename T>
+cudaError_t launch_embed(Launch L, const int32_t* tok, int N, const T* embed, int V, int d, float* h,
+                         DevHeader* hdr) {
+    k_embed<T><<<N, 128, 0, L.stream>>>(tok, N, embed, V, d, h, hdr);
+    return done(L);
+}
+
+template <typename T>
+cudaError_t launch_rmsnorm(Launch L, const float* x, int N, int d, const float* gain, float eps, T* out,
+                           int out_ld, int rows_per_seq, int out_rows_per_seq, T* out2) {
+    k_rmsnorm<T><<<cdiv(N, 8), 256, 0, L.stream>>>(x, N, d, gain, eps, out, out_ld, rows_per_seq,
+                                                     out_rows_per_seq, out2);
+    return done(L);
+}
+
+template <typename T>
+cudaError_t launch_merge_prep(Launch L, const T* e, int T_alloc, int t, const float* s, T* A, int B,
+                              int d, const StateHeader* sh, uint64_t version, DevHeader* hdr) {
+    k_merge_prep<T><<<B, 256, 0, L.stream>>>(e, T_alloc, t, s, A, B, d, sh, version, hdr);
+    return done(L);
+}
+
+template <typename T>
+cudaError_t launch_final_norm(Launch L, const float* x, int B, int d, const float* gain, float eps,
+                              float* s, T* hs, StateHeader* sh, int t) {
+    k_final_norm<T><<<cdiv(B, 8), 256, 0, L.stream>>>(x, B, d, gain, eps, s, hs, sh, t);
+    return done(L);
+}
+
+cudaError_t launch_lse_gather(Launch L, const float* logits, int B, int V, float tau, const int32_t* tok,
+                              int tok_stride, float* logp_tok, int lp_stride, float* lse,
+                              float* logp_full, float* score, const int32_t* prompt_len, int t,
+                              DevHeader* hdr) {
+    k_lse_gather<<<B, 512, 0, L.stream>>>(logits, B, V, tau, tok, tok_stride, logp_tok, lp_stride, lse,
+                                          logp_full, score, prompt_len, t, hdr);
+    return done(L);
+}
+
+template <typename T>
+cudaError_t launch_enc_qkv_layout(Launch L, const float* qkv, int B, int Tn, int H, int hd,
+                                  const float2* rope, T* planes) {
+    k_enc_qkv_layout<T><<<grid_for((long long)B * Tn * H * (hd / 2), 256), 256, 0, L.stream>>>(
+        qkv, B, Tn, H, hd, rope, planes);
+    return done(L);
+}
+
+template <typename T>
+cudaError_t launch_mem_layout(Launch L, const float* kv, int B, int Tn, int T_alloc, int H, int hd, T* Mg) {
+    k_mem_layout<T><<<grid_for((long long)B * Tn * 2 * H * hd, 256), 256, 0, L.stream>>>(
+        kv, B, Tn, T_alloc, H, hd, Mg);
+    return done(L);
+}
+
+cudaError_t launch_state_init(Launch L, const float* s_star, int B, int d, float* s, StateHeader* sh,
+                              uint64_t version) {
+    k_state_init<<<grid_for((long long)B * d, 256), 256, 0, L.stream>>>(s_star, B, d, s, sh, version);
+    return done(L);
+}
+
+#define RLT_INST(T)                                                                                   \
+    template cudaError_t launch_pack_rows<T>(Launch, const float*, T*, int, int, int, int, int, int); \
+    template cudaError_t launch_embed<T>(Launch, const int32_t*, int, const T*, int, int, float*,     \
+                                         DevHeader*);                                                 \
+    template cudaError_t launch_rmsnorm<T>(Launch, const float*, int, int, const float*, float, T*,   \
+                                           int, int, int, T*);                                        \
+    template cudaError_t launch_merge_prep<T>(Launch, const T*, int, int, const float*, T*, int, int, \
+                                              const StateHeader*, uint64_t, DevHeader*);              \
+    template cudaError_t launch_final_norm<T>(Launch, const float*, int, int, const float*, float,    \
+                                              float*, T*, StateHeader*, int);                         \
+    template cudaError_t launch_enc_qkv_layout<T>(Launch, const float*, int, int, int, int,           \
+                                                  const float2*, T*);                                 \
+    template cudaError_t launch_mem_layout<T>(Launch, const float*, int, int, int, int, int, T*);
+RLT_INST(float)
+RLT_INST(bf16)
+#undef RLT_INST
+
+}  // namespace rlt

@@ -1,0 +1,89 @@
+// Host-side launchers of the RLT kernels.  Every launcher enqueues exactly the kernels
+// it names on `L.stream`, adds their number to *L.count and returns the launch status.
+#pragma once
+
+#include "common.cuh"
+
+namespace rlt {
+
+struct Launch {
+    cudaStream_t stream;
+    uint64_t* count;
+};
+
+// ------------------------------------------------------------------ elementwise.cu
+// dst[(r*row_mult + row_off) * dst_ld + col_off + c] = T(src[r*cols + c])
+template <typename T>
+cudaError_t launch_pack_rows(Launch L, const float* src, T* dst, int rows, int cols, int dst_ld,
+                             int row_mult, int row_off, int col_off);
+// table[p*half + i] = (cos, sin)(p * base^(-2i/hd)), computed in double precision
+cudaError_t launch_rope_table(Launch L, float2* table, int max_pos, int head_dim, float base);
+// h[n, :] = embed[tok[n], :] in float32
+template <typename T>
+cudaError_t launch_embed(Launch L, const int32_t* tok, int N, const T* embed, int V, int d, float* h,
+                         DevHeader* hdr);
+// out[row_map(n), out_col_off + :] = T(RMSNorm(x[n, :]) * gain).  row_map(n) =
+// (n / rows_per_seq) * out_rows_per_seq + n % rows_per_seq; out2 (optional) is a second
+// contiguous T copy with leading dimension d.
+template <typename T>
+cudaError_t launch_rmsnorm(Launch L, const float* x, int N, int d, const float* gain, float eps,
+                           T* out, int out_ld, int rows_per_seq, int out_rows_per_seq, T* out2);
+// A[b, :] = [e[b, t-1, :] | T(s[b, :])]; also checks the state header
+template <typename T>
+cudaError_t launch_merge_prep(Launch L, const T* e, int T_alloc, int t, const float* s, T* A, int B,
+                              int d, const StateHeader* sh, uint64_t version, DevHeader* hdr);
+// s[b, :] = RMSNorm(x[b, :]) * gain (float32) and hs = T(s); sets the state header's t
+template <typename T>
+cudaError_t launch_final_norm(Launch L, const float* x, int B, int d, const float* gain, float eps,
+                              float* s, T* hs, StateHeader* sh, int t);
+// Per row b: z = logits[b, :] / tau, lse = logsumexp(z), gather z[tok] - lse, optional full
+// row, optional score accumulation when t >= P[b].
+cudaError_t launch_lse_gather(Launch L, const float* logits, int B, int V, float tau,
+                              const int32_t* tok, int tok_stride, float* logp_tok, int lp_stride,
+                              float* lse, float* logp_full, float* score, const int32_t* prompt_len,
+                              int t, DevHeader* hdr);
+// Encoder q/k/v: qkv float32 [B*T, 3d] -> planes T [3][B][H][T][hd], RoPE on q and k.
+template <typename T>
+cudaError_t launch_enc_qkv_layout(Launch L, const float* qkv, int B, int Tn, int H, int hd,
+                                  const float2* rope, T* planes);
+// Memory projection output float32 [B*T, 2d] -> M_g T [2][B][H][T_alloc][hd]
+template <typename T>
+cudaError_t launch_mem_layout(Launch L, const float* kv, int B, int Tn, int T_alloc, int H, int hd,
+                              T* Mg);
+// H_0: s[b, :] = s_star, header (t=0, version, B)
+cudaError_t launch_state_init(Launch L, const float* s_star, int B, int d, float* s, StateHeader* sh,
+                              uint64_t version);
+
+// ------------------------------------------------------------------ gemm_simt.cu
+// C[M, N] = A[M, K] (leading dim lda) x W[N, K]^T, float32 accumulation, then an epilogue.
+enum class Epi { StoreF32, ResidAdd, SwiGLU, Merge };
+struct EpiArgs {
+    float* out_f32 = nullptr;   // StoreF32 target / ResidAdd accumulator / Merge output x
+    void* out_t = nullptr;      // SwiGLU output (storage type)
+    int ld_out = 0;
+    float scale = 1.0f;         // StoreF32 multiplier
+    const void* merge_e = nullptr;  // Merge: e_t rows (storage type), leading dim ld_e
+    int ld_e = 0;
+    const float* bias = nullptr;    // Merge: gate bias b_g
+};
+template <typename T>
+cudaError_t launch_gemm(Launch L, Epi epi, const T* A, int lda, const T* W, int M, int N, int K,
+                        const EpiArgs& ea);
+
+// ------------------------------------------------------------------ attention.cu
+// Decoder sliding-window self-attention for one layer at step t (1-based): RoPE at
+// position t-1 on q/k from qkv [B, 3d]; attends over the min(t-1, W-1) cached entries plus
+// the current token; then stores k_t, v_t into ring slot (t-1) mod (W-1).
+template <typename T>
+cudaError_t launch_swa_decode(Launch L, const float* qkv, const float2* rope_row, T* ring, T* o,
+                              int B, int H, int hd, int W, int t);
+// Decoder cross-attention over M_{<=t} (positions 0..t-1) of one memory group.
+// Splits the keys of each (b, h) into n_splits chunks when n_splits > 1 (partials in `part`).
+template <typename T>
+cudaError_t launch_xattn_decode(Launch L, const float* qc, const T* Mg, int T_alloc, int t, T* o,
+                                int B, int H, int hd, int n_splits, float* part);
+// Encoder causal self-attention: planes T [3][B][H][T][hd] -> o T [B*T, d]
+template <typename T>
+cudaError_t launch_enc_attention(Launch L, const T* planes, T* o, int B, int Tn, int H, int hd);
+
+}  // namespace rlt

@@ -1,0 +1,695 @@
+// C ABI of the RLT library (declared in include/rlt.h): model arena layout, weight
+// packing, the decoder-state registry and the encode / decode-step / replay drivers.
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <unordered_map>
+#include <unordered_set>
+#include <vector>
+
+#include "rlt.h"
+#include "kernels.cuh"
+
+using namespace rlt;
+
+namespace {
+
+constexpr size_t ALIGN = 256;
+inline size_t align_up(size_t x) { return (x + ALIGN - 1) / ALIGN * ALIGN; }
+inline bool aligned(const void* p, size_t a = ALIGN) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Cross-attention key-split partials: capacity in (sequence, head, split) work items.
+constexpr long long XATTN_PART_ITEMS = 32768;
+constexpr int XATTN_MAX_SPLITS = 64;
+constexpr int XATTN_MIN_CHUNK = 64;
+constexpr long long XATTN_TARGET_WARPS = 148LL * 64 * 2;
+
+struct Layout {
+    size_t esz = 0;             // bytes per stored element
+    size_t rope = 0, embed = 0, enc_norm = 0, mem = 0, merge_w = 0, merge_b = 0, s_star = 0,
+           dec_norm = 0, unembed = 0, total = 0;
+    std::vector<size_t> attn_norm, wqkv, wo, ffn_norm, wgu, wdown, xattn_norm, wqc, woc;
+};
+
+bool config_ok(const rlt_config& c) {
+    if (c.V < 8 || c.d < 8 || c.n_heads < 1 || c.L_E < 1 || c.L_D < 1 || c.F < 8 || c.W < 1) return false;
+    if (c.head_dim != 16 && c.head_dim != 32 && c.head_dim != 64 && c.head_dim != 128) return false;
+    if (c.n_heads * c.head_dim != c.d) return false;
+    if (c.d % 8 || c.F % 8 || c.V % 8) return false;
+    if (c.L_E != c.L_D) return false;
+    if (c.G != 1 && c.G != c.L_D) return false;
+    if (c.dtype != RLT_F32 && c.dtype != RLT_BF16) return false;
+    if (c.max_pos < 1 || !(c.rms_eps >= 0.f) || !(c.rope_base > 1.f)) return false;
+    return true;
+}
+
+Layout make_layout(const rlt_config& c) {
+    Layout L;
+    L.esz = c.dtype == RLT_BF16 ? 2 : 4;
+    size_t off = ALIGN;   // DevHeader
+    auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes); return o; };
+    size_t d = c.d, F = c.F, V = c.V, e = L.esz;
+    L.rope = take((size_t)c.max_pos * (c.head_dim / 2) * sizeof(float2));
+    L.embed = take(V * d * e);
+    for (int l = 0; l < c.L_E; ++l) {
+        L.attn_norm.push_back(take(d * 4));
+        L.wqkv.push_back(take(3 * d * d * e));
+        L.wo.push_back(take(d * d * e));
+        L.ffn_norm.push_back(take(d * 4));
+        L.wgu.push_back(take(2 * F * d * e));
+        L.wdown.push_back(take(d * F * e));
+    }
+    L.enc_norm = take(d * 4);
+    L.mem = take((size_t)c.G * 2 * d * d * e);
+    for (int l = 0; l < c.L_D; ++l) {
+        L.xattn_norm.push_back(take(d * 4));
+        L.wqc.push_back(take(d * d * e));
+        L.woc.push_back(take(d * d * e));
+    }
+    L.merge_w = take(4 * d * d * e);
+    L.merge_b = take(d * 4);
+    L.s_star = take(d * 4);
+    L.dec_norm = take(d * 4);
+    L.unembed = take(V * d * e);
+    L.total = off;
+    return L;
+}
+
+struct StateInfo {
+    int B;
+    int64_t t;
+    uint64_t version;
+};
+
+// How one canonical weight maps into the arena.
+struct Dest {
+    bool ok = false;
+    bool vec = false;          // float32 vector copy
+    size_t off = 0;            // arena byte offset
+    size_t numel = 0;
+    int rows = 0, cols = 0, dst_ld = 0, row_mult = 1, row_off = 0, col_off = 0;
+    int groups = 1;            // mem_k / mem_v: G separate [d, d] blocks
+    size_t group_stride = 0;   // bytes between group blocks in the arena
+};
+
+bool parse_layer(const std::string& name, const char* prefix, int& l, std::string& field) {
+    size_t n = strlen(prefix);
+    if (name.compare(0, n, prefix) != 0) return false;
+    size_t dot = name.find('.', n);
+    if (dot == std::string::npos || dot == n) return false;
+    for (size_t i = n; i < dot; ++i)
+        if (name[i] < '0' || name[i] > '9') return false;
+    l = std::stoi(name.substr(n, dot - n));
+    field = name.substr(dot + 1);
+    return true;
+}
+
+}  // namespace
+
+// Event pairs around selected launches (rlt_profile_start / rlt_profile_stop).
+struct Profiler {
+    bool on = false;
+    uint32_t mask = 0;
+    std::vector<cudaEvent_t> pool;
+    size_t used = 0;
+    std::vector<std::pair<int, size_t>> recs;   // (kind, index of the start event)
+
+    int begin(int kind, cudaStream_t st) {
+        if (!on || !(mask & (1u << kind))) return -1;
+        while (pool.size() < used + 2) {
+            cudaEvent_t e;
+            if (cudaEventCreate(&e) != cudaSuccess) return -1;
+            pool.push_back(e);
+        }
+        size_t i = used;
+        used += 2;
+        cudaEventRecord(pool[i], st);
+        recs.push_back({kind, i});
+        return (int)i;
+    }
+    void end(int i, cudaStream_t st) {
+        if (i >= 0) cudaEventRecord(pool[i + 1], st);
+    }
+    ~Profiler() {
+        for (auto e : pool) cudaEventDestroy(e);
+    }
+};
+
+struct rlt_model {
+    Profiler prof;
+    rlt_config cfg;
+    Layout lay;
+    uint8_t* arena = nullptr;
+    uint64_t version = 0;
+    std::unordered_set<std::string> loaded;
+    std::vector<std::string> required;
+    std::unordered_map<const void*, StateInfo> states;
+    uint64_t launches = 0;
+
+    DevHeader* hdr() const { return reinterpret_cast<DevHeader*>(arena); }
+    template <typename T> T* at(size_t off) const { return reinterpret_cast<T*>(arena + off); }
+    Launch launch(void* stream) { return Launch{reinterpret_cast<cudaStream_t>(stream), &launches}; }
+
+    Dest dest(const std::string& name) const {
+        const rlt_config& c = cfg;
+        Dest D;
+        int d = c.d, F = c.F, V = c.V;
+        auto mat = [&](size_t off, int rows, int cols, int dst_ld, int mult, int roff, int coff) {
+            D.ok = true; D.off = off; D.rows = rows; D.cols = cols; D.dst_ld = dst_ld;
+            D.row_mult = mult; D.row_off = roff; D.col_off = coff; D.numel = (size_t)rows * cols;
+        };
+        auto vec = [&](size_t off) { D.ok = true; D.vec = true; D.off = off; D.numel = d; };
+        int l;
+        std::string f;
+        if (name == "embed") mat(lay.embed, V, d, d, 1, 0, 0);
+        else if (name == "unembed") mat(lay.unembed, V, d, d, 1, 0, 0);
+        else if (name == "enc_norm") vec(lay.enc_norm);
+        else if (name == "dec_norm") vec(lay.dec_norm);
+        else if (name == "s_star") vec(lay.s_star);
+        else if (name == "merge_bias") vec(lay.merge_b);
+        else if (name == "merge_ge") mat(lay.merge_w, d, d, 2 * d, 2, 0, 0);
+        else if (name == "merge_gs") mat(lay.merge_w, d, d, 2 * d, 2, 0, d);
+        else if (name == "merge_fb") mat(lay.merge_w, d, d, 2 * d, 2, 1, d);
+        else if (name == "mem_k" || name == "mem_v") {
+            mat(lay.mem, d, d, d, 1, name == "mem_k" ? 0 : d, 0);
+            D.groups = c.G;
+            D.group_stride = (size_t)2 * d * d * lay.esz;
+            D.numel = (size_t)c.G * d * d;
+        } else if (parse_layer(name, "layers.", l, f) && l >= 0 && l < c.L_E) {
+            if (f == "attn_norm") vec(lay.attn_norm[l]);
+            else if (f == "ffn_norm") vec(lay.ffn_norm[l]);
+            else if (f == "wq") mat(lay.wqkv[l], d, d, d, 1, 0, 0);
+            else if (f == "wk") mat(lay.wqkv[l], d, d, d, 1, d, 0);
+            else if (f == "wv") mat(lay.wqkv[l], d, d, d, 1, 2 * d, 0);
+            else if (f == "wo") mat(lay.wo[l], d, d, d, 1, 0, 0);
+            else if (f == "w_gate") mat(lay.wgu[l], F, d, d, 2, 0, 0);
+            else if (f == "w_up") mat(lay.wgu[l], F, d, d, 2, 1, 0);
+            else if (f == "w_down") mat(lay.wdown[l], d, F, F, 1, 0, 0);
+        } else if (parse_layer(name, "dec.", l, f) && l >= 0 && l < c.L_D) {
+            if (f == "xattn_norm") vec(lay.xattn_norm[l]);
+            else if (f == "w_qc") mat(lay.wqc[l], d, d, d, 1, 0, 0);
+            else if (f == "w_oc") mat(lay.woc[l], d, d, d, 1, 0, 0);
+        }
+        return D;
+    }
+};
+
+namespace {
+
+#define CK(x)                                  \
+    do {                                       \
+        cudaError_t e__ = (x);                 \
+        if (e__ != cudaSuccess) return RLT_ECUDA; \
+    } while (0)
+
+// CK() with an optional timing bracket of the given kernel kind.
+#define CKP(kind, x)                                   \
+    do {                                               \
+        int p__ = m->prof.begin((kind), L.stream);     \
+        cudaError_t e__ = (x);                         \
+        m->prof.end(p__, L.stream);                    \
+        if (e__ != cudaSuccess) return RLT_ECUDA;      \
+    } while (0)
+
+size_t state_s_off() { return ALIGN; }
+size_t state_ring_off(const rlt_config& c, int B) { return align_up(ALIGN + (size_t)B * c.d * 4); }
+size_t ring_layer_elems(const rlt_config& c, int B) {
+    return (size_t)B * 2 * c.n_heads * (size_t)(c.W - 1) * c.head_dim;
+}
+
+struct EncWS {
+    size_t h, a, act, qkv, planes, att, ews, total;
+};
+EncWS enc_ws(const rlt_config& c, int B, int T) {
+    EncWS w;
+    size_t N = (size_t)B * T, d = c.d, e = c.dtype == RLT_BF16 ? 2 : 4;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes); return o; };
+    w.h = take(N * d * 4);
+    w.a = take(N * d * e);
+    w.act = take(N * (size_t)c.F * e);
+    w.qkv = take(N * 3 * d * 4);
+    w.planes = take(3 * N * d * e);
+    w.att = take(N * d * e);
+    w.ews = take(N * d * e);
+    w.total = off;
+    return w;
+}
+
+struct DecWS {
+    size_t x, A, qkv, att, qc, act, logits, part, total;
+};
+DecWS dec_ws(const rlt_config& c, int B) {
+    DecWS w;
+    size_t d = c.d, e = c.dtype == RLT_BF16 ? 2 : 4;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes); return o; };
+    w.x = take((size_t)B * d * 4);
+    w.A = take((size_t)B * 2 * d * e);
+    w.qkv = take((size_t)B * 3 * d * 4);
+    w.att = take((size_t)B * d * e);
+    w.qc = take((size_t)B * d * 4);
+    w.act = take((size_t)B * c.F * e);
+    w.logits = take((size_t)B * c.V * 4);
+    w.part = take((size_t)XATTN_PART_ITEMS * (c.head_dim + 2) * 4);
+    w.total = off;
+    return w;
+}
+
+int xattn_splits(const rlt_config& c, int B, int t) {
+    long long bh = (long long)B * c.n_heads;
+    long long want = (XATTN_TARGET_WARPS + bh - 1) / bh;
+    long long by_len = (t + XATTN_MIN_CHUNK - 1) / XATTN_MIN_CHUNK;
+    long long cap = XATTN_PART_ITEMS / bh;
+    long long s = want;
+    if (s > by_len) s = by_len;
+    if (s > XATTN_MAX_SPLITS) s = XATTN_MAX_SPLITS;
+    if (s > cap) s = cap;
+    return s < 1 ? 1 : (int)s;
+}
+
+// ------------------------------------------------------------------ encoder driver
+template <typename T>
+rlt_status encode_impl(rlt_model* m, const int32_t* tokens, int B, int Tn, int T_alloc, T* e, T* M,
+                       uint8_t* ws, cudaStream_t st) {
+    const rlt_config& c = m->cfg;
+    Launch L{st, &m->launches};
+    EncWS w = enc_ws(c, B, Tn);
+    int N = B * Tn, d = c.d, F = c.F, H = c.n_heads, hd = c.head_dim;
+    float* h = reinterpret_cast<float*>(ws + w.h);
+    T* a = reinterpret_cast<T*>(ws + w.a);
+    T* act = reinterpret_cast<T*>(ws + w.act);
+    float* qkv = reinterpret_cast<float*>(ws + w.qkv);
+    T* planes = reinterpret_cast<T*>(ws + w.planes);
+    T* att = reinterpret_cast<T*>(ws + w.att);
+    T* ews = reinterpret_cast<T*>(ws + w.ews);
+    const float2* rope = m->at<float2>(m->lay.rope);
+    CK(launch_embed<T>(L, tokens, N, m->at<T>(m->lay.embed), c.V, d, h, m->hdr()));
+    for (int l = 0; l < c.L_E; ++l) {
+        EpiArgs ea;
+        CK(launch_rmsnorm<T>(L, h, N, d, m->at<float>(m->lay.attn_norm[l]), c.rms_eps, a, d, N, N, nullptr));
+        ea.out_f32 = qkv; ea.ld_out = 3 * d;
+        CK(launch_gemm<T>(L, Epi::StoreF32, a, d, m->at<T>(m->lay.wqkv[l]), N, 3 * d, d, ea));
+        CK(launch_enc_qkv_layout<T>(L, qkv, B, Tn, H, hd, rope, planes));
+        CK(launch_enc_attention<T>(L, planes, att, B, Tn, H, hd));
+        ea = EpiArgs(); ea.out_f32 = h; ea.ld_out = d;
+        CK(launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.wo[l]), N, d, d, ea));
+        CK(launch_rmsnorm<T>(L, h, N, d, m->at<float>(m->lay.ffn_norm[l]), c.rms_eps, a, d, N, N, nullptr));
+        ea = EpiArgs(); ea.out_t = act; ea.ld_out = F;
+        CK(launch_gemm<T>(L, Epi::SwiGLU, a, d, m->at<T>(m->lay.wgu[l]), N, 2 * F, d, ea));
+        ea = EpiArgs(); ea.out_f32 = h; ea.ld_out = d;
+        CK(launch_gemm<T>(L, Epi::ResidAdd, act, F, m->at<T>(m->lay.wdown[l]), N, d, F, ea));
+    }
+    // e = RMSNorm(h) written with row capacity T_alloc, plus a contiguous copy for M
+    CK(launch_rmsnorm<T>(L, h, N, d, m->at<float>(m->lay.enc_norm), c.rms_eps, e, d, Tn, T_alloc, ews));
+    size_t group_elems = (size_t)2 * B * H * (size_t)T_alloc * hd;
+    for (int g = 0; g < c.G; ++g) {
+        EpiArgs ea;
+        ea.out_f32 = qkv; ea.ld_out = 2 * d;
+        CK(launch_gemm<T>(L, Epi::StoreF32, ews, d, m->at<T>(m->lay.mem) + (size_t)g * 2 * d * d, N, 2 * d, d, ea));
+        CK(launch_mem_layout<T>(L, qkv, B, Tn, T_alloc, H, hd, M + g * group_elems));
+    }
+    return RLT_OK;
+}
+
+// ------------------------------------------------------------------ one decoder step
+struct StepIO {
+    const int32_t* tok = nullptr;
+    int tok_stride = 1;
+    float* logp_tok = nullptr;
+    int lp_stride = 1;
+    float* lse = nullptr;
+    float* logp_full = nullptr;
+    float* score = nullptr;
+    const int32_t* prompt_len = nullptr;
+    float tau = 1.f;
+    bool head = true;
+};
+
+template <typename T>
+rlt_status step_impl(rlt_model* m, uint8_t* state, int B, const T* e, const T* M, int T_alloc, int t,
+                     const StepIO& io, uint8_t* ws, cudaStream_t st) {
+    const rlt_config& c = m->cfg;
+    Launch L{st, &m->launches};
+    DecWS w = dec_ws(c, B);
+    int d = c.d, F = c.F, H = c.n_heads, hd = c.head_dim;
+    StateHeader* sh = reinterpret_cast<StateHeader*>(state);
+    float* s = reinterpret_cast<float*>(state + state_s_off());
+    T* ring = reinterpret_cast<T*>(state + state_ring_off(c, B));
+    float* x = reinterpret_cast<float*>(ws + w.x);
+    T* A = reinterpret_cast<T*>(ws + w.A);
+    float* qkv = reinterpret_cast<float*>(ws + w.qkv);
+    T* att = reinterpret_cast<T*>(ws + w.att);
+    float* qc = reinterpret_cast<float*>(ws + w.qc);
+    T* act = reinterpret_cast<T*>(ws + w.act);
+    float* logits = reinterpret_cast<float*>(ws + w.logits);
+    float* part = reinterpret_cast<float*>(ws + w.part);
+    const float2* rope_row = m->at<float2>(m->lay.rope) + (size_t)(t - 1) * (hd / 2);
+    size_t group_elems = (size_t)2 * B * H * (size_t)T_alloc * hd;
+    int splits = xattn_splits(c, B, t);
+
+    // gated merge: x = e_t + sigmoid(W_ge e_t + W_gs s + b_g) * (W_fb s)
+    CKP(RLT_K_MERGE, launch_merge_prep<T>(L, e, T_alloc, t, s, A, B, d, sh, m->version, m->hdr()));
+    {
+        EpiArgs ea;
+        ea.out_f32 = x; ea.ld_out = d; ea.merge_e = A; ea.ld_e = 2 * d; ea.bias = m->at<float>(m->lay.merge_b);
+        CKP(RLT_K_MERGE, launch_gemm<T>(L, Epi::Merge, A, 2 * d, m->at<T>(m->lay.merge_w), B, 2 * d, 2 * d, ea));
+    }
+    for (int l = 0; l < c.L_D; ++l) {
+        EpiArgs ea;
+        // sliding-window self-attention (weights of encoder layer l)
+        CKP(RLT_K_NORM, launch_rmsnorm<T>(L, x, B, d, m->at<float>(m->lay.attn_norm[l]), c.rms_eps, A, d, B, B, nullptr));
+        ea.out_f32 = qkv; ea.ld_out = 3 * d;
+        CKP(RLT_K_QKV, launch_gemm<T>(L, Epi::StoreF32, A, d, m->at<T>(m->lay.wqkv[l]), B, 3 * d, d, ea));
+        CKP(RLT_K_SWA, launch_swa_decode<T>(L, qkv, rope_row, ring + (size_t)l * ring_layer_elems(c, B), att, B, H, hd,
+                                c.W, t));
+        ea = EpiArgs(); ea.out_f32 = x; ea.ld_out = d;
+        CKP(RLT_K_O, launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.wo[l]), B, d, d, ea));
+        // cross-attention to M_{<=t}
+        CKP(RLT_K_NORM, launch_rmsnorm<T>(L, x, B, d, m->at<float>(m->lay.xattn_norm[l]), c.rms_eps, A, d, B, B, nullptr));
+        ea = EpiArgs(); ea.out_f32 = qc; ea.ld_out = d;
+        CKP(RLT_K_QC, launch_gemm<T>(L, Epi::StoreF32, A, d, m->at<T>(m->lay.wqc[l]), B, d, d, ea));
+        const T* Mg = M + (c.G == 1 ? 0 : (size_t)l * group_elems);
+        CKP(RLT_K_XATTN, launch_xattn_decode<T>(L, qc, Mg, T_alloc, t, att, B, H, hd, splits, part));
+        ea = EpiArgs(); ea.out_f32 = x; ea.ld_out = d;
+        CKP(RLT_K_OC, launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.woc[l]), B, d, d, ea));
+        // SwiGLU FFN (weights of encoder layer l)
+        CKP(RLT_K_NORM, launch_rmsnorm<T>(L, x, B, d, m->at<float>(m->lay.ffn_norm[l]), c.rms_eps, A, d, B, B, nullptr));
+        ea = EpiArgs(); ea.out_t = act; ea.ld_out = F;
+        CKP(RLT_K_FFN_UP, launch_gemm<T>(L, Epi::SwiGLU, A, d, m->at<T>(m->lay.wgu[l]), B, 2 * F, d, ea));
+        ea = EpiArgs(); ea.out_f32 = x; ea.ld_out = d;
+        CKP(RLT_K_FFN_DOWN, launch_gemm<T>(L, Epi::ResidAdd, act, F, m->at<T>(m->lay.wdown[l]), B, d, F, ea));
+    }
+    // split: s_t = RMSNorm(x) becomes the state; the same s_t feeds the head
+    CKP(RLT_K_FINAL, launch_final_norm<T>(L, x, B, d, m->at<float>(m->lay.dec_norm), c.rms_eps, s, A, sh, t));
+    if (io.head) {
+        EpiArgs ea;
+        ea.out_f32 = logits; ea.ld_out = c.V;
+        CKP(RLT_K_HEAD, launch_gemm<T>(L, Epi::StoreF32, A, d, m->at<T>(m->lay.unembed), B, c.V, d, ea));
+        CKP(RLT_K_LSE, launch_lse_gather(L, logits, B, c.V, io.tau, io.tok, io.tok_stride, io.logp_tok, io.lp_stride,
+                             io.lse, io.logp_full, io.score, io.prompt_len, t, m->hdr()));
+    }
+    return RLT_OK;
+}
+
+template <typename T>
+rlt_status state_init_impl(rlt_model* m, uint8_t* state, int B, cudaStream_t st) {
+    Launch L{st, &m->launches};
+    CK(launch_state_init(L, m->at<float>(m->lay.s_star), B, m->cfg.d,
+                         reinterpret_cast<float*>(state + state_s_off()),
+                         reinterpret_cast<StateHeader*>(state), m->version));
+    return RLT_OK;
+}
+
+size_t replay_e_bytes(const rlt_config& c, int B, int T) {
+    return align_up((size_t)B * T * c.d * (c.dtype == RLT_BF16 ? 2 : 4));
+}
+size_t replay_M_bytes(const rlt_config& c, int B, int T) {
+    return align_up((size_t)c.G * 2 * B * (size_t)T * c.d * (c.dtype == RLT_BF16 ? 2 : 4));
+}
+
+}  // namespace
+
+// ====================================================================== public API
+
+extern "C" {
+
+const char* rlt_status_string(rlt_status s) {
+    switch (s) {
+        case RLT_OK: return "ok";
+        case RLT_EINVAL: return "invalid argument";
+        case RLT_ECUDA: return "CUDA error";
+        case RLT_ESTALE: return "state is stale (weights were replaced since it was built)";
+        case RLT_ETIMEOUT: return "device wait timed out";
+        case RLT_EUNSUPPORTED: return "unsupported shape";
+        case RLT_EDEVICE: return "device-side check failed";
+        case RLT_ESTATE: return "state not registered with this model or wrong batch";
+    }
+    return "unknown status";
+}
+
+size_t rlt_weights_bytes(const rlt_config* cfg) {
+    if (!cfg || !config_ok(*cfg)) return 0;
+    return make_layout(*cfg).total;
+}
+
+rlt_status rlt_model_create(const rlt_config* cfg, void* arena, size_t arena_bytes, void* stream,
+                            rlt_model** out) {
+    if (!cfg || !out || !arena || !config_ok(*cfg) || !aligned(arena)) return RLT_EINVAL;
+    Layout lay = make_layout(*cfg);
+    if (arena_bytes < lay.total) return RLT_EINVAL;
+    rlt_model* m = new rlt_model();
+    m->cfg = *cfg;
+    m->lay = lay;
+    m->arena = reinterpret_cast<uint8_t*>(arena);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(arena, 0, lay.total, st) != cudaSuccess ||
+        launch_rope_table(m->launch(stream), m->at<float2>(lay.rope), cfg->max_pos, cfg->head_dim,
+                          cfg->rope_base) != cudaSuccess) {
+        delete m;
+        return RLT_ECUDA;
+    }
+    const char* fixed[] = {"embed", "enc_norm", "mem_k", "mem_v", "merge_ge", "merge_gs", "merge_fb",
+                           "merge_bias", "s_star", "dec_norm", "unembed"};
+    for (const char* n : fixed) m->required.push_back(n);
+    const char* lf[] = {"attn_norm", "wq", "wk", "wv", "wo", "ffn_norm", "w_gate", "w_up", "w_down"};
+    for (int l = 0; l < cfg->L_E; ++l)
+        for (const char* f : lf) m->required.push_back("layers." + std::to_string(l) + "." + f);
+    const char* df[] = {"xattn_norm", "w_qc", "w_oc"};
+    for (int l = 0; l < cfg->L_D; ++l)
+        for (const char* f : df) m->required.push_back("dec." + std::to_string(l) + "." + f);
+    *out = m;
+    return RLT_OK;
+}
+
+void rlt_model_destroy(rlt_model* m) { delete m; }
+
+rlt_status rlt_model_set_weight(rlt_model* m, const char* name, const float* src, size_t numel, void* stream) {
+    if (!m || !name || !src || !aligned(src, 16)) return RLT_EINVAL;
+    std::string n(name);
+    Dest D = m->dest(n);
+    if (!D.ok || D.numel != numel) return RLT_EINVAL;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    Launch L = m->launch(stream);
+    if (D.vec) {
+        CK(cudaMemcpyAsync(m->arena + D.off, src, numel * 4, cudaMemcpyDeviceToDevice, st));
+    } else {
+        for (int g = 0; g < D.groups; ++g) {
+            const float* s = src + (size_t)g * D.rows * D.cols;
+            uint8_t* dst = m->arena + D.off + g * D.group_stride;
+            cudaError_t e = m->cfg.dtype == RLT_BF16
+                ? launch_pack_rows<bf16>(L, s, reinterpret_cast<bf16*>(dst), D.rows, D.cols, D.dst_ld,
+                                         D.row_mult, D.row_off, D.col_off)
+                : launch_pack_rows<float>(L, s, reinterpret_cast<float*>(dst), D.rows, D.cols, D.dst_ld,
+                                          D.row_mult, D.row_off, D.col_off);
+            CK(e);
+        }
+    }
+    m->loaded.insert(n);
+    return RLT_OK;
+}
+
+rlt_status rlt_model_commit(rlt_model* m) {
+    if (!m) return RLT_EINVAL;
+    for (const auto& n : m->required)
+        if (!m->loaded.count(n)) return RLT_EINVAL;
+    m->version += 1;
+    return RLT_OK;
+}
+
+uint64_t rlt_model_version(const rlt_model* m) { return m ? m->version : 0; }
+
+size_t rlt_encode_workspace_bytes(const rlt_model* m, int B, int T) {
+    if (!m || B < 1 || T < 1) return 0;
+    return enc_ws(m->cfg, B, T).total;
+}
+
+rlt_status rlt_encode(rlt_model* m, const int32_t* tokens, int B, int T, int T_alloc, void* e, void* M,
+                      void* ws, size_t ws_bytes, void* stream) {
+    if (!m || !tokens || !e || !M || !ws || B < 1 || T < 1 || T > T_alloc || T_alloc > m->cfg.max_pos)
+        return RLT_EINVAL;
+    if (m->version == 0) return RLT_EINVAL;
+    if (!aligned(e) || !aligned(M) || !aligned(ws) || !aligned(tokens, 4)) return RLT_EINVAL;
+    if (ws_bytes < enc_ws(m->cfg, B, T).total) return RLT_EINVAL;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* w = reinterpret_cast<uint8_t*>(ws);
+    int p = m->prof.begin(RLT_K_ENCODER, st);
+    rlt_status s = m->cfg.dtype == RLT_BF16
+        ? encode_impl<bf16>(m, tokens, B, T, T_alloc, (bf16*)e, (bf16*)M, w, st)
+        : encode_impl<float>(m, tokens, B, T, T_alloc, (float*)e, (float*)M, w, st);
+    m->prof.end(p, st);
+    return s;
+}
+
+size_t rlt_state_bytes(const rlt_model* m, int B) {
+    if (!m || B < 1) return 0;
+    const rlt_config& c = m->cfg;
+    return align_up(state_ring_off(c, B) + (size_t)c.L_D * ring_layer_elems(c, B) * m->lay.esz);
+}
+
+rlt_status rlt_state_init(rlt_model* m, void* state, int B, void* stream) {
+    if (!m || !state || B < 1 || !aligned(state)) return RLT_EINVAL;
+    if (m->version == 0) return RLT_EINVAL;
+    rlt_status s = m->cfg.dtype == RLT_BF16
+        ? state_init_impl<bf16>(m, (uint8_t*)state, B, (cudaStream_t)stream)
+        : state_init_impl<float>(m, (uint8_t*)state, B, (cudaStream_t)stream);
+    if (s != RLT_OK) return s;
+    m->states[state] = StateInfo{B, 0, m->version};
+    return RLT_OK;
+}
+
+rlt_status rlt_state_copy(rlt_model* m, void* dst, const void* src, void* stream) {
+    if (!m || !dst || !src || !aligned(dst)) return RLT_EINVAL;
+    auto it = m->states.find(src);
+    if (it == m->states.end()) return RLT_ESTATE;
+    StateInfo info = it->second;
+    CK(cudaMemcpyAsync(dst, src, rlt_state_bytes(m, info.B), cudaMemcpyDeviceToDevice,
+                       reinterpret_cast<cudaStream_t>(stream)));
+    m->states[dst] = info;
+    return RLT_OK;
+}
+
+rlt_status rlt_state_position(const rlt_model* m, const void* state, int64_t* t) {
+    if (!m || !state || !t) return RLT_EINVAL;
+    auto it = m->states.find(state);
+    if (it == m->states.end()) return RLT_ESTATE;
+    *t = it->second.t;
+    return RLT_OK;
+}
+
+rlt_status rlt_state_release(rlt_model* m, const void* state) {
+    if (!m || !state) return RLT_EINVAL;
+    return m->states.erase(state) ? RLT_OK : RLT_ESTATE;
+}
+
+size_t rlt_decode_workspace_bytes(const rlt_model* m, int B) {
+    if (!m || B < 1) return 0;
+    return dec_ws(m->cfg, B).total;
+}
+
+rlt_status rlt_decode_step(rlt_model* m, void* state, int B, const void* e, const void* M, int T_alloc,
+                           const int32_t* next_tok, float tau, float* logp_tok, float* lse, float* logp_full,
+                           void* ws, size_t ws_bytes, void* stream) {
+    if (!m || !state || !e || !M || !ws || B < 1 || !(tau > 0.f)) return RLT_EINVAL;
+    auto it = m->states.find(state);
+    if (it == m->states.end() || it->second.B != B) return RLT_ESTATE;
+    if (it->second.version != m->version) return RLT_ESTALE;
+    int64_t t = it->second.t + 1;
+    if (t > T_alloc || T_alloc > m->cfg.max_pos) return RLT_EINVAL;
+    if (!aligned(e) || !aligned(M) || !aligned(ws)) return RLT_EINVAL;
+    if (ws_bytes < dec_ws(m->cfg, B).total) return RLT_EINVAL;
+    if ((next_tok && !aligned(next_tok, 4)) || (logp_tok && !aligned(logp_tok, 4)) ||
+        (lse && !aligned(lse, 4)) || (logp_full && !aligned(logp_full, 4)))
+        return RLT_EINVAL;
+    StepIO io;
+    io.tok = next_tok; io.logp_tok = next_tok ? logp_tok : nullptr; io.lse = lse; io.logp_full = logp_full;
+    io.tau = tau;
+    io.head = (next_tok && logp_tok) || lse || logp_full;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    rlt_status s = m->cfg.dtype == RLT_BF16
+        ? step_impl<bf16>(m, (uint8_t*)state, B, (const bf16*)e, (const bf16*)M, T_alloc, (int)t, io,
+                          (uint8_t*)ws, st)
+        : step_impl<float>(m, (uint8_t*)state, B, (const float*)e, (const float*)M, T_alloc, (int)t, io,
+                           (uint8_t*)ws, st);
+    if (s == RLT_OK) it->second.t = t;
+    return s;
+}
+
+size_t rlt_replay_workspace_bytes(const rlt_model* m, int B, int T) {
+    if (!m || B < 1 || T < 1) return 0;
+    const rlt_config& c = m->cfg;
+    size_t enc = enc_ws(c, B, T).total, dec = dec_ws(c, B).total;
+    return replay_e_bytes(c, B, T) + replay_M_bytes(c, B, T) + rlt_state_bytes(m, B) + (enc > dec ? enc : dec);
+}
+
+rlt_status rlt_replay(rlt_model* m, const int32_t* tokens, int B, int T, const int32_t* prompt_len, float tau,
+                      float* score, float* logp_tok, void* final_state, void* ws, size_t ws_bytes, void* stream) {
+    if (!m || !tokens || !prompt_len || !score || !ws || B < 1 || T < 1 || !(tau > 0.f)) return RLT_EINVAL;
+    if (m->version == 0 || T > m->cfg.max_pos) return RLT_EINVAL;
+    if (!aligned(ws) || !aligned(tokens, 4) || !aligned(prompt_len, 4) || !aligned(score, 4) ||
+        (logp_tok && !aligned(logp_tok, 4)) || (final_state && !aligned(final_state)))
+        return RLT_EINVAL;
+    if (ws_bytes < rlt_replay_workspace_bytes(m, B, T)) return RLT_EINVAL;
+    const rlt_config& c = m->cfg;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* w = reinterpret_cast<uint8_t*>(ws);
+    uint8_t* e = w;
+    uint8_t* M = e + replay_e_bytes(c, B, T);
+    uint8_t* own_state = M + replay_M_bytes(c, B, T);
+    uint8_t* scratch = own_state + rlt_state_bytes(m, B);
+    uint8_t* state = final_state ? reinterpret_cast<uint8_t*>(final_state) : own_state;
+    bool bf = c.dtype == RLT_BF16;
+    int p = m->prof.begin(RLT_K_ENCODER, st);
+    rlt_status s = bf ? encode_impl<bf16>(m, tokens, B, T, T, (bf16*)e, (bf16*)M, scratch, st)
+                      : encode_impl<float>(m, tokens, B, T, T, (float*)e, (float*)M, scratch, st);
+    m->prof.end(p, st);
+    if (s != RLT_OK) return s;
+    s = bf ? state_init_impl<bf16>(m, state, B, st) : state_init_impl<float>(m, state, B, st);
+    if (s != RLT_OK) return s;
+    CK(cudaMemsetAsync(score, 0, (size_t)B * 4, st));
+    if (logp_tok) CK(cudaMemsetAsync(logp_tok, 0, (size_t)B * T * 4, st));
+    for (int t = 1; t <= T; ++t) {
+        StepIO io;
+        io.tau = tau;
+        io.head = t < T;
+        if (t < T) {
+            io.tok = tokens + t;          // x_{t+1} is column t (0-based) of row b
+            io.tok_stride = T;
+            io.logp_tok = logp_tok ? logp_tok + (t - 1) : nullptr;
+            io.lp_stride = T;
+            io.score = score;
+            io.prompt_len = prompt_len;
+        }
+        s = bf ? step_impl<bf16>(m, state, B, (const bf16*)e, (const bf16*)M, T, t, io, scratch, st)
+               : step_impl<float>(m, state, B, (const float*)e, (const float*)M, T, t, io, scratch, st);
+        if (s != RLT_OK) return s;
+    }
+    if (final_state) m->states[final_state] = StateInfo{B, T, m->version};
+    return RLT_OK;
+}
+
+rlt_status rlt_last_error(rlt_model* m, void* stream) {
+    if (!m) return RLT_EINVAL;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return RLT_ECUDA;
+    uint32_t flags = 0;
+    if (cudaMemcpy(&flags, &m->hdr()->err_flags, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return RLT_ECUDA;
+    if (flags) {
+        uint32_t zero = 0;
+        if (cudaMemcpy(&m->hdr()->err_flags, &zero, 4, cudaMemcpyHostToDevice) != cudaSuccess) return RLT_ECUDA;
+    }
+    if (flags & ERR_TIMEOUT) return RLT_ETIMEOUT;
+    if (flags) return RLT_EDEVICE;
+    return RLT_OK;
+}
+
+uint64_t rlt_launch_count(const rlt_model* m) { return m ? m->launches : 0; }
+
+rlt_status rlt_profile_start(rlt_model* m, uint32_t kind_mask) {
+    if (!m) return RLT_EINVAL;
+    m->prof.on = true;
+    m->prof.mask = kind_mask;
+    m->prof.used = 0;
+    m->prof.recs.clear();
+    return RLT_OK;
+}
+
+rlt_status rlt_profile_stop(rlt_model* m, double* ms, uint64_t* launches) {
+    if (!m) return RLT_EINVAL;
+    Profiler& P = m->prof;
+    P.on = false;
+    if (ms) for (int k = 0; k < RLT_K_COUNT; ++k) ms[k] = 0.0;
+    if (launches) for (int k = 0; k < RLT_K_COUNT; ++k) launches[k] = 0;
+    if (P.used && cudaEventSynchronize(P.pool[P.used - 1]) != cudaSuccess) return RLT_ECUDA;
+    for (const auto& r : P.recs) {
+        float e = 0.f;
+        if (cudaEventElapsedTime(&e, P.pool[r.second], P.pool[r.second + 1]) != cudaSuccess) return RLT_ECUDA;
+        if (ms) ms[r.first] += e;
+        if (launches) launches[r.first] += 1;
+    }
+    P.recs.clear();
+    P.used = 0;
+    return RLT_OK;
+}
+
+}  // extern "C"

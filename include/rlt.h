@@ -1,0 +1,244 @@
+/*
+ * rlt.h -- C ABI of the Recurrent Looped Transformer (RLT) decoder-transition library
+ * for NVIDIA B200 (sm_100a).
+ *
+ * What it computes.  The RLT pairs a causal encoder with a recurrent decoder
+ * ("普林斯顿提出 RLT：跨 Token 携带解码器状态的循环 Transformer", news summary:
+ * the encoder/memory paragraph and the decoder-state paragraph):
+ *
+ *   encoder     e_t = causal encoder output at position t, M_{<=t} = key/value memory
+ *               projected from e (G = 1 group shared by all decoder layers, or G = L_D);
+ *   state       H_t = (s_t, C_t^D): s_t the normalised final decoder output, C_t^D the
+ *               per-layer sliding-window (SWA) key/value cache holding W-1 entries;
+ *               H_0 = (s*, empty);
+ *   transition  x = e_t + sigmoid(W_ge e_t + W_gs s_{t-1} + b_g) * (W_fb s_{t-1})
+ *               then L_D blocks of [SWA over cache + current token, cross-attention to
+ *               M_{<=t}, SwiGLU FFN], decoder SWA/FFN weights tied to encoder layer l
+ *               (news summary, weight-tying paragraph); s_t = RMSNorm(x);
+ *               logp_t = log_softmax(W_U s_t / tau) predicts x_{t+1};
+ *   replay      exact current-policy replay: rebuild M, every SWA cache and s from the
+ *               sequence start under the current weights, then score the response
+ *               tokens (news summary, model-RL co-design principle; alphalab review,
+ *               section 4).
+ *
+ * Conventions shared by every entry point.
+ *   - Every device buffer is owned by the caller.  The library never allocates device
+ *     memory: sizes come from the *_bytes() queries, the caller allocates and passes
+ *     pointers.  Device buffers must be 256-byte aligned unless stated otherwise.
+ *   - Calls are asynchronous on the given stream (a cudaStream_t passed as void*; NULL
+ *     is the legacy default stream).  Argument errors are detected on the host before
+ *     anything is launched and returned synchronously; nothing is then modified.
+ *   - Device-side checks (token id out of range, a state that does not match its
+ *     registered position) latch a flag in the model's device header; the next
+ *     rlt_last_error() call reports and clears it.
+ *   - A model handle is not re-entrant: calls on one handle must be serialised by the
+ *     caller.  Distinct handles are independent.
+ *   - dtype RLT_F32 stores weights, e, M and the SWA cache in float32; RLT_BF16 stores
+ *     them in bfloat16 (round to nearest even) and accumulates in float32.  The
+ *     residual stream, s_t, softmax statistics and log-probabilities are float32 in
+ *     both modes.
+ */
+#ifndef RLT_H
+#define RLT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RLT_OK = 0,
+    RLT_EINVAL = 1,        /* invalid argument: NULL, size, alignment, unknown name      */
+    RLT_ECUDA = 2,         /* a CUDA runtime call or kernel launch failed                */
+    RLT_ESTALE = 3,        /* state was built under weights that have since been replaced */
+    RLT_ETIMEOUT = 4,      /* a device-side bounded wait gave up                         */
+    RLT_EUNSUPPORTED = 5,  /* shape outside what the kernels implement                   */
+    RLT_EDEVICE = 6,       /* a device-side check failed (see rlt_last_error)            */
+    RLT_ESTATE = 7         /* state pointer not registered with this model / wrong batch */
+} rlt_status;
+
+enum { RLT_F32 = 0, RLT_BF16 = 1 };
+
+/* Model shape.  head_dim must be 16, 32, 64 or 128 and n_heads * head_dim == d;
+ * d, F and V multiples of 8; G is 1 or L_D; L_E == L_D (tied weights); W >= 1.
+ * max_pos is the largest sequence length any call will use (sizes the rotary table). */
+typedef struct {
+    int32_t V, d, n_heads, head_dim, L_E, L_D, F, W, G;
+    int32_t dtype;          /* RLT_F32 or RLT_BF16 */
+    float rms_eps;          /* RMSNorm epsilon (1e-6 in the workloads)        */
+    float rope_base;        /* rotary base (10000)                            */
+    int32_t max_pos;        /* positions 0 .. max_pos-1 are supported         */
+} rlt_config;
+
+typedef struct rlt_model rlt_model;
+
+/* Human-readable name of a status code (static string). */
+const char* rlt_status_string(rlt_status s);
+
+/* Bytes of device memory the model's weight arena needs (library layout, plus a small
+ * header and the rotary table).  Returns 0 for an invalid config. */
+size_t rlt_weights_bytes(const rlt_config* cfg);
+
+/* Create a model handle over a caller-owned device arena of at least
+ * rlt_weights_bytes(cfg) bytes.  The arena must stay allocated until
+ * rlt_model_destroy.  Fills the rotary table and clears the device header on
+ * `stream`.  Errors: RLT_EINVAL (bad config, NULL, small or misaligned arena),
+ * RLT_ECUDA. */
+rlt_status rlt_model_create(const rlt_config* cfg, void* arena, size_t arena_bytes,
+                            void* stream, rlt_model** out);
+
+/* Release the host handle (the arena stays the caller's). */
+void rlt_model_destroy(rlt_model* m);
+
+/* Copy one weight tensor into the arena, converting it to the library layout and dtype.
+ * `name` is a canonical name (the layout is [out, in] for a linear map y = x W^T):
+ *   "embed" [V,d]; "layers.<l>.attn_norm" [d]; "layers.<l>.wq|wk|wv|wo" [d,d];
+ *   "layers.<l>.ffn_norm" [d]; "layers.<l>.w_gate|w_up" [F,d]; "layers.<l>.w_down" [d,F];
+ *   "enc_norm" [d]; "mem_k", "mem_v" [G,d,d]; "dec.<l>.xattn_norm" [d];
+ *   "dec.<l>.w_qc|w_oc" [d,d]; "merge_ge|merge_gs|merge_fb" [d,d]; "merge_bias" [d];
+ *   "s_star" [d]; "dec_norm" [d]; "unembed" [V,d].
+ * `src` is a device float32 array of `numel` elements, contiguous, read on `stream`.
+ * Errors: RLT_EINVAL (unknown name, wrong numel, NULL), RLT_ECUDA. */
+rlt_status rlt_model_set_weight(rlt_model* m, const char* name, const float* src,
+                                size_t numel, void* stream);
+
+/* Declare the weights complete: fails with RLT_EINVAL if any tensor was never set.
+ * Every commit starts a new model version; states initialised earlier become stale
+ * (a weight update invalidates old states: news summary, multi-turn paragraph). */
+rlt_status rlt_model_commit(rlt_model* m);
+
+/* Current model version (0 before the first commit). */
+uint64_t rlt_model_version(const rlt_model* m);
+
+/* ---------------------------------------------------------------- encoder */
+
+/* Workspace bytes rlt_encode needs for B sequences of T tokens. */
+size_t rlt_encode_workspace_bytes(const rlt_model* m, int B, int T);
+
+/* Causal, token-parallel encoder (news summary, encoder paragraph; the model-hardware
+ * principle: known tokens are encoded token-parallel).
+ *   tokens  device int32 [B, T] row-major, ids in [0, V)
+ *   e       device out [B, T_alloc, d] (dtype of the model); rows 0..T-1 written
+ *   M       device out [G, 2, B, n_heads, T_alloc, head_dim]: plane 0 keys, plane 1
+ *           values, head-major so that one head's memory is contiguous; positions
+ *           0..T-1 written
+ *   ws      device workspace of at least rlt_encode_workspace_bytes(m, B, T) bytes
+ * Requires 1 <= T <= T_alloc <= max_pos.  Out-of-range token ids latch RLT_EDEVICE
+ * (their rows read id 0).  Errors: RLT_EINVAL, RLT_ECUDA. */
+rlt_status rlt_encode(rlt_model* m, const int32_t* tokens, int B, int T, int T_alloc,
+                      void* e, void* M, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------- decoder state */
+
+/* Bytes of one decoder state H for B sequences: a 256-byte header, s [B, d] float32 and
+ * the SWA ring cache [L_D, B, 2, n_heads, W-1, head_dim] (model dtype). */
+size_t rlt_state_bytes(const rlt_model* m, int B);
+
+/* H_0 = (s*, empty cache) at position t = 0 for B sequences (news summary,
+ * decoder-state paragraph: initialisation runs once before BOS with the learned start
+ * state and an empty cache).  Registers the state with the model and stamps it with
+ * the current model version.  Errors: RLT_EINVAL, RLT_ECUDA. */
+rlt_status rlt_state_init(rlt_model* m, void* state, int B, void* stream);
+
+/* Copy a registered state (a prefix snapshot) to another caller buffer of the same size
+ * and register the copy at the same position and version. */
+rlt_status rlt_state_copy(rlt_model* m, void* dst, const void* src, void* stream);
+
+/* Position t (tokens consumed) of a registered state, from the host-side registry. */
+rlt_status rlt_state_position(const rlt_model* m, const void* state, int64_t* t);
+
+/* Forget a state (it may then be freed by the caller). */
+rlt_status rlt_state_release(rlt_model* m, const void* state);
+
+/* ---------------------------------------------------------------- one decoder step */
+
+/* Workspace bytes one rlt_decode_step needs for B sequences. */
+size_t rlt_decode_workspace_bytes(const rlt_model* m, int B);
+
+/* One recurrent transition H_{t-1}, e_t -> H_t for all B sequences in lockstep (the
+ * decoder-state paragraph of the news summary; deepsonar teardown, sections 2.3-2.4).
+ *   state      registered state holding H_{t-1}; overwritten in place with H_t
+ *   e, M       encoder outputs as written by rlt_encode with row capacity T_alloc;
+ *              position t-1 (0-based) of e and positions 0..t-1 of M are read
+ *   next_tok   device int32 [B] or NULL: the token x_{t+1} whose log-probability is
+ *              gathered into logp_tok
+ *   tau        temperature > 0 of the next-token distribution
+ *   logp_tok   device float [B] or NULL: log p(next_tok | x_{<=t}) at temperature tau
+ *   lse        device float [B] or NULL: log-sum-exp of W_U s_t / tau
+ *   logp_full  device float [B, V] or NULL: the full log-probability row
+ *   ws         workspace of at least rlt_decode_workspace_bytes(m, B) bytes
+ * The step reads its position from the registry; t = position + 1 must satisfy
+ * t <= T_alloc <= max_pos.  Errors: RLT_ESTATE (unknown state or B mismatch),
+ * RLT_ESTALE (state older than the current weights), RLT_EINVAL, RLT_ECUDA. */
+rlt_status rlt_decode_step(rlt_model* m, void* state, int B, const void* e, const void* M,
+                           int T_alloc, const int32_t* next_tok, float tau, float* logp_tok,
+                           float* lse, float* logp_full, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* ---------------------------------------------------------------- exact replay */
+
+/* Workspace bytes rlt_replay needs for B sequences of T tokens (e, M, a state and the
+ * step workspace). */
+size_t rlt_replay_workspace_bytes(const rlt_model* m, int B, int T);
+
+/* Exact current-policy replay (news summary, model-RL co-design principle; alphalab
+ * review, section 4): encode the whole sequence, start from H_0 = (s*, empty) and step
+ * through every token -- prompt and response alike, with no reset at the boundary --
+ * then score the response.
+ *   tokens      device int32 [B, T]
+ *   prompt_len  device int32 [B], 1 <= P_b <= T: tokens x_1..x_P are the prompt
+ *   score       device float out [B]: sum_{t=P_b}^{T-1} log p(x_{t+1} | x_{<=t}) at tau
+ *   logp_tok    device float out [B, T] or NULL: entry t-1 = log p(x_{t+1} | x_{<=t})
+ *               for t = 1..T-1, entry T-1 = 0
+ *   final_state caller buffer of rlt_state_bytes(m, B) or NULL: receives H_T and is
+ *               registered at position T
+ * Errors: RLT_EINVAL, RLT_ECUDA; bad token ids latch RLT_EDEVICE. */
+rlt_status rlt_replay(rlt_model* m, const int32_t* tokens, int B, int T,
+                      const int32_t* prompt_len, float tau, float* score, float* logp_tok,
+                      void* final_state, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, then return and clear the device-side error flags:
+ * RLT_OK, RLT_EDEVICE (bad token id or state/registry mismatch) or RLT_ETIMEOUT. */
+rlt_status rlt_last_error(rlt_model* m, void* stream);
+
+/* Number of kernels the library has launched since the model was created (all entry
+ * points).  Used by benchmarks to count launches inside a timed region. */
+uint64_t rlt_launch_count(const rlt_model* m);
+
+/* ---------------------------------------------------------------- kernel timing */
+
+/* Kernel kinds of the decoder step (and the encoder as one kind) for live timing. */
+enum {
+    RLT_K_NORM = 0,      /* pre-norm RMSNorm of a sublayer                              */
+    RLT_K_MERGE = 1,     /* merge input assembly + gated-merge GEMM                      */
+    RLT_K_QKV = 2,       /* self-attention q/k/v projection                              */
+    RLT_K_SWA = 3,       /* sliding-window attention over the ring cache (+ ring write)  */
+    RLT_K_O = 4,         /* self-attention output projection + residual                  */
+    RLT_K_QC = 5,        /* cross-attention query projection                             */
+    RLT_K_XATTN = 6,     /* cross-attention over M_{<=t} (key splits and their combine)  */
+    RLT_K_OC = 7,        /* cross-attention output projection + residual                 */
+    RLT_K_FFN_UP = 8,    /* SwiGLU gate/up projection                                    */
+    RLT_K_FFN_DOWN = 9,  /* SwiGLU down projection + residual                            */
+    RLT_K_FINAL = 10,    /* final RMSNorm: s_t                                           */
+    RLT_K_HEAD = 11,     /* LM-head projection                                           */
+    RLT_K_LSE = 12,      /* log-sum-exp + gather + score                                 */
+    RLT_K_ENCODER = 13,  /* a whole rlt_encode call                                      */
+    RLT_K_COUNT = 14
+};
+
+/* Start recording a CUDA event pair on the launch stream around every launch of the kinds
+ * in `kind_mask` (bit i = kind i).  Timing adds two event records per bracketed launch. */
+rlt_status rlt_profile_start(rlt_model* m, uint32_t kind_mask);
+
+/* Stop recording; wait for the recorded events and write, per kind, the summed elapsed
+ * milliseconds (ms[RLT_K_COUNT]) and the number of bracketed launches
+ * (launches[RLT_K_COUNT]).  Either array may be NULL. */
+rlt_status rlt_profile_stop(rlt_model* m, double* ms, uint64_t* launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RLT_H */
