@@ -89,17 +89,30 @@ __global__ void __launch_bounds__(256) k_gemm_simt(const T* __restrict__ A, int 
 }  // namespace
 
 template <typename T>
-cudaError_t launch_gemm(Launch L, Epi epi, const T* A, int lda, const T* W, int M, int N, int K,
-                        const EpiArgs& ea) {
+cudaError_t launch_gemm_simt(Launch L, Epi epi, const T* A, int lda, const T* W, int M, int N, int K,
+                             const EpiArgs& ea) {
     dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
     k_gemm_simt<T><<<grid, 256, 0, L.stream>>>(A, lda, W, M, N, K, epi, ea);
     *L.count += 1;
     return cudaGetLastError();
 }
 
-template cudaError_t launch_gemm<float>(Launch, Epi, const float*, int, const float*, int, int, int,
-                                        const EpiArgs&);
-template cudaError_t launch_gemm<bf16>(Launch, Epi, const bf16*, int, const bf16*, int, int, int,
-                                       const EpiArgs&);
+template <>
+cudaError_t launch_gemm<float>(Launch L, Epi epi, const float* A, int lda, const float* W, int M, int N, int K,
+                               const EpiArgs& ea) {
+    return launch_gemm_simt<float>(L, epi, A, lda, W, M, N, K, ea);
+}
+
+template <>
+cudaError_t launch_gemm<bf16>(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
+                              const EpiArgs& ea) {
+    if (gemm_tc_supported(A, lda, W, K)) return launch_gemm_tc(L, epi, A, lda, W, M, N, K, ea, ea.hdr);
+    return launch_gemm_simt<bf16>(L, epi, A, lda, W, M, N, K, ea);
+}
+
+template cudaError_t launch_gemm_simt<float>(Launch, Epi, const float*, int, const float*, int, int, int,
+                                             const EpiArgs&);
+template cudaError_t launch_gemm_simt<bf16>(Launch, Epi, const bf16*, int, const bf16*, int, int, int,
+                                            const EpiArgs&);
 
 }  // namespace rlt

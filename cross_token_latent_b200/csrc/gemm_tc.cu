@@ -1,0 +1,333 @@
+// Tensor-core GEMM for sm_100a: C[M, N] = A[M, K] x W[N, K]^T with bf16 operands, float32
+// accumulation in tensor memory (TMEM) and the fused epilogues of the RLT path.
+//
+// One CTA computes one 128 x BN output tile with 4 warps:
+//   warp 0, lane 0  TMA producer: 2-D tiled loads (128-byte swizzle) of A and W k-blocks of
+//                   64 elements into a ring of STAGES shared-memory slots (mbarrier full[s]);
+//   warp 1, lane 0  MMA issuer: four tcgen05.mma (M=128, N=BN, K=16) per k-block into the
+//                   TMEM accumulator; tcgen05.commit frees the slot (empty[s]) and, after
+//                   the last block, signals the epilogue (done);
+//   warp 2          allocates / frees the TMEM columns;
+//   all 4 warps     epilogue: warp w reads TMEM lanes 32w..32w+31 (one output row per
+//                   thread) with tcgen05.ld and applies the fused epilogue.
+// No multicast is used anywhere.  Every mbarrier wait is bounded by %globaltimer; on
+// expiry the CTA raises ERR_TIMEOUT, stops issuing work, frees its TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "kernels.cuh"
+
+namespace rlt {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;                       // 64 bf16 = 128 bytes = one swizzle row
+constexpr int A_BYTES = BM * BK * 2;         // 16 KB
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait for the phase with the given parity.  False on timeout or abort.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    if (mbar_try(bar, parity)) return true;
+    uint64_t t0 = globaltimer();
+    while (true) {
+        if (mbar_try(bar, parity)) return true;
+        if (*abort) return false;
+        if (globaltimer() - t0 > WAIT_LIMIT_NS) return false;
+    }
+}
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major operand tile in the 128-byte swizzle layout that
+// TMA writes (8-row groups of 1024 bytes).  Fields: start address >> 4 [0,14), leading byte
+// offset >> 4 [16,30) (unused for this layout), stride byte offset >> 4 [32,46) = 1024 B
+// between 8-row groups, descriptor version 1 [46,48), layout 2 = 128-byte swizzle [61,64).
+__device__ __forceinline__ uint64_t sdesc_sw128(const void* tile) {
+    uint64_t a = smem_u32(tile);
+    return ((a >> 4) & 0x3FFFull) | (1ull << 16) | ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+// Instruction descriptor of kind::f16: D float32 [4,6)=1, A bf16 [7,10)=1, B bf16 [10,13)=1,
+// both K-major, N >> 3 at [17,23), M >> 4 at [24,29).
+__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Fused epilogue on 16 consecutive columns n..n+15 of row m (cnt of them inside N).
+__device__ __forceinline__ void epilogue16(Epi epi, const EpiArgs& ea, int m, int n, int cnt, const float* v) {
+    switch (epi) {
+        case Epi::StoreF32: {
+            float* o = ea.out_f32 + (long long)m * ea.ld_out + n;
+            if (cnt == 16) {
+#pragma unroll
+                for (int j = 0; j < 16; j += 4)
+                    *reinterpret_cast<float4*>(o + j) =
+                        make_float4(v[j] * ea.scale, v[j + 1] * ea.scale, v[j + 2] * ea.scale, v[j + 3] * ea.scale);
+            } else {
+                for (int j = 0; j < cnt; ++j) o[j] = v[j] * ea.scale;
+            }
+            break;
+        }
+        case Epi::ResidAdd: {
+            float* o = ea.out_f32 + (long long)m * ea.ld_out + n;
+            if (cnt == 16) {
+#pragma unroll
+                for (int j = 0; j < 16; j += 4) {
+                    float4 x = *reinterpret_cast<float4*>(o + j);
+                    x.x += v[j]; x.y += v[j + 1]; x.z += v[j + 2]; x.w += v[j + 3];
+                    *reinterpret_cast<float4*>(o + j) = x;
+                }
+            } else {
+                for (int j = 0; j < cnt; ++j) o[j] += v[j];
+            }
+            break;
+        }
+        case Epi::SwiGLU: {     // columns 2j = gate_j, 2j+1 = up_j
+            bf16* o = reinterpret_cast<bf16*>(ea.out_t) + (long long)m * ea.ld_out + n / 2;
+            if (cnt == 16) {
+                float h[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) h[j] = siluf_(v[2 * j]) * v[2 * j + 1];
+                st16(o, Vec16<bf16>::pack(h));
+            } else {
+                for (int j = 0; j + 1 < cnt; j += 2) o[j / 2] = __float2bfloat16_rn(siluf_(v[j]) * v[j + 1]);
+            }
+            break;
+        }
+        case Epi::Merge: {      // columns 2j = gate pre-activation, 2j+1 = feedback projection
+            const bf16* e = reinterpret_cast<const bf16*>(ea.merge_e) + (long long)m * ea.ld_e;
+            float* o = ea.out_f32 + (long long)m * ea.ld_out;
+            for (int j = 0; j + 1 < cnt; j += 2) {
+                int c = (n + j) / 2;
+                o[c] = __bfloat162float(e[c]) + sigmoidf_(v[j] + ea.bias[c]) * v[j + 1];
+            }
+            break;
+        }
+    }
+}
+
+template <int BN, int STAGES>
+struct TcShape {
+    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int TMEM_COLS = BN < 32 ? 32 : BN;
+    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
+};
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(128, 1)
+k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW, int M, int N, int K,
+          Epi epi, EpiArgs ea, DevHeader* hdr) {
+    using S = TcShape<BN, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES);
+    uint64_t* empty = full + STAGES;
+    uint64_t* done = empty + STAGES;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    __shared__ int abort_flag;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+    const int nkb = (K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(done, 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 2) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(S::TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0 && lane == 0) {
+        // TMA producer
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&tmW) : "memory");
+        for (int kb = 0; kb < nkb; ++kb) {
+            int s = kb % STAGES;
+            uint32_t ph = (kb / STAGES) & 1;
+            if (!mbar_wait(&empty[s], ph ^ 1, &abort_flag)) { abort_flag = 1; break; }
+            uint8_t* a = smem + s * S::STAGE_BYTES;
+            mbar_expect_tx(&full[s], S::STAGE_BYTES);
+            tma_load_2d(a, &tmA, &full[s], kb * BK, m0);
+            tma_load_2d(a + A_BYTES, &tmW, &full[s], kb * BK, n0);
+        }
+    } else if (warp == 1 && lane == 0) {
+        // MMA issuer
+        constexpr uint32_t idesc = idesc_bf16(BM, BN);
+        for (int kb = 0; kb < nkb; ++kb) {
+            int s = kb % STAGES;
+            uint32_t ph = (kb / STAGES) & 1;
+            if (!mbar_wait(&full[s], ph, &abort_flag)) { abort_flag = 1; break; }
+            tc_fence_after();
+            uint8_t* a = smem + s * S::STAGE_BYTES;
+            uint64_t da = sdesc_sw128(a), dw = sdesc_sw128(a + A_BYTES);
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k)      // advance 16 elements = 32 bytes = 2 in (addr >> 4)
+                umma(tmem, da + 2 * k, dw + 2 * k, idesc, (kb | k) != 0);
+            umma_commit(&empty[s]);
+        }
+        umma_commit(done);
+    }
+    __syncwarp();
+
+    // epilogue: thread owns output row m0 + 32*warp + lane
+    bool ok = mbar_wait(done, 0, &abort_flag);
+    ok = __all_sync(0xffffffffu, ok);
+    tc_fence_after();
+    if (ok) {
+        const int m = m0 + warp * 32 + lane;
+        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+            float v[16];
+            tmem_ld16(lane_base + c, v);
+            int n = n0 + c;
+            if (m < M && n < N) epilogue16(epi, ea, m, n, min(16, N - n), v);
+        }
+    } else if (lane == 0) {
+        abort_flag = 1;
+        raise_flag(hdr, ERR_TIMEOUT);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(S::TMEM_COLS));
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void* p = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D bf16 tensor [rows, cols] with leading dimension ld (elements), box of BK x box_rows.
+bool make_map(CUtensorMap* map, const void* ptr, int rows, int cols, int ld, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int BN, int STAGES>
+cudaError_t run_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K, const EpiArgs& ea,
+                   DevHeader* hdr) {
+    using S = TcShape<BN, STAGES>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    CUtensorMap ta, tw;
+    if (!make_map(&ta, A, M, K, lda, BM) || !make_map(&tw, W, N, K, K, BN)) return cudaErrorInvalidValue;
+    dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
+    k_gemm_tc<BN, STAGES><<<grid, 128, S::SMEM, L.stream>>>(ta, tw, M, N, K, epi, ea, hdr);
+    *L.count += 1;
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool gemm_tc_supported(const void* A, int lda, const void* W, int K) {
+    // TMA: 16-byte aligned base addresses and row pitches
+    return (reinterpret_cast<uintptr_t>(A) % 16 == 0) && (reinterpret_cast<uintptr_t>(W) % 16 == 0) &&
+           (lda % 8 == 0) && (K % 8 == 0) && encode_fn() != nullptr;
+}
+
+cudaError_t launch_gemm_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
+                           const EpiArgs& ea, DevHeader* hdr) {
+    // Pick the widest tile that still gives at least one wave of CTAs over the 148 SMs.
+    long long mt = (M + BM - 1) / BM;
+    auto tiles = [&](int bn) { return mt * ((N + bn - 1) / bn); };
+    if (tiles(128) >= 148) return run_tc<128, 4>(L, epi, A, lda, W, M, N, K, ea, hdr);
+    if (tiles(64) >= 148) return run_tc<64, 6>(L, epi, A, lda, W, M, N, K, ea, hdr);
+    return run_tc<32, 8>(L, epi, A, lda, W, M, N, K, ea, hdr);
+}
+
+}  // namespace rlt

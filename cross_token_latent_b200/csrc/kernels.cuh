@@ -65,10 +65,21 @@ struct EpiArgs {
     const void* merge_e = nullptr;  // Merge: e_t rows (storage type), leading dim ld_e
     int ld_e = 0;
     const float* bias = nullptr;    // Merge: gate bias b_g
+    DevHeader* hdr = nullptr;       // error flags (tensor-core path: bounded-wait timeouts)
 };
+// Dispatch: bf16 operands go to the tcgen05 kernel (gemm_tc.cu) when TMA can address them,
+// otherwise (and for float32 models) to the CUDA-core kernel.
 template <typename T>
 cudaError_t launch_gemm(Launch L, Epi epi, const T* A, int lda, const T* W, int M, int N, int K,
                         const EpiArgs& ea);
+template <typename T>
+cudaError_t launch_gemm_simt(Launch L, Epi epi, const T* A, int lda, const T* W, int M, int N, int K,
+                             const EpiArgs& ea);
+
+// ------------------------------------------------------------------ gemm_tc.cu
+bool gemm_tc_supported(const void* A, int lda, const void* W, int K);
+cudaError_t launch_gemm_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
+                           const EpiArgs& ea, DevHeader* hdr);
 
 // ------------------------------------------------------------------ attention.cu
 // Decoder sliding-window self-attention for one layer at step t (1-based): RoPE at

@@ -286,25 +286,25 @@ rlt_status encode_impl(rlt_model* m, const int32_t* tokens, int B, int Tn, int T
     const float2* rope = m->at<float2>(m->lay.rope);
     CK(launch_embed<T>(L, tokens, N, m->at<T>(m->lay.embed), c.V, d, h, m->hdr()));
     for (int l = 0; l < c.L_E; ++l) {
-        EpiArgs ea;
+        EpiArgs ea; ea.hdr = m->hdr();
         CK(launch_rmsnorm<T>(L, h, N, d, m->at<float>(m->lay.attn_norm[l]), c.rms_eps, a, d, N, N, nullptr));
         ea.out_f32 = qkv; ea.ld_out = 3 * d;
         CK(launch_gemm<T>(L, Epi::StoreF32, a, d, m->at<T>(m->lay.wqkv[l]), N, 3 * d, d, ea));
         CK(launch_enc_qkv_layout<T>(L, qkv, B, Tn, H, hd, rope, planes));
         CK(launch_enc_attention<T>(L, planes, att, B, Tn, H, hd));
-        ea = EpiArgs(); ea.out_f32 = h; ea.ld_out = d;
+        ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = h; ea.ld_out = d;
         CK(launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.wo[l]), N, d, d, ea));
         CK(launch_rmsnorm<T>(L, h, N, d, m->at<float>(m->lay.ffn_norm[l]), c.rms_eps, a, d, N, N, nullptr));
-        ea = EpiArgs(); ea.out_t = act; ea.ld_out = F;
+        ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_t = act; ea.ld_out = F;
         CK(launch_gemm<T>(L, Epi::SwiGLU, a, d, m->at<T>(m->lay.wgu[l]), N, 2 * F, d, ea));
-        ea = EpiArgs(); ea.out_f32 = h; ea.ld_out = d;
+        ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = h; ea.ld_out = d;
         CK(launch_gemm<T>(L, Epi::ResidAdd, act, F, m->at<T>(m->lay.wdown[l]), N, d, F, ea));
     }
     // e = RMSNorm(h) written with row capacity T_alloc, plus a contiguous copy for M
     CK(launch_rmsnorm<T>(L, h, N, d, m->at<float>(m->lay.enc_norm), c.rms_eps, e, d, Tn, T_alloc, ews));
     size_t group_elems = (size_t)2 * B * H * (size_t)T_alloc * hd;
     for (int g = 0; g < c.G; ++g) {
-        EpiArgs ea;
+        EpiArgs ea; ea.hdr = m->hdr();
         ea.out_f32 = qkv; ea.ld_out = 2 * d;
         CK(launch_gemm<T>(L, Epi::StoreF32, ews, d, m->at<T>(m->lay.mem) + (size_t)g * 2 * d * d, N, 2 * d, d, ea));
         CK(launch_mem_layout<T>(L, qkv, B, Tn, T_alloc, H, hd, M + g * group_elems));
@@ -351,39 +351,39 @@ rlt_status step_impl(rlt_model* m, uint8_t* state, int B, const T* e, const T* M
     // gated merge: x = e_t + sigmoid(W_ge e_t + W_gs s + b_g) * (W_fb s)
     CKP(RLT_K_MERGE, launch_merge_prep<T>(L, e, T_alloc, t, s, A, B, d, sh, m->version, m->hdr()));
     {
-        EpiArgs ea;
+        EpiArgs ea; ea.hdr = m->hdr();
         ea.out_f32 = x; ea.ld_out = d; ea.merge_e = A; ea.ld_e = 2 * d; ea.bias = m->at<float>(m->lay.merge_b);
         CKP(RLT_K_MERGE, launch_gemm<T>(L, Epi::Merge, A, 2 * d, m->at<T>(m->lay.merge_w), B, 2 * d, 2 * d, ea));
     }
     for (int l = 0; l < c.L_D; ++l) {
-        EpiArgs ea;
+        EpiArgs ea; ea.hdr = m->hdr();
         // sliding-window self-attention (weights of encoder layer l)
         CKP(RLT_K_NORM, launch_rmsnorm<T>(L, x, B, d, m->at<float>(m->lay.attn_norm[l]), c.rms_eps, A, d, B, B, nullptr));
         ea.out_f32 = qkv; ea.ld_out = 3 * d;
         CKP(RLT_K_QKV, launch_gemm<T>(L, Epi::StoreF32, A, d, m->at<T>(m->lay.wqkv[l]), B, 3 * d, d, ea));
         CKP(RLT_K_SWA, launch_swa_decode<T>(L, qkv, rope_row, ring + (size_t)l * ring_layer_elems(c, B), att, B, H, hd,
                                 c.W, t));
-        ea = EpiArgs(); ea.out_f32 = x; ea.ld_out = d;
+        ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = x; ea.ld_out = d;
         CKP(RLT_K_O, launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.wo[l]), B, d, d, ea));
         // cross-attention to M_{<=t}
         CKP(RLT_K_NORM, launch_rmsnorm<T>(L, x, B, d, m->at<float>(m->lay.xattn_norm[l]), c.rms_eps, A, d, B, B, nullptr));
-        ea = EpiArgs(); ea.out_f32 = qc; ea.ld_out = d;
+        ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = qc; ea.ld_out = d;
         CKP(RLT_K_QC, launch_gemm<T>(L, Epi::StoreF32, A, d, m->at<T>(m->lay.wqc[l]), B, d, d, ea));
         const T* Mg = M + (c.G == 1 ? 0 : (size_t)l * group_elems);
         CKP(RLT_K_XATTN, launch_xattn_decode<T>(L, qc, Mg, T_alloc, t, att, B, H, hd, splits, part));
-        ea = EpiArgs(); ea.out_f32 = x; ea.ld_out = d;
+        ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = x; ea.ld_out = d;
         CKP(RLT_K_OC, launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.woc[l]), B, d, d, ea));
         // SwiGLU FFN (weights of encoder layer l)
         CKP(RLT_K_NORM, launch_rmsnorm<T>(L, x, B, d, m->at<float>(m->lay.ffn_norm[l]), c.rms_eps, A, d, B, B, nullptr));
-        ea = EpiArgs(); ea.out_t = act; ea.ld_out = F;
+        ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_t = act; ea.ld_out = F;
         CKP(RLT_K_FFN_UP, launch_gemm<T>(L, Epi::SwiGLU, A, d, m->at<T>(m->lay.wgu[l]), B, 2 * F, d, ea));
-        ea = EpiArgs(); ea.out_f32 = x; ea.ld_out = d;
+        ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = x; ea.ld_out = d;
         CKP(RLT_K_FFN_DOWN, launch_gemm<T>(L, Epi::ResidAdd, act, F, m->at<T>(m->lay.wdown[l]), B, d, F, ea));
     }
     // split: s_t = RMSNorm(x) becomes the state; the same s_t feeds the head
     CKP(RLT_K_FINAL, launch_final_norm<T>(L, x, B, d, m->at<float>(m->lay.dec_norm), c.rms_eps, s, A, sh, t));
     if (io.head) {
-        EpiArgs ea;
+        EpiArgs ea; ea.hdr = m->hdr();
         ea.out_f32 = logits; ea.ld_out = c.V;
         CKP(RLT_K_HEAD, launch_gemm<T>(L, Epi::StoreF32, A, d, m->at<T>(m->lay.unembed), B, c.V, d, ea));
         CKP(RLT_K_LSE, launch_lse_gather(L, logits, B, c.V, io.tau, io.tok, io.tok_stride, io.logp_tok, io.lp_stride,
@@ -664,6 +664,22 @@ rlt_status rlt_last_error(rlt_model* m, void* stream) {
 }
 
 uint64_t rlt_launch_count(const rlt_model* m) { return m ? m->launches : 0; }
+
+rlt_status rlt_gemm_bf16(rlt_model* m, const void* A, const void* W, float* C, int M, int N, int K, int kernel,
+                         void* stream) {
+    if (!m || !A || !W || !C || M < 1 || N < 1 || K < 1 || (kernel != 0 && kernel != 1)) return RLT_EINVAL;
+    if (!aligned(A, 16) || !aligned(W, 16) || !aligned(C, 16) || K % 8 || N % 4) return RLT_EINVAL;
+    Launch L = m->launch(stream);
+    EpiArgs ea;
+    ea.hdr = m->hdr();
+    ea.out_f32 = C;
+    ea.ld_out = N;
+    const bf16* a = reinterpret_cast<const bf16*>(A);
+    const bf16* w = reinterpret_cast<const bf16*>(W);
+    CK(kernel == 0 ? launch_gemm_tc(L, Epi::StoreF32, a, K, w, M, N, K, ea, m->hdr())
+                   : launch_gemm_simt<bf16>(L, Epi::StoreF32, a, K, w, M, N, K, ea));
+    return RLT_OK;
+}
 
 rlt_status rlt_profile_start(rlt_model* m, uint32_t kind_mask) {
     if (!m) return RLT_EINVAL;

@@ -64,6 +64,8 @@ _EXPORTS = {
                                   ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "rlt_last_error": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "rlt_launch_count": (ctypes.c_uint64, [ctypes.c_void_p]),
+    "rlt_gemm_bf16": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                     ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "rlt_profile_start": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_uint32]),
     "rlt_profile_stop": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_double),
                                         ctypes.POINTER(ctypes.c_uint64)]),
@@ -259,6 +261,17 @@ class RLTModel:
         _check(lib().rlt_replay(self.handle, _ptr(tokens), B, T, _ptr(P), float(tau), _ptr(score), _ptr(lp),
                                 _ptr(st.buf) if st else None, _ptr(ws), ws.numel(), _stream()), "rlt_replay")
         return score, lp, st
+
+    def gemm_bf16(self, A: torch.Tensor, W: torch.Tensor, kernel: int = 0) -> torch.Tensor:
+        """C = A W^T (bf16 in, float32 out) with the library's tensor-core (0) or CUDA-core (1) kernel."""
+        A = A.to(self.device, torch.bfloat16).contiguous()
+        W = W.to(self.device, torch.bfloat16).contiguous()
+        M, K = A.shape
+        N = W.shape[0]
+        C = torch.empty((M, N), dtype=torch.float32, device=self.device)
+        _check(lib().rlt_gemm_bf16(self.handle, _ptr(A), _ptr(W), _ptr(C), M, N, K, kernel, _stream()),
+               "rlt_gemm_bf16")
+        return C
 
     def profile_start(self, kinds=None) -> None:
         """Bracket every launch of the given kernel kinds (names of KERNEL_KINDS) with CUDA events."""

@@ -207,6 +207,17 @@ rlt_status rlt_last_error(rlt_model* m, void* stream);
  * points).  Used by benchmarks to count launches inside a timed region. */
 uint64_t rlt_launch_count(const rlt_model* m);
 
+/* ---------------------------------------------------------------- building block */
+
+/* C[M, N] = A[M, K] W[N, K]^T with bf16 operands (row-major, K contiguous) and float32
+ * accumulation/output, on the model's stream-ordered error flags.  kernel 0 = the
+ * tensor-core (tcgen05 + TMA) kernel the bf16 decoder and encoder use, kernel 1 = the
+ * CUDA-core kernel.  A, W, C 16-byte aligned, K a multiple of 8, N a multiple of 4.
+ * Errors: RLT_EINVAL, RLT_ECUDA; a tensor-core wait that times out latches
+ * RLT_ETIMEOUT (rlt_last_error). */
+rlt_status rlt_gemm_bf16(rlt_model* m, const void* A, const void* W, float* C, int M, int N, int K,
+                         int kernel, void* stream);
+
 /* ---------------------------------------------------------------- kernel timing */
 
 /* Kernel kinds of the decoder step (and the encoder as one kind) for live timing. */

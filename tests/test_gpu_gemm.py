@@ -1,0 +1,52 @@
+"""The tcgen05/TMA GEMM against float64 matmul of the same bf16 operands (and the CUDA-core kernel).
+
+Bound: float32 accumulation of K products, |dC| <= 1e-4 * (|A| |W|^T) elementwise.
+"""
+import numpy as np
+import pytest
+import torch
+
+from workloads import TINY
+from gpu_util import build_model
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [
+    (512, 3072, 1024),    # 300M-class decoder q/k/v at B=512
+    (512, 1024, 4096),    # FFN down
+    (64, 2048, 2048),     # small-batch decoder row count
+    (1, 256, 128),        # single row
+    (300, 200, 136),      # ragged M, N and K (K not a multiple of the 64-wide k-block)
+    (4096, 1536, 1024),   # encoder-like
+    (129, 40, 64),
+]
+
+
+@pytest.fixture(scope="module")
+def model():
+    return build_model(TINY.model, max_pos=8)
+
+
+@pytest.mark.parametrize("M,N,K", SHAPES)
+def test_tcgen05_gemm_matches_float64(model, M, N, K):
+    g = torch.Generator().manual_seed(M * 7919 + N * 31 + K)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    W = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16)
+    ref = A.double() @ W.double().T
+    bound = A.double().abs() @ W.double().abs().T
+    c_tc = model.gemm_bf16(A, W, kernel=0).cpu().double()
+    torch.cuda.synchronize()
+    assert model.last_error() == 0
+    err = (c_tc - ref).abs()
+    assert bool((err <= 1e-4 * bound + 1e-6).all()), float((err / (bound + 1e-6)).max())
+    c_simt = model.gemm_bf16(A, W, kernel=1).cpu().double()
+    assert bool(((c_simt - ref).abs() <= 1e-4 * bound + 1e-6).all())
+
+
+def test_tcgen05_gemm_is_deterministic(model):
+    g = torch.Generator().manual_seed(5)
+    A = torch.randn(512, 1024, generator=g).to(torch.bfloat16)
+    W = torch.randn(3072, 1024, generator=g).to(torch.bfloat16)
+    a = model.gemm_bf16(A, W)
+    b = model.gemm_bf16(A, W)
+    assert torch.equal(a, b)
