@@ -248,7 +248,8 @@ def main() -> int:
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=RLT_300M.name, choices=sorted(WORKLOADS))
-    ap.add_argument("--T", type=int, default=None, help="override the sweep length (parity/debug runs only)")
+    ap.add_argument("--T", type=int, default=None, help="override the sweep length (profiling runs only)")
+    ap.add_argument("--B", type=int, default=None, help="override the batch (profiling runs only)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-replay", action="store_true")
@@ -257,8 +258,8 @@ def main() -> int:
         ap.error("--warmup must be >= 3")
 
     wl = WORKLOADS[args.workload]
-    if args.T:
-        wl = wl.with_batch(wl.B, args.T)
+    if args.T or args.B:
+        wl = wl.with_batch(args.B or wl.B, args.T or wl.T)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -287,6 +288,8 @@ def main() -> int:
     tok = torch.from_numpy(tokens).to(dev)
     tok_tb = tok.t().contiguous()                        # row t = x_{t+1} of every sequence
     e, M = model.encode(tok)
+    torch.cuda.synchronize()
+    model.release_workspaces()
     state = model.new_state(B)
     lp_tb = torch.zeros((T, B), dtype=torch.float32, device=dev)
 
@@ -315,10 +318,12 @@ def main() -> int:
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(gpu_id_for(local)) as clk:
         model.profile_start([dominant])
+        torch.cuda.nvtx.range_push("timed")
         ev0.record()
         for _ in range(args.steps):
             sweep()
         ev1.record()
+        torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize()
         dom = model.profile_stop()
     launches = model.launch_count - launches0

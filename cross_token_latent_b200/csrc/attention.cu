@@ -107,17 +107,28 @@ __device__ __forceinline__ void merge_groups(float& m, float& l, float* acc) {
     }
 }
 
+// One CTA of SWA_WARPS warps per (sequence, head).  Every warp computes q and the current
+// k/v (RoPE at position t-1); warp w streams a contiguous share of the n = min(t-1, W-1)
+// cached entries; the warps' partial softmax states are merged through shared memory, then
+// warp 0 writes the output and stores k_t, v_t into ring slot (t-1) mod (W-1) (after every
+// warp has read the ring, so the slot's old entry -- token t-W+1, still in the window -- is
+// used first).
+constexpr int SWA_WARPS = 4;
+
 template <typename T, int HD>
-__global__ void __launch_bounds__(WARPS * 32) k_swa_decode(const float* __restrict__ qkv,
-                                                           const float2* __restrict__ rope_row,
-                                                           T* __restrict__ ring, T* __restrict__ o,
-                                                           int B, int H, int W, int t, float qscale) {
+__global__ void __launch_bounds__(SWA_WARPS * 32) k_swa_decode(const float* __restrict__ qkv,
+                                                               const float2* __restrict__ rope_row,
+                                                               T* __restrict__ ring, T* __restrict__ o,
+                                                               int B, int H, int W, int t, float qscale) {
     using G = Geom<T, HD>;
     constexpr int EPL = G::EPL, LPK = G::LPK;
-    int item = blockIdx.x * WARPS + (threadIdx.x >> 5);
-    if (item >= B * H) return;
-    int lane = threadIdx.x & 31, g = lane / LPK, li = lane % LPK;
-    int b = item / H, h = item % H;
+    __shared__ float sm_m[SWA_WARPS], sm_l[SWA_WARPS];
+    __shared__ __align__(16) float sm_acc[SWA_WARPS][HD];
+    pdl_wait();
+    pdl_trigger();
+    const int item = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane / LPK, li = lane % LPK;
+    const int b = item / H, h = item % H;
     const int d = H * HD, half = HD / 2;
     const float* row = qkv + (long long)b * 3 * d + h * HD;
     float q[EPL], k[EPL], v[EPL];
@@ -132,19 +143,19 @@ __global__ void __launch_bounds__(WARPS * 32) k_swa_decode(const float* __restri
         k[i] = round_to<T>(c < half ? ka * cs.x - kp * cs.y : kp * cs.y + ka * cs.x);
         v[i] = round_to<T>(row[2 * d + c]);
     }
-    float sc = 0.f;
+    float m = NEG_BIG, l = 0.f, acc[EPL];
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) sc = fmaf(q[i], k[i], sc);
-    sc = group_sum<LPK>(sc);
-    float m, l, acc[EPL];
-    if (g == 0) {
-        m = sc; l = 1.f;
+    for (int i = 0; i < EPL; ++i) acc[i] = 0.f;
+    if (warp == 0) {
+        float sc = 0.f;
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) acc[i] = v[i];
-    } else {
-        m = NEG_BIG; l = 0.f;
+        for (int i = 0; i < EPL; ++i) sc = fmaf(q[i], k[i], sc);
+        sc = group_sum<LPK>(sc);
+        if (g == 0) {
+            m = sc; l = 1.f;
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) acc[i] = 0.f;
+            for (int i = 0; i < EPL; ++i) acc[i] = v[i];
+        }
     }
     T* Kr = nullptr;
     T* Vr = nullptr;
@@ -152,20 +163,40 @@ __global__ void __launch_bounds__(WARPS * 32) k_swa_decode(const float* __restri
         Kr = ring + (((long long)b * 2 + 0) * H + h) * (long long)(W - 1) * HD;
         Vr = ring + (((long long)b * 2 + 1) * H + h) * (long long)(W - 1) * HD;
         int n = min(t - 1, W - 1);
-        attend<T, HD, 4, true>(q, Kr, Vr, n, g, li, m, l, acc);
+        int per = (n + SWA_WARPS - 1) / SWA_WARPS;
+        int j0 = min(n, warp * per);
+        int nj = min(n, j0 + per) - j0;
+        attend<T, HD, 4, true>(q, Kr + (long long)j0 * HD, Vr + (long long)j0 * HD, nj, g, li, m, l, acc);
     }
     merge_groups<T, HD>(m, l, acc);
-    __syncwarp();
     if (g == 0) {
-        if (W > 1) {
-            int slot = (t - 1) % (W - 1);
-            st16(Kr + (long long)slot * HD + li * EPL, Vec16<T>::pack(k));
-            st16(Vr + (long long)slot * HD + li * EPL, Vec16<T>::pack(v));
-        }
-        float inv = 1.0f / l, out[EPL];
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) out[i] = acc[i] * inv;
-        st16(o + (long long)b * d + h * HD + li * EPL, Vec16<T>::pack(out));
+        for (int i = 0; i < EPL; ++i) sm_acc[warp][li * EPL + i] = acc[i];
+        if (li == 0) { sm_m[warp] = m; sm_l[warp] = l; }
+    }
+    __syncthreads();
+    if (warp != 0 || g != 0) return;
+    float mx = NEG_BIG;
+#pragma unroll
+    for (int w = 0; w < SWA_WARPS; ++w) mx = fmaxf(mx, sm_m[w]);
+    float L = 0.f, out[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) out[i] = 0.f;
+#pragma unroll
+    for (int w = 0; w < SWA_WARPS; ++w) {
+        float c = exp2f(sm_m[w] - mx);
+        L += sm_l[w] * c;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) out[i] += sm_acc[w][li * EPL + i] * c;
+    }
+    float inv = 1.0f / L;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) out[i] *= inv;
+    st16(o + (long long)b * d + h * HD + li * EPL, Vec16<T>::pack(out));
+    if (W > 1) {
+        int slot = (t - 1) % (W - 1);
+        st16(Kr + (long long)slot * HD + li * EPL, Vec16<T>::pack(k));
+        st16(Vr + (long long)slot * HD + li * EPL, Vec16<T>::pack(v));
     }
 }
 
@@ -176,6 +207,8 @@ __global__ void __launch_bounds__(WARPS * 32) k_xattn_decode(const float* __rest
                                                              int chunk, float* __restrict__ part, float qscale) {
     using G = Geom<T, HD>;
     constexpr int EPL = G::EPL, LPK = G::LPK;
+    pdl_wait();
+    pdl_trigger();
     int item = blockIdx.x * WARPS + (threadIdx.x >> 5);
     if (item >= B * H * n_splits) return;
     int lane = threadIdx.x & 31, g = lane / LPK, li = lane % LPK;
@@ -214,6 +247,8 @@ __global__ void __launch_bounds__(WARPS * 32) k_xattn_decode(const float* __rest
 template <typename T>
 __global__ void k_attn_combine(const float* __restrict__ part, int n_splits, int HD, int H,
                                T* __restrict__ o) {
+    pdl_wait();
+    pdl_trigger();
     int bh = blockIdx.x, c = threadIdx.x;
     if (c >= HD) return;
     const float* p = part + (long long)bh * n_splits * (HD + 2);
@@ -234,6 +269,8 @@ __global__ void __launch_bounds__(WARPS * 32) k_enc_attn(const T* __restrict__ p
                                                          int B, int Tn, int H, float qscale) {
     using G = Geom<T, HD>;
     constexpr int EPL = G::EPL, LPK = G::LPK;
+    pdl_wait();
+    pdl_trigger();
     long long item = (long long)blockIdx.x * WARPS + (threadIdx.x >> 5);
     if (item >= (long long)B * H * Tn) return;
     int lane = threadIdx.x & 31, g = lane / LPK, li = lane % LPK;
@@ -265,22 +302,27 @@ inline unsigned blocks_for(long long items) { return (unsigned)((items + WARPS -
 
 }  // namespace
 
-#define RLT_HD_SWITCH(hd, KERNEL_CALL)          \
-    switch (hd) {                               \
-        case 16: { constexpr int HD = 16; KERNEL_CALL; break; }   \
-        case 32: { constexpr int HD = 32; KERNEL_CALL; break; }   \
-        case 64: { constexpr int HD = 64; KERNEL_CALL; break; }   \
-        case 128: { constexpr int HD = 128; KERNEL_CALL; break; } \
-        default: return cudaErrorInvalidValue;  \
+#define RLT_HD_DISPATCH(hd, EXPR)                                  \
+    switch (hd) {                                                  \
+        case 16: { constexpr int HD = 16; return EXPR; }           \
+        case 32: { constexpr int HD = 32; return EXPR; }           \
+        case 64: { constexpr int HD = 64; return EXPR; }           \
+        case 128: { constexpr int HD = 128; return EXPR; }         \
+        default: return cudaErrorInvalidValue;                     \
     }
 
 template <typename T>
 cudaError_t launch_swa_decode(Launch L, const float* qkv, const float2* rope_row, T* ring, T* o, int B,
                               int H, int hd, int W, int t) {
-    RLT_HD_SWITCH(hd, (k_swa_decode<T, HD><<<blocks_for((long long)B * H), WARPS * 32, 0, L.stream>>>(
-                           qkv, rope_row, ring, o, B, H, W, t, qscale_for(hd))));
-    *L.count += 1;
-    return cudaGetLastError();
+    RLT_HD_DISPATCH(hd, launch_k(L, k_swa_decode<T, HD>, (unsigned)(B * H), SWA_WARPS * 32, 0, qkv, rope_row,
+                                 ring, o, B, H, W, t, qscale_for(hd)));
+}
+
+template <typename T>
+static cudaError_t xattn_main(Launch L, const float* qc, const T* Mg, int T_alloc, int t, T* o, int B, int H,
+                              int hd, int n_splits, int chunk, float* part) {
+    RLT_HD_DISPATCH(hd, launch_k(L, k_xattn_decode<T, HD>, blocks_for((long long)B * H * n_splits), WARPS * 32, 0,
+                                 qc, Mg, T_alloc, t, o, B, H, n_splits, chunk, part, qscale_for(hd)));
 }
 
 template <typename T>
@@ -288,23 +330,15 @@ cudaError_t launch_xattn_decode(Launch L, const float* qc, const T* Mg, int T_al
                                 int H, int hd, int n_splits, float* part) {
     if (n_splits < 1) n_splits = 1;
     int chunk = (t + n_splits - 1) / n_splits;
-    RLT_HD_SWITCH(hd, (k_xattn_decode<T, HD><<<blocks_for((long long)B * H * n_splits), WARPS * 32, 0,
-                                               L.stream>>>(qc, Mg, T_alloc, t, o, B, H, n_splits, chunk,
-                                                           part, qscale_for(hd))));
-    *L.count += 1;
-    if (n_splits > 1) {
-        k_attn_combine<T><<<B * H, hd, 0, L.stream>>>(part, n_splits, hd, H, o);
-        *L.count += 1;
-    }
-    return cudaGetLastError();
+    cudaError_t e = xattn_main<T>(L, qc, Mg, T_alloc, t, o, B, H, hd, n_splits, chunk, part);
+    if (e != cudaSuccess || n_splits == 1) return e;
+    return launch_k(L, k_attn_combine<T>, (unsigned)(B * H), (unsigned)hd, 0, (const float*)part, n_splits, hd, H, o);
 }
 
 template <typename T>
 cudaError_t launch_enc_attention(Launch L, const T* planes, T* o, int B, int Tn, int H, int hd) {
-    RLT_HD_SWITCH(hd, (k_enc_attn<T, HD><<<blocks_for((long long)B * H * Tn), WARPS * 32, 0, L.stream>>>(
-                           planes, o, B, Tn, H, qscale_for(hd))));
-    *L.count += 1;
-    return cudaGetLastError();
+    RLT_HD_DISPATCH(hd, launch_k(L, k_enc_attn<T, HD>, blocks_for((long long)B * H * Tn), WARPS * 32, 0, planes, o,
+                                 B, Tn, H, qscale_for(hd)));
 }
 
 #define RLT_INST(T)                                                                                    \

@@ -101,6 +101,13 @@ __device__ __forceinline__ float warp_max(float v) {
 
 __device__ __forceinline__ void raise_flag(DevHeader* h, uint32_t f) { atomicOr(&h->err_flags, f); }
 
+// Programmatic dependent launch.  Every kernel of the library is launched so that it may
+// start while its predecessor on the stream drains; it must call pdl_wait() before it reads
+// anything an earlier kernel wrote or writes anything an earlier kernel reads.  pdl_trigger()
+// lets the next kernel on the stream be scheduled early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + expf(-x)); }
 __device__ __forceinline__ float siluf_(float x) { return x / (1.0f + expf(-x)); }
 

@@ -12,6 +12,8 @@ inline unsigned cdiv(long long a, long long b) { return (unsigned)((a + b - 1) /
 template <typename T>
 __global__ void k_pack_rows(const float* __restrict__ src, T* __restrict__ dst, int rows, int cols,
                             int dst_ld, int row_mult, int row_off, int col_off) {
+    pdl_wait();
+    pdl_trigger();
     long long n = (long long)rows * cols;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
          i += (long long)gridDim.x * blockDim.x) {
@@ -21,6 +23,8 @@ __global__ void k_pack_rows(const float* __restrict__ src, T* __restrict__ dst, 
 }
 
 __global__ void k_rope_table(float2* table, int max_pos, int half, int hd, double base) {
+    pdl_wait();
+    pdl_trigger();
     long long n = (long long)max_pos * half;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
          i += (long long)gridDim.x * blockDim.x) {
@@ -35,6 +39,8 @@ __global__ void k_rope_table(float2* table, int max_pos, int half, int hd, doubl
 template <typename T>
 __global__ void k_embed(const int32_t* __restrict__ tok, int N, const T* __restrict__ embed, int V,
                         int d, float* __restrict__ h, DevHeader* hdr) {
+    pdl_wait();
+    pdl_trigger();
     int n = blockIdx.x;
     if (n >= N) return;
     int id = tok[n];
@@ -52,6 +58,8 @@ template <typename T>
 __global__ void k_rmsnorm(const float* __restrict__ x, int N, int d, const float* __restrict__ gain,
                           float eps, T* __restrict__ out, int out_ld, int rows_per_seq,
                           int out_rows_per_seq, T* __restrict__ out2) {
+    pdl_wait();
+    pdl_trigger();
     int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     int lane = threadIdx.x & 31;
     if (warp >= N) return;
@@ -82,6 +90,8 @@ template <typename T>
 __global__ void k_merge_prep(const T* __restrict__ e, int T_alloc, int t, const float* __restrict__ s,
                              T* __restrict__ A, int B, int d, const StateHeader* sh, uint64_t version,
                              DevHeader* hdr) {
+    pdl_wait();
+    pdl_trigger();
     int b = blockIdx.x;
     if (b == 0 && threadIdx.x == 0 && sh) {
         if (sh->magic != STATE_MAGIC || sh->t != t - 1 || sh->version != version)
@@ -99,6 +109,8 @@ __global__ void k_merge_prep(const T* __restrict__ e, int T_alloc, int t, const 
 template <typename T>
 __global__ void k_final_norm(const float* __restrict__ x, int B, int d, const float* __restrict__ gain,
                              float eps, float* __restrict__ s, T* __restrict__ hs, StateHeader* sh, int t) {
+    pdl_wait();
+    pdl_trigger();
     int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     int lane = threadIdx.x & 31;
     if (warp == 0 && lane == 0 && sh) sh->t = t;
@@ -120,6 +132,8 @@ __global__ void k_lse_gather(const float* __restrict__ logits, int B, int V, flo
                              const int32_t* __restrict__ tok, int tok_stride, float* logp_tok,
                              int lp_stride, float* lse_out, float* logp_full, float* score,
                              const int32_t* prompt_len, int t, DevHeader* hdr) {
+    pdl_wait();
+    pdl_trigger();
     int b = blockIdx.x;
     const float* z = logits + (long long)b * V;
     float m = -INFINITY, l = 0.f;
@@ -165,6 +179,8 @@ __global__ void k_lse_gather(const float* __restrict__ logits, int B, int V, flo
 template <typename T>
 __global__ void k_enc_qkv_layout(const float* __restrict__ qkv, int B, int Tn, int H, int hd,
                                  const float2* __restrict__ rope, T* __restrict__ planes) {
+    pdl_wait();
+    pdl_trigger();
     int half = hd / 2;
     int d = H * hd;
     long long total = (long long)B * Tn * H * half;
@@ -193,6 +209,8 @@ __global__ void k_enc_qkv_layout(const float* __restrict__ qkv, int B, int Tn, i
 template <typename T>
 __global__ void k_mem_layout(const float* __restrict__ kv, int B, int Tn, int T_alloc, int H, int hd,
                              T* __restrict__ Mg) {
+    pdl_wait();
+    pdl_trigger();
     int d = H * hd;
     long long total = (long long)B * Tn * 2 * d;
     long long plane = (long long)B * H * T_alloc * hd;
@@ -208,6 +226,8 @@ __global__ void k_mem_layout(const float* __restrict__ kv, int B, int Tn, int T_
 
 __global__ void k_state_init(const float* __restrict__ s_star, int B, int d, float* __restrict__ s,
                              StateHeader* sh, uint64_t version) {
+    pdl_wait();
+    pdl_trigger();
     long long n = (long long)B * d;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
          i += (long long)gridDim.x * blockDim.x)
@@ -225,85 +245,71 @@ inline unsigned grid_for(long long n, int threads) {
     return (unsigned)(g > 148LL * 64 ? 148LL * 64 : (g < 1 ? 1 : g));
 }
 
-inline cudaError_t done(Launch L, int n = 1) {
-    *L.count += n;
-    return cudaGetLastError();
-}
 
 }  // namespace
 
 template <typename T>
 cudaError_t launch_pack_rows(Launch L, const float* src, T* dst, int rows, int cols, int dst_ld,
                              int row_mult, int row_off, int col_off) {
-    k_pack_rows<T><<<grid_for((long long)rows * cols, 256), 256, 0, L.stream>>>(
-        src, dst, rows, cols, dst_ld, row_mult, row_off, col_off);
-    return done(L);
+    return launch_k(L, k_pack_rows<T>, grid_for((long long)rows * cols, 256), 256, 0, src, dst, rows, cols, dst_ld,
+                    row_mult, row_off, col_off);
 }
 
 cudaError_t launch_rope_table(Launch L, float2* table, int max_pos, int head_dim, float base) {
     int half = head_dim / 2;
-    k_rope_table<<<grid_for((long long)max_pos * half, 256), 256, 0, L.stream>>>(
-        table, max_pos, half, head_dim, (double)base);
-    return done(L);
+    return launch_k(L, k_rope_table, grid_for((long long)max_pos * half, 256), 256, 0, table, max_pos, half, head_dim,
+                    (double)base);
 }
 
 template <typename T>
 cudaError_t launch_embed(Launch L, const int32_t* tok, int N, const T* embed, int V, int d, float* h,
                          DevHeader* hdr) {
-    k_embed<T><<<N, 128, 0, L.stream>>>(tok, N, embed, V, d, h, hdr);
-    return done(L);
+    return launch_k(L, k_embed<T>, N, 128, 0, tok, N, embed, V, d, h, hdr);
 }
 
 template <typename T>
 cudaError_t launch_rmsnorm(Launch L, const float* x, int N, int d, const float* gain, float eps, T* out,
                            int out_ld, int rows_per_seq, int out_rows_per_seq, T* out2) {
-    k_rmsnorm<T><<<cdiv(N, 8), 256, 0, L.stream>>>(x, N, d, gain, eps, out, out_ld, rows_per_seq,
-                                                     out_rows_per_seq, out2);
-    return done(L);
+    return launch_k(L, k_rmsnorm<T>, cdiv(N, 8), 256, 0, x, N, d, gain, eps, out, out_ld, rows_per_seq,
+                    out_rows_per_seq, out2);
 }
 
 template <typename T>
 cudaError_t launch_merge_prep(Launch L, const T* e, int T_alloc, int t, const float* s, T* A, int B,
                               int d, const StateHeader* sh, uint64_t version, DevHeader* hdr) {
-    k_merge_prep<T><<<B, 256, 0, L.stream>>>(e, T_alloc, t, s, A, B, d, sh, version, hdr);
-    return done(L);
+    return launch_k(L, k_merge_prep<T>, B, 256, 0, e, T_alloc, t, s, A, B, d, sh, version, hdr);
 }
 
 template <typename T>
 cudaError_t launch_final_norm(Launch L, const float* x, int B, int d, const float* gain, float eps,
                               float* s, T* hs, StateHeader* sh, int t) {
-    k_final_norm<T><<<cdiv(B, 8), 256, 0, L.stream>>>(x, B, d, gain, eps, s, hs, sh, t);
-    return done(L);
+    return launch_k(L, k_final_norm<T>, cdiv(B, 8), 256, 0, x, B, d, gain, eps, s, hs, sh, t);
 }
 
 cudaError_t launch_lse_gather(Launch L, const float* logits, int B, int V, float tau, const int32_t* tok,
                               int tok_stride, float* logp_tok, int lp_stride, float* lse,
                               float* logp_full, float* score, const int32_t* prompt_len, int t,
                               DevHeader* hdr) {
-    k_lse_gather<<<B, 512, 0, L.stream>>>(logits, B, V, tau, tok, tok_stride, logp_tok, lp_stride, lse,
-                                          logp_full, score, prompt_len, t, hdr);
-    return done(L);
+    return launch_k(L, k_lse_gather, B, 512, 0, logits, B, V, tau, tok, tok_stride, logp_tok, lp_stride, lse,
+                    logp_full, score, prompt_len, t, hdr);
 }
 
 template <typename T>
 cudaError_t launch_enc_qkv_layout(Launch L, const float* qkv, int B, int Tn, int H, int hd,
                                   const float2* rope, T* planes) {
-    k_enc_qkv_layout<T><<<grid_for((long long)B * Tn * H * (hd / 2), 256), 256, 0, L.stream>>>(
-        qkv, B, Tn, H, hd, rope, planes);
-    return done(L);
+    return launch_k(L, k_enc_qkv_layout<T>, grid_for((long long)B * Tn * H * (hd / 2), 256), 256, 0, qkv, B, Tn, H,
+                    hd, rope, planes);
 }
 
 template <typename T>
 cudaError_t launch_mem_layout(Launch L, const float* kv, int B, int Tn, int T_alloc, int H, int hd, T* Mg) {
-    k_mem_layout<T><<<grid_for((long long)B * Tn * 2 * H * hd, 256), 256, 0, L.stream>>>(
-        kv, B, Tn, T_alloc, H, hd, Mg);
-    return done(L);
+    return launch_k(L, k_mem_layout<T>, grid_for((long long)B * Tn * 2 * H * hd, 256), 256, 0, kv, B, Tn, T_alloc,
+                    H, hd, Mg);
 }
 
 cudaError_t launch_state_init(Launch L, const float* s_star, int B, int d, float* s, StateHeader* sh,
                               uint64_t version) {
-    k_state_init<<<grid_for((long long)B * d, 256), 256, 0, L.stream>>>(s_star, B, d, s, sh, version);
-    return done(L);
+    return launch_k(L, k_state_init, grid_for((long long)B * d, 256), 256, 0, s_star, B, d, s, sh, version);
 }
 
 #define RLT_INST(T)                                                                                   \

@@ -46,6 +46,8 @@ struct EpiOps {
 template <typename T>
 __global__ void __launch_bounds__(256) k_gemm_simt(const T* __restrict__ A, int lda, const T* __restrict__ W,
                                                    int M, int N, int K, Epi epi, EpiArgs ea) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ float As[BK][BM + 4];
     __shared__ float Ws[BK][BN + 4];
     int tid = threadIdx.x;
@@ -92,9 +94,7 @@ template <typename T>
 cudaError_t launch_gemm_simt(Launch L, Epi epi, const T* A, int lda, const T* W, int M, int N, int K,
                              const EpiArgs& ea) {
     dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
-    k_gemm_simt<T><<<grid, 256, 0, L.stream>>>(A, lda, W, M, N, K, epi, ea);
-    *L.count += 1;
-    return cudaGetLastError();
+    return launch_k(L, k_gemm_simt<T>, grid, 256, 0, A, lda, W, M, N, K, epi, ea);
 }
 
 template <>

@@ -186,6 +186,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
     const int nkb = (K + BK - 1) / BK;
+    pdl_trigger();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -207,10 +208,21 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0 && lane == 0) {
-        // TMA producer
+        // TMA producer.  Weight tiles do not depend on the previous kernel: the first stages'
+        // W loads are issued before the programmatic-launch dependency wait, the activation
+        // (A) loads after it.
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmW) : "memory");
-        for (int kb = 0; kb < nkb; ++kb) {
+        const int pre = nkb < STAGES ? nkb : STAGES;
+        for (int kb = 0; kb < pre; ++kb) {
+            uint8_t* a = smem + kb * S::STAGE_BYTES;
+            mbar_expect_tx(&full[kb], S::STAGE_BYTES);
+            tma_load_2d(a + A_BYTES, &tmW, &full[kb], kb * BK, n0);
+        }
+        pdl_wait();
+        for (int kb = 0; kb < pre; ++kb)
+            tma_load_2d(smem + kb * S::STAGE_BYTES, &tmA, &full[kb], kb * BK, m0);
+        for (int kb = pre; kb < nkb; ++kb) {
             int s = kb % STAGES;
             uint32_t ph = (kb / STAGES) & 1;
             if (!mbar_wait(&empty[s], ph ^ 1, &abort_flag)) { abort_flag = 1; break; }
@@ -237,6 +249,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         umma_commit(done);
     }
     __syncwarp();
+    pdl_wait();
 
     // epilogue: thread owns output row m0 + 32*warp + lane
     bool ok = mbar_wait(done, 0, &abort_flag);
@@ -307,9 +320,7 @@ cudaError_t run_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int
     CUtensorMap ta, tw;
     if (!make_map(&ta, A, M, K, lda, BM) || !make_map(&tw, W, N, K, K, BN)) return cudaErrorInvalidValue;
     dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
-    k_gemm_tc<BN, STAGES><<<grid, 128, S::SMEM, L.stream>>>(ta, tw, M, N, K, epi, ea, hdr);
-    *L.count += 1;
-    return cudaGetLastError();
+    return launch_k(L, k_gemm_tc<BN, STAGES>, grid, 128, S::SMEM, ta, tw, M, N, K, epi, ea, hdr);
 }
 
 }  // namespace

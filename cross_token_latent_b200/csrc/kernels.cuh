@@ -2,6 +2,8 @@
 // it names on `L.stream`, adds their number to *L.count and returns the launch status.
 #pragma once
 
+#include <utility>
+
 #include "common.cuh"
 
 namespace rlt {
@@ -10,6 +12,25 @@ struct Launch {
     cudaStream_t stream;
     uint64_t* count;
 };
+
+// Launch `kernel` on L.stream with programmatic stream serialization (see pdl_wait in
+// common.cuh) and count it.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(Launch L, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                            Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = L.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    *L.count += 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // ------------------------------------------------------------------ elementwise.cu
 // dst[(r*row_mult + row_off) * dst_ld + col_off + c] = T(src[r*cols + c])
