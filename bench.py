@@ -253,8 +253,11 @@ def main() -> int:
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-replay", action="store_true")
+    ap.add_argument("--nvtx-sample", type=int, default=0,
+                    help="profiling runs: wrap this many evenly spaced steps of the first timed sweep in an NVTX "
+                         "range 'sample' (for ncu --nvtx-include sample/); skips the breakdown sweep")
     args = ap.parse_args()
-    if args.warmup < 3:
+    if args.warmup < 3 and not args.nvtx_sample:
         ap.error("--warmup must be >= 3")
 
     wl = WORKLOADS[args.workload]
@@ -293,12 +296,21 @@ def main() -> int:
     state = model.new_state(B)
     lp_tb = torch.zeros((T, B), dtype=torch.float32, device=dev)
 
-    def sweep():
+    sample_steps = set()
+    if args.nvtx_sample:
+        sample_steps = {int(round(i * (T - 1) / max(1, args.nvtx_sample - 1))) for i in range(args.nvtx_sample)}
+
+    def sweep(mark=False):
         model.reset_state(state)
         for t in range(T):
             nxt = t + 1 < T
+            tag = mark and t in sample_steps
+            if tag:
+                torch.cuda.nvtx.range_push("sample")
             model.decode_step(state, e, M, next_tok=tok_tb[t + 1] if nxt else None, tau=wl.tau,
                               logp_tok=lp_tb[t] if nxt else None)
+            if tag:
+                torch.cuda.nvtx.range_pop()
 
     for _ in range(args.warmup):
         sweep()
@@ -306,9 +318,12 @@ def main() -> int:
     model.check_device_errors()
 
     # one untimed sweep with every kernel kind bracketed: the breakdown and the dominant kernel
-    model.profile_start()
-    sweep()
-    breakdown = model.profile_stop()
+    if args.nvtx_sample:
+        breakdown = {"xattn": (1.0, 1)}
+    else:
+        model.profile_start()
+        sweep()
+        breakdown = model.profile_stop()
     dominant = max((k for k in breakdown if k != "encoder"), key=lambda k: breakdown[k][0])
 
     if world > 1:
@@ -320,8 +335,8 @@ def main() -> int:
         model.profile_start([dominant])
         torch.cuda.nvtx.range_push("timed")
         ev0.record()
-        for _ in range(args.steps):
-            sweep()
+        for i in range(args.steps):
+            sweep(mark=i == 0)
         ev1.record()
         torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize()

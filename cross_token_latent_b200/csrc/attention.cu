@@ -116,14 +116,15 @@ __device__ __forceinline__ void merge_groups(float& m, float& l, float* acc) {
 constexpr int SWA_WARPS = 4;
 
 template <typename T, int HD>
-__global__ void __launch_bounds__(SWA_WARPS * 32) k_swa_decode(const float* __restrict__ qkv,
-                                                               const float2* __restrict__ rope_row,
-                                                               T* __restrict__ ring, T* __restrict__ o,
-                                                               int B, int H, int W, int t, float qscale) {
+__global__ void __launch_bounds__(SWA_WARPS * 32, 6) k_swa_decode(const float* __restrict__ qkv,
+                                                                  const float2* __restrict__ rope_row,
+                                                                  T* __restrict__ ring, T* __restrict__ o,
+                                                                  int B, int H, int W, int t, float qscale) {
     using G = Geom<T, HD>;
     constexpr int EPL = G::EPL, LPK = G::LPK;
     __shared__ float sm_m[SWA_WARPS], sm_l[SWA_WARPS];
     __shared__ __align__(16) float sm_acc[SWA_WARPS][HD];
+    __shared__ __align__(16) uint4 sm_kv[2][LPK];      // current k_t, v_t in storage type
     pdl_wait();
     pdl_trigger();
     const int item = blockIdx.x;
@@ -131,22 +132,30 @@ __global__ void __launch_bounds__(SWA_WARPS * 32) k_swa_decode(const float* __re
     const int b = item / H, h = item % H;
     const int d = H * HD, half = HD / 2;
     const float* row = qkv + (long long)b * 3 * d + h * HD;
-    float q[EPL], k[EPL], v[EPL];
+    float q[EPL];
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
         int c = li * EPL + i;
         int cp = c < half ? c + half : c - half;
         float2 cs = rope_row[c % half];
         float qa = row[c], qp = row[cp];
-        float ka = row[d + c], kp = row[d + cp];
         q[i] = (c < half ? qa * cs.x - qp * cs.y : qp * cs.y + qa * cs.x) * qscale;
-        k[i] = round_to<T>(c < half ? ka * cs.x - kp * cs.y : kp * cs.y + ka * cs.x);
-        v[i] = round_to<T>(row[2 * d + c]);
     }
     float m = NEG_BIG, l = 0.f, acc[EPL];
 #pragma unroll
     for (int i = 0; i < EPL; ++i) acc[i] = 0.f;
     if (warp == 0) {
+        // the current token: k_t (rotated) and v_t rounded to the storage type, as cached
+        float k[EPL], v[EPL];
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            int c = li * EPL + i;
+            int cp = c < half ? c + half : c - half;
+            float2 cs = rope_row[c % half];
+            float ka = row[d + c], kp = row[d + cp];
+            k[i] = round_to<T>(c < half ? ka * cs.x - kp * cs.y : kp * cs.y + ka * cs.x);
+            v[i] = round_to<T>(row[2 * d + c]);
+        }
         float sc = 0.f;
 #pragma unroll
         for (int i = 0; i < EPL; ++i) sc = fmaf(q[i], k[i], sc);
@@ -155,6 +164,8 @@ __global__ void __launch_bounds__(SWA_WARPS * 32) k_swa_decode(const float* __re
             m = sc; l = 1.f;
 #pragma unroll
             for (int i = 0; i < EPL; ++i) acc[i] = v[i];
+            sm_kv[0][li] = Vec16<T>::pack(k);
+            sm_kv[1][li] = Vec16<T>::pack(v);
         }
     }
     T* Kr = nullptr;
@@ -195,8 +206,8 @@ __global__ void __launch_bounds__(SWA_WARPS * 32) k_swa_decode(const float* __re
     st16(o + (long long)b * d + h * HD + li * EPL, Vec16<T>::pack(out));
     if (W > 1) {
         int slot = (t - 1) % (W - 1);
-        st16(Kr + (long long)slot * HD + li * EPL, Vec16<T>::pack(k));
-        st16(Vr + (long long)slot * HD + li * EPL, Vec16<T>::pack(v));
+        st16(Kr + (long long)slot * HD + li * EPL, sm_kv[0][li]);
+        st16(Vr + (long long)slot * HD + li * EPL, sm_kv[1][li]);
     }
 }
 
@@ -265,7 +276,7 @@ __global__ void k_attn_combine(const float* __restrict__ part, int n_splits, int
 }
 
 template <typename T, int HD>
-__global__ void __launch_bounds__(WARPS * 32) k_enc_attn(const T* __restrict__ planes, T* __restrict__ o,
+__global__ void __launch_bounds__(WARPS * 32, 8) k_enc_attn(const T* __restrict__ planes, T* __restrict__ o,
                                                          int B, int Tn, int H, float qscale) {
     using G = Geom<T, HD>;
     constexpr int EPL = G::EPL, LPK = G::LPK;

@@ -323,7 +323,49 @@ cudaError_t run_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int
     return launch_k(L, k_gemm_tc<BN, STAGES>, grid, 128, S::SMEM, ta, tw, M, N, K, epi, ea, hdr);
 }
 
+// Tile variants: (BN, stages) and how many CTAs fit on one SM (shared memory bound).
+struct TcVariant {
+    int bn, stages, per_sm;
+};
+constexpr TcVariant VARIANTS[] = {
+    {32, 5, 2},    // 100 KB
+    {64, 4, 2},    //  96 KB
+    {128, 3, 2},   //  96 KB
+    {128, 5, 1},   // 160 KB
+    {256, 4, 1},   // 192 KB
+};
+constexpr int N_VARIANTS = sizeof(VARIANTS) / sizeof(VARIANTS[0]);
+
+cudaError_t run_variant(int v, Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
+                        const EpiArgs& ea, DevHeader* hdr) {
+    switch (v) {
+        case 0: return run_tc<32, 5>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 1: return run_tc<64, 4>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 2: return run_tc<128, 3>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 3: return run_tc<128, 5>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 4: return run_tc<256, 4>(L, epi, A, lda, W, M, N, K, ea, hdr);
+    }
+    return cudaErrorInvalidValue;
+}
+
+// One output tile per CTA and a latency-bound k-loop at decode sizes: the widest tile whose
+// grid still fits in one wave of co-resident CTAs wins; grids larger than a wave use the
+// widest tile.
+int pick_variant(int M, int N) {
+    long long mt = (M + BM - 1) / BM;
+    for (int v = N_VARIANTS - 1; v >= 0; --v) {
+        const TcVariant& t = VARIANTS[v];
+        long long tiles = mt * ((N + t.bn - 1) / t.bn);
+        if (tiles <= 148LL * t.per_sm && tiles >= 74) return v;
+    }
+    long long tiles256 = mt * ((N + 255) / 256);
+    if (tiles256 > 148) return 4;
+    return 0;
+}
+
 }  // namespace
+
+int gemm_tc_variants() { return N_VARIANTS; }
 
 bool gemm_tc_supported(const void* A, int lda, const void* W, int K) {
     // TMA: 16-byte aligned base addresses and row pitches
@@ -332,13 +374,9 @@ bool gemm_tc_supported(const void* A, int lda, const void* W, int K) {
 }
 
 cudaError_t launch_gemm_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
-                           const EpiArgs& ea, DevHeader* hdr) {
-    // Pick the widest tile that still gives at least one wave of CTAs over the 148 SMs.
-    long long mt = (M + BM - 1) / BM;
-    auto tiles = [&](int bn) { return mt * ((N + bn - 1) / bn); };
-    if (tiles(128) >= 148) return run_tc<128, 4>(L, epi, A, lda, W, M, N, K, ea, hdr);
-    if (tiles(64) >= 148) return run_tc<64, 6>(L, epi, A, lda, W, M, N, K, ea, hdr);
-    return run_tc<32, 8>(L, epi, A, lda, W, M, N, K, ea, hdr);
+                           const EpiArgs& ea, DevHeader* hdr, int variant) {
+    int v = (variant >= 0 && variant < N_VARIANTS) ? variant : pick_variant(M, N);
+    return run_variant(v, L, epi, A, lda, W, M, N, K, ea, hdr);
 }
 
 }  // namespace rlt

@@ -99,8 +99,10 @@ cudaError_t launch_gemm_simt(Launch L, Epi epi, const T* A, int lda, const T* W,
 
 // ------------------------------------------------------------------ gemm_tc.cu
 bool gemm_tc_supported(const void* A, int lda, const void* W, int K);
+int gemm_tc_variants();
+// variant < 0: pick the tile shape from (M, N); otherwise force tile variant `variant`.
 cudaError_t launch_gemm_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
-                           const EpiArgs& ea, DevHeader* hdr);
+                           const EpiArgs& ea, DevHeader* hdr, int variant = -1);
 
 // ------------------------------------------------------------------ attention.cu
 // Decoder sliding-window self-attention for one layer at step t (1-based): RoPE at

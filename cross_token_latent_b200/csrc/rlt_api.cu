@@ -667,7 +667,8 @@ uint64_t rlt_launch_count(const rlt_model* m) { return m ? m->launches : 0; }
 
 rlt_status rlt_gemm_bf16(rlt_model* m, const void* A, const void* W, float* C, int M, int N, int K, int kernel,
                          void* stream) {
-    if (!m || !A || !W || !C || M < 1 || N < 1 || K < 1 || (kernel != 0 && kernel != 1)) return RLT_EINVAL;
+    if (!m || !A || !W || !C || M < 1 || N < 1 || K < 1 || kernel < 0 || kernel > 1 + gemm_tc_variants())
+        return RLT_EINVAL;
     if (!aligned(A, 16) || !aligned(W, 16) || !aligned(C, 16) || K % 8 || N % 4) return RLT_EINVAL;
     Launch L = m->launch(stream);
     EpiArgs ea;
@@ -676,8 +677,8 @@ rlt_status rlt_gemm_bf16(rlt_model* m, const void* A, const void* W, float* C, i
     ea.ld_out = N;
     const bf16* a = reinterpret_cast<const bf16*>(A);
     const bf16* w = reinterpret_cast<const bf16*>(W);
-    CK(kernel == 0 ? launch_gemm_tc(L, Epi::StoreF32, a, K, w, M, N, K, ea, m->hdr())
-                   : launch_gemm_simt<bf16>(L, Epi::StoreF32, a, K, w, M, N, K, ea));
+    CK(kernel == 1 ? launch_gemm_simt<bf16>(L, Epi::StoreF32, a, K, w, M, N, K, ea)
+                   : launch_gemm_tc(L, Epi::StoreF32, a, K, w, M, N, K, ea, m->hdr(), kernel - 2));
     return RLT_OK;
 }
 
