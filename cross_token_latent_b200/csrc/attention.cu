@@ -213,9 +213,10 @@ __global__ void __launch_bounds__(SWA_WARPS * 32, 6) k_swa_decode(const float* _
 
 template <typename T, int HD>
 __global__ void __launch_bounds__(WARPS * 32) k_xattn_decode(const float* __restrict__ qc,
-                                                             const T* __restrict__ Mg, int T_alloc, int t,
-                                                             T* __restrict__ o, int B, int H, int n_splits,
-                                                             int chunk, float* __restrict__ part, float qscale) {
+                                                             const T* __restrict__ Mg, long long plane,
+                                                             int T_alloc, int t, T* __restrict__ o, int B, int H,
+                                                             int n_splits, int chunk, float* __restrict__ part,
+                                                             float qscale) {
     using G = Geom<T, HD>;
     constexpr int EPL = G::EPL, LPK = G::LPK;
     pdl_wait();
@@ -230,7 +231,6 @@ __global__ void __launch_bounds__(WARPS * 32) k_xattn_decode(const float* __rest
     const float* qr = qc + (long long)b * d + h * HD + li * EPL;
 #pragma unroll
     for (int i = 0; i < EPL; ++i) q[i] = qr[i] * qscale;
-    long long plane = (long long)B * H * T_alloc * HD;
     const T* K = Mg + (long long)bh * T_alloc * HD;
     const T* V = K + plane;
     int j0 = sp * chunk;
@@ -330,18 +330,18 @@ cudaError_t launch_swa_decode(Launch L, const float* qkv, const float2* rope_row
 }
 
 template <typename T>
-static cudaError_t xattn_main(Launch L, const float* qc, const T* Mg, int T_alloc, int t, T* o, int B, int H,
-                              int hd, int n_splits, int chunk, float* part) {
+static cudaError_t xattn_main(Launch L, const float* qc, const T* Mg, long long plane, int T_alloc, int t, T* o,
+                              int B, int H, int hd, int n_splits, int chunk, float* part) {
     RLT_HD_DISPATCH(hd, launch_k(L, k_xattn_decode<T, HD>, blocks_for((long long)B * H * n_splits), WARPS * 32, 0,
-                                 qc, Mg, T_alloc, t, o, B, H, n_splits, chunk, part, qscale_for(hd)));
+                                 qc, Mg, plane, T_alloc, t, o, B, H, n_splits, chunk, part, qscale_for(hd)));
 }
 
 template <typename T>
-cudaError_t launch_xattn_decode(Launch L, const float* qc, const T* Mg, int T_alloc, int t, T* o, int B,
-                                int H, int hd, int n_splits, float* part) {
+cudaError_t launch_xattn_decode(Launch L, const float* qc, const T* Mg, long long plane, int T_alloc, int t, T* o,
+                                int B, int H, int hd, int n_splits, float* part) {
     if (n_splits < 1) n_splits = 1;
     int chunk = (t + n_splits - 1) / n_splits;
-    cudaError_t e = xattn_main<T>(L, qc, Mg, T_alloc, t, o, B, H, hd, n_splits, chunk, part);
+    cudaError_t e = xattn_main<T>(L, qc, Mg, plane, T_alloc, t, o, B, H, hd, n_splits, chunk, part);
     if (e != cudaSuccess || n_splits == 1) return e;
     return launch_k(L, k_attn_combine<T>, (unsigned)(B * H), (unsigned)hd, 0, (const float*)part, n_splits, hd, H, o);
 }
@@ -355,8 +355,8 @@ cudaError_t launch_enc_attention(Launch L, const T* planes, T* o, int B, int Tn,
 #define RLT_INST(T)                                                                                    \
     template cudaError_t launch_swa_decode<T>(Launch, const float*, const float2*, T*, T*, int, int,   \
                                               int, int, int);                                          \
-    template cudaError_t launch_xattn_decode<T>(Launch, const float*, const T*, int, int, T*, int, int, \
-                                                int, int, float*);                                     \
+    template cudaError_t launch_xattn_decode<T>(Launch, const float*, const T*, long long, int, int, T*, int, \
+                                                int, int, int, float*);                                \
     template cudaError_t launch_enc_attention<T>(Launch, const T*, T*, int, int, int, int);
 RLT_INST(float)
 RLT_INST(bf16)

@@ -16,6 +16,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <unordered_map>
 
 #include "kernels.cuh"
 
@@ -307,6 +308,39 @@ bool make_map(CUtensorMap* map, const void* ptr, int rows, int cols, int ld, int
     return r == CUDA_SUCCESS;
 }
 
+// Host cache of encoded tensor maps: weights and workspaces keep their addresses and shapes
+// across steps, so each (address, shape, box) is encoded once.
+struct MapKey {
+    const void* p;
+    int rows, cols, ld, box;
+    bool operator==(const MapKey& o) const {
+        return p == o.p && rows == o.rows && cols == o.cols && ld == o.ld && box == o.box;
+    }
+};
+struct MapKeyHash {
+    size_t operator()(const MapKey& k) const {
+        size_t h = std::hash<const void*>()(k.p);
+        for (int v : {k.rows, k.cols, k.ld, k.box}) h = h * 1000003u ^ std::hash<int>()(v);
+        return h;
+    }
+};
+
+bool cached_map(CUtensorMap* map, const void* ptr, int rows, int cols, int ld, int box_rows) {
+    static std::mutex mu;
+    static std::unordered_map<MapKey, CUtensorMap, MapKeyHash> cache;
+    MapKey k{ptr, rows, cols, ld, box_rows};
+    std::lock_guard<std::mutex> g(mu);
+    auto it = cache.find(k);
+    if (it != cache.end()) {
+        *map = it->second;
+        return true;
+    }
+    if (!make_map(map, ptr, rows, cols, ld, box_rows)) return false;
+    if (cache.size() > 8192) cache.clear();
+    cache.emplace(k, *map);
+    return true;
+}
+
 template <int BN, int STAGES>
 cudaError_t run_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K, const EpiArgs& ea,
                    DevHeader* hdr) {
@@ -318,7 +352,7 @@ cudaError_t run_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int
         attr_set = true;
     }
     CUtensorMap ta, tw;
-    if (!make_map(&ta, A, M, K, lda, BM) || !make_map(&tw, W, N, K, K, BN)) return cudaErrorInvalidValue;
+    if (!cached_map(&ta, A, M, K, lda, BM) || !cached_map(&tw, W, N, K, K, BN)) return cudaErrorInvalidValue;
     dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
     return launch_k(L, k_gemm_tc<BN, STAGES>, grid, 128, S::SMEM, ta, tw, M, N, K, epi, ea, hdr);
 }

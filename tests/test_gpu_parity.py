@@ -158,6 +158,26 @@ def test_small_bf16_parity_full_batch():
     assert np.abs(to_np(score)[sample] - score_r).max() <= BF16_LP_TOL * 4
 
 
+@pytest.mark.parametrize("B", [259, 256])
+def test_row_groups_on_two_streams_match_the_oracle(B):
+    """Large bf16 batches run each step as two row groups on two streams (ragged split for odd B);
+    every sequence of both groups must still match the oracle, and the step stays lockstep."""
+    cfg = replace(TINY.model, dtype="bf16", W=5, G=2)
+    w = make_weights(cfg, seed=3)
+    T = 20
+    tok = np.random.default_rng([5, B]).integers(0, cfg.V, size=(B, T)).astype(np.int32)
+    model = build_model(cfg, max_pos=T, weights=w)
+    _, _, s, lp, _, st = gpu_run(model, tok, tau=1.0)
+    assert st.position == T
+    sample = [0, 1, B // 2 - 1, B // 2, B // 2 + 1, B - 1]
+    _, _, s_r, lp_r = RLTOracle(cfg, w).run(tok[sample])
+    check(cfg, s[sample], lp[sample], s_r, lp_r)
+    # replay over the same batch agrees with stepping
+    score, lp_tok, _ = model.replay(torch.from_numpy(tok).cuda(), 8, 1.0, want_logp=True)
+    _, _, _, _, lp_step, _ = gpu_run(model, tok, full=False)
+    np.testing.assert_array_equal(to_np(lp_tok), lp_step)
+
+
 # ------------------------------------------------------------------ error handling at the boundary
 
 def test_errors_are_reported_not_hung(tiny):
