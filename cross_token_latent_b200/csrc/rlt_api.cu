@@ -145,21 +145,6 @@ struct rlt_model {
     std::vector<std::string> required;
     std::unordered_map<const void*, StateInfo> states;
     uint64_t launches = 0;
-    cudaStream_t side = nullptr;          // second stream for row groups of a decode step
-    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
-
-    bool side_stream_ready() {
-        if (side) return true;
-        if (cudaStreamCreateWithFlags(&side, cudaStreamNonBlocking) != cudaSuccess) return false;
-        if (cudaEventCreateWithFlags(&ev_fork, cudaEventDisableTiming) != cudaSuccess) return false;
-        if (cudaEventCreateWithFlags(&ev_join, cudaEventDisableTiming) != cudaSuccess) return false;
-        return true;
-    }
-    ~rlt_model() {
-        if (ev_fork) cudaEventDestroy(ev_fork);
-        if (ev_join) cudaEventDestroy(ev_join);
-        if (side) cudaStreamDestroy(side);
-    }
 
     DevHeader* hdr() const { return reinterpret_cast<DevHeader*>(arena); }
     template <typename T> T* at(size_t off) const { return reinterpret_cast<T*>(arena + off); }
@@ -341,139 +326,69 @@ struct StepIO {
     bool head = true;
 };
 
-// Within one lockstep step the batch may be split into row groups that run their kernel
-// chains on separate streams (the caller's stream and the model's side stream), joined at the
-// end of the step: one group's latency-bound projections then overlap another group's
-// bandwidth-bound attention.  Every group holds whole sequences, so results do not depend on
-// the split.
-int decode_groups(const rlt_config& c, int B) { return (c.dtype == RLT_BF16 && B >= 256) ? 2 : 1; }
-int group_rows(int B, int ng, int g) { return g < ng - 1 ? B / ng : B - (B / ng) * (ng - 1); }
-size_t dec_ws_total(const rlt_config& c, int B) {
-    int ng = decode_groups(c, B);
-    size_t tot = 0;
-    for (int g = 0; g < ng; ++g) tot += align_up(dec_ws(c, group_rows(B, ng, g)).total);
-    return tot;
-}
-
 template <typename T>
 rlt_status step_impl(rlt_model* m, uint8_t* state, int B, const T* e, const T* M, int T_alloc, int t,
                      const StepIO& io, uint8_t* ws, cudaStream_t st) {
     const rlt_config& c = m->cfg;
-    const int d = c.d, F = c.F, H = c.n_heads, hd = c.head_dim;
-    const int ng = decode_groups(c, B);
+    Launch L{st, &m->launches};
+    DecWS w = dec_ws(c, B);
+    int d = c.d, F = c.F, H = c.n_heads, hd = c.head_dim;
     StateHeader* sh = reinterpret_cast<StateHeader*>(state);
+    float* s = reinterpret_cast<float*>(state + state_s_off());
+    T* ring = reinterpret_cast<T*>(state + state_ring_off(c, B));
+    float* x = reinterpret_cast<float*>(ws + w.x);
+    T* A = reinterpret_cast<T*>(ws + w.A);
+    float* qkv = reinterpret_cast<float*>(ws + w.qkv);
+    T* att = reinterpret_cast<T*>(ws + w.att);
+    float* qc = reinterpret_cast<float*>(ws + w.qc);
+    T* act = reinterpret_cast<T*>(ws + w.act);
+    float* logits = reinterpret_cast<float*>(ws + w.logits);
+    float* part = reinterpret_cast<float*>(ws + w.part);
     const float2* rope_row = m->at<float2>(m->lay.rope) + (size_t)(t - 1) * (hd / 2);
-    const size_t group_elems = (size_t)2 * B * H * (size_t)T_alloc * hd;   // one memory group of M
-    const long long m_plane = (long long)B * H * T_alloc * hd;              // K plane -> V plane
-
-    struct Grp {
-        int b0, Bg, splits;
-        Launch L;
-        float *x, *qkv, *qc, *logits, *part, *s;
-        T *A, *att, *act, *ring;
-        const T *e, *M;
-        StepIO io;
-    } G[2];
-    if (ng > 1 && !m->side_stream_ready()) return RLT_ECUDA;
-    size_t woff = 0;
-    for (int g = 0, b0 = 0; g < ng; ++g) {
-        Grp& q = G[g];
-        q.b0 = b0;
-        q.Bg = group_rows(B, ng, g);
-        b0 += q.Bg;
-        q.L = Launch{g == 0 ? st : m->side, &m->launches};
-        DecWS w = dec_ws(c, q.Bg);
-        uint8_t* wg = ws + woff;
-        woff += align_up(w.total);
-        q.x = reinterpret_cast<float*>(wg + w.x);
-        q.A = reinterpret_cast<T*>(wg + w.A);
-        q.qkv = reinterpret_cast<float*>(wg + w.qkv);
-        q.att = reinterpret_cast<T*>(wg + w.att);
-        q.qc = reinterpret_cast<float*>(wg + w.qc);
-        q.act = reinterpret_cast<T*>(wg + w.act);
-        q.logits = reinterpret_cast<float*>(wg + w.logits);
-        q.part = reinterpret_cast<float*>(wg + w.part);
-        q.s = reinterpret_cast<float*>(state + state_s_off()) + (size_t)q.b0 * d;
-        q.ring = reinterpret_cast<T*>(state + state_ring_off(c, B)) + (size_t)q.b0 * 2 * H * (c.W - 1) * hd;
-        q.e = e + (size_t)q.b0 * T_alloc * d;
-        q.M = M + (size_t)q.b0 * H * T_alloc * hd;
-        q.splits = xattn_splits(c, q.Bg, t);
-        q.io = io;
-        if (io.tok) q.io.tok = io.tok + (size_t)q.b0 * io.tok_stride;
-        if (io.logp_tok) q.io.logp_tok = io.logp_tok + (size_t)q.b0 * io.lp_stride;
-        if (io.lse) q.io.lse = io.lse + q.b0;
-        if (io.logp_full) q.io.logp_full = io.logp_full + (size_t)q.b0 * c.V;
-        if (io.score) q.io.score = io.score + q.b0;
-        if (io.prompt_len) q.io.prompt_len = io.prompt_len + q.b0;
-    }
-    if (ng > 1) {
-        CK(cudaEventRecord(m->ev_fork, st));
-        CK(cudaStreamWaitEvent(m->side, m->ev_fork, 0));
-    }
-    const size_t ring_layer = ring_layer_elems(c, B);
+    size_t group_elems = (size_t)2 * B * H * (size_t)T_alloc * hd;
+    int splits = xattn_splits(c, B, t);
 
     // gated merge: x = e_t + sigmoid(W_ge e_t + W_gs s + b_g) * (W_fb s)
-    for (int g = 0; g < ng; ++g) {
-        Grp& q = G[g];
-        Launch L = q.L;
-        CKP(RLT_K_MERGE, launch_merge_prep<T>(L, q.e, T_alloc, t, q.s, q.A, q.Bg, d, g == 0 ? sh : nullptr,
-                                              m->version, m->hdr()));
+    CKP(RLT_K_MERGE, launch_merge_prep<T>(L, e, T_alloc, t, s, A, B, d, sh, m->version, m->hdr()));
+    {
         EpiArgs ea; ea.hdr = m->hdr();
-        ea.out_f32 = q.x; ea.ld_out = d; ea.merge_e = q.A; ea.ld_e = 2 * d; ea.bias = m->at<float>(m->lay.merge_b);
-        CKP(RLT_K_MERGE, launch_gemm<T>(L, Epi::Merge, q.A, 2 * d, m->at<T>(m->lay.merge_w), q.Bg, 2 * d, 2 * d, ea));
+        ea.out_f32 = x; ea.ld_out = d; ea.merge_e = A; ea.ld_e = 2 * d; ea.bias = m->at<float>(m->lay.merge_b);
+        CKP(RLT_K_MERGE, launch_gemm<T>(L, Epi::Merge, A, 2 * d, m->at<T>(m->lay.merge_w), B, 2 * d, 2 * d, ea));
     }
     for (int l = 0; l < c.L_D; ++l) {
-        for (int g = 0; g < ng; ++g) {
-            Grp& q = G[g];
-            Launch L = q.L;
-            const int Bg = q.Bg;
-            EpiArgs ea; ea.hdr = m->hdr();
-            // sliding-window self-attention (weights of encoder layer l)
-            CKP(RLT_K_NORM, launch_rmsnorm<T>(L, q.x, Bg, d, m->at<float>(m->lay.attn_norm[l]), c.rms_eps, q.A, d,
-                                              Bg, Bg, nullptr));
-            ea.out_f32 = q.qkv; ea.ld_out = 3 * d;
-            CKP(RLT_K_QKV, launch_gemm<T>(L, Epi::StoreF32, q.A, d, m->at<T>(m->lay.wqkv[l]), Bg, 3 * d, d, ea));
-            CKP(RLT_K_SWA, launch_swa_decode<T>(L, q.qkv, rope_row, q.ring + (size_t)l * ring_layer, q.att, Bg, H, hd,
-                                                c.W, t));
-            ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = q.x; ea.ld_out = d;
-            CKP(RLT_K_O, launch_gemm<T>(L, Epi::ResidAdd, q.att, d, m->at<T>(m->lay.wo[l]), Bg, d, d, ea));
-            // cross-attention to M_{<=t}
-            CKP(RLT_K_NORM, launch_rmsnorm<T>(L, q.x, Bg, d, m->at<float>(m->lay.xattn_norm[l]), c.rms_eps, q.A, d,
-                                              Bg, Bg, nullptr));
-            ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = q.qc; ea.ld_out = d;
-            CKP(RLT_K_QC, launch_gemm<T>(L, Epi::StoreF32, q.A, d, m->at<T>(m->lay.wqc[l]), Bg, d, d, ea));
-            const T* Mg = q.M + (c.G == 1 ? 0 : (size_t)l * group_elems);
-            CKP(RLT_K_XATTN, launch_xattn_decode<T>(L, q.qc, Mg, m_plane, T_alloc, t, q.att, Bg, H, hd, q.splits,
-                                                    q.part));
-            ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = q.x; ea.ld_out = d;
-            CKP(RLT_K_OC, launch_gemm<T>(L, Epi::ResidAdd, q.att, d, m->at<T>(m->lay.woc[l]), Bg, d, d, ea));
-            // SwiGLU FFN (weights of encoder layer l)
-            CKP(RLT_K_NORM, launch_rmsnorm<T>(L, q.x, Bg, d, m->at<float>(m->lay.ffn_norm[l]), c.rms_eps, q.A, d,
-                                              Bg, Bg, nullptr));
-            ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_t = q.act; ea.ld_out = F;
-            CKP(RLT_K_FFN_UP, launch_gemm<T>(L, Epi::SwiGLU, q.A, d, m->at<T>(m->lay.wgu[l]), Bg, 2 * F, d, ea));
-            ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = q.x; ea.ld_out = d;
-            CKP(RLT_K_FFN_DOWN, launch_gemm<T>(L, Epi::ResidAdd, q.act, F, m->at<T>(m->lay.wdown[l]), Bg, d, F, ea));
-        }
+        EpiArgs ea; ea.hdr = m->hdr();
+        // sliding-window self-attention (weights of encoder layer l)
+        CKP(RLT_K_NORM, launch_rmsnorm<T>(L, x, B, d, m->at<float>(m->lay.attn_norm[l]), c.rms_eps, A, d, B, B, nullptr));
+        ea.out_f32 = qkv; ea.ld_out = 3 * d;
+        CKP(RLT_K_QKV, launch_gemm<T>(L, Epi::StoreF32, A, d, m->at<T>(m->lay.wqkv[l]), B, 3 * d, d, ea));
+        CKP(RLT_K_SWA, launch_swa_decode<T>(L, qkv, rope_row, ring + (size_t)l * ring_layer_elems(c, B), att, B, H, hd,
+                                c.W, t));
+        ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = x; ea.ld_out = d;
+        CKP(RLT_K_O, launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.wo[l]), B, d, d, ea));
+        // cross-attention to M_{<=t}
+        CKP(RLT_K_NORM, launch_rmsnorm<T>(L, x, B, d, m->at<float>(m->lay.xattn_norm[l]), c.rms_eps, A, d, B, B, nullptr));
+        ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = qc; ea.ld_out = d;
+        CKP(RLT_K_QC, launch_gemm<T>(L, Epi::StoreF32, A, d, m->at<T>(m->lay.wqc[l]), B, d, d, ea));
+        const T* Mg = M + (c.G == 1 ? 0 : (size_t)l * group_elems);
+        CKP(RLT_K_XATTN, launch_xattn_decode<T>(L, qc, Mg, (long long)B * H * T_alloc * hd, T_alloc, t, att, B, H, hd,
+                                                splits, part));
+        ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = x; ea.ld_out = d;
+        CKP(RLT_K_OC, launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.woc[l]), B, d, d, ea));
+        // SwiGLU FFN (weights of encoder layer l)
+        CKP(RLT_K_NORM, launch_rmsnorm<T>(L, x, B, d, m->at<float>(m->lay.ffn_norm[l]), c.rms_eps, A, d, B, B, nullptr));
+        ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_t = act; ea.ld_out = F;
+        CKP(RLT_K_FFN_UP, launch_gemm<T>(L, Epi::SwiGLU, A, d, m->at<T>(m->lay.wgu[l]), B, 2 * F, d, ea));
+        ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = x; ea.ld_out = d;
+        CKP(RLT_K_FFN_DOWN, launch_gemm<T>(L, Epi::ResidAdd, act, F, m->at<T>(m->lay.wdown[l]), B, d, F, ea));
     }
-    for (int g = 0; g < ng; ++g) {
-        Grp& q = G[g];
-        Launch L = q.L;
-        // split: s_t = RMSNorm(x) becomes the state; the same s_t feeds the head
-        CKP(RLT_K_FINAL, launch_final_norm<T>(L, q.x, q.Bg, d, m->at<float>(m->lay.dec_norm), c.rms_eps, q.s, q.A,
-                                              g == 0 ? sh : nullptr, t));
-        if (io.head) {
-            EpiArgs ea; ea.hdr = m->hdr();
-            ea.out_f32 = q.logits; ea.ld_out = c.V;
-            CKP(RLT_K_HEAD, launch_gemm<T>(L, Epi::StoreF32, q.A, d, m->at<T>(m->lay.unembed), q.Bg, c.V, d, ea));
-            CKP(RLT_K_LSE, launch_lse_gather(L, q.logits, q.Bg, c.V, q.io.tau, q.io.tok, q.io.tok_stride,
-                                             q.io.logp_tok, q.io.lp_stride, q.io.lse, q.io.logp_full, q.io.score,
-                                             q.io.prompt_len, t, m->hdr()));
-        }
-    }
-    if (ng > 1) {
-        CK(cudaEventRecord(m->ev_join, m->side));
-        CK(cudaStreamWaitEvent(st, m->ev_join, 0));
+    // split: s_t = RMSNorm(x) becomes the state; the same s_t feeds the head
+    CKP(RLT_K_FINAL, launch_final_norm<T>(L, x, B, d, m->at<float>(m->lay.dec_norm), c.rms_eps, s, A, sh, t));
+    if (io.head) {
+        EpiArgs ea; ea.hdr = m->hdr();
+        ea.out_f32 = logits; ea.ld_out = c.V;
+        CKP(RLT_K_HEAD, launch_gemm<T>(L, Epi::StoreF32, A, d, m->at<T>(m->lay.unembed), B, c.V, d, ea));
+        CKP(RLT_K_LSE, launch_lse_gather(L, logits, B, c.V, io.tau, io.tok, io.tok_stride, io.logp_tok, io.lp_stride,
+                             io.lse, io.logp_full, io.score, io.prompt_len, t, m->hdr()));
     }
     return RLT_OK;
 }
@@ -650,7 +565,7 @@ rlt_status rlt_state_release(rlt_model* m, const void* state) {
 
 size_t rlt_decode_workspace_bytes(const rlt_model* m, int B) {
     if (!m || B < 1) return 0;
-    return dec_ws_total(m->cfg, B);
+    return dec_ws(m->cfg, B).total;
 }
 
 rlt_status rlt_decode_step(rlt_model* m, void* state, int B, const void* e, const void* M, int T_alloc,
@@ -663,7 +578,7 @@ rlt_status rlt_decode_step(rlt_model* m, void* state, int B, const void* e, cons
     int64_t t = it->second.t + 1;
     if (t > T_alloc || T_alloc > m->cfg.max_pos) return RLT_EINVAL;
     if (!aligned(e) || !aligned(M) || !aligned(ws)) return RLT_EINVAL;
-    if (ws_bytes < dec_ws_total(m->cfg, B)) return RLT_EINVAL;
+    if (ws_bytes < dec_ws(m->cfg, B).total) return RLT_EINVAL;
     if ((next_tok && !aligned(next_tok, 4)) || (logp_tok && !aligned(logp_tok, 4)) ||
         (lse && !aligned(lse, 4)) || (logp_full && !aligned(logp_full, 4)))
         return RLT_EINVAL;
@@ -684,7 +599,7 @@ rlt_status rlt_decode_step(rlt_model* m, void* state, int B, const void* e, cons
 size_t rlt_replay_workspace_bytes(const rlt_model* m, int B, int T) {
     if (!m || B < 1 || T < 1) return 0;
     const rlt_config& c = m->cfg;
-    size_t enc = enc_ws(c, B, T).total, dec = dec_ws_total(c, B);
+    size_t enc = enc_ws(c, B, T).total, dec = dec_ws(c, B).total;
     return replay_e_bytes(c, B, T) + replay_M_bytes(c, B, T) + rlt_state_bytes(m, B) + (enc > dec ? enc : dec);
 }
 
