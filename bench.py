@@ -94,6 +94,24 @@ def run_roofline_s(m, B: int, T: int, peaks: dict) -> float:
     return tot
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def rank_sequences(rank: int, B: int) -> range:
+    """Sequences of the seeded batch stream that rank `rank` decodes (B per rank, disjoint)."""
+    return range(rank * B, (rank + 1) * B)
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Slowest rank's time: the job's time.  Identity without a process group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -287,7 +305,7 @@ def main() -> int:
     w = make_weights(m, wl.weight_seed)
     model.load_weights(w)
     del w
-    tokens = make_tokens(wl, range(rank * B, (rank + 1) * B))
+    tokens = make_tokens(wl, rank_sequences(rank, B))
     tok = torch.from_numpy(tokens).to(dev)
     tok_tb = tok.t().contiguous()                        # row t = x_{t+1} of every sequence
     e, M = model.encode(tok)
@@ -345,9 +363,7 @@ def main() -> int:
     ms = ev0.elapsed_time(ev1)
     if world > 1:
         dist.barrier()
-        tmax = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
-        ms = float(tmax.item())
+    ms = max_over_ranks(ms, dev)
     ms_per_step = ms / args.steps
     value = world * B * T / (ms_per_step / 1e3)
 
@@ -397,11 +413,7 @@ def main() -> int:
         e2e_once()
         b.record()
         torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b)
-        if world > 1:
-            tm = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-            e_ms = float(tm.item())
+        e_ms = max_over_ranks(a.elapsed_time(b), dev)
         e2e = {"value": world * B * T / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": tokens.nbytes,
                "d2h_bytes_per_step": int(lp_host.numel() * 4), "ms_per_step": e_ms,
                "includes": "H2D tokens, rlt_encode, T rlt_decode_step calls, D2H log-probs"}
@@ -416,7 +428,7 @@ def main() -> int:
         model.replay(tok, P, wl.tau)
         b.record()
         torch.cuda.synchronize()
-        r_ms = a.elapsed_time(b)
+        r_ms = max_over_ranks(a.elapsed_time(b), dev)
         replay = {"value": world * B * T / (r_ms / 1e3), "unit": "tokens/s", "ms": r_ms,
                   "includes": "rlt_replay: encode + T steps + response scoring"}
     model.check_device_errors()
