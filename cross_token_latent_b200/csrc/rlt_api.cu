@@ -2,6 +2,7 @@
 // packing, the decoder-state registry and the encode / decode-step / replay drivers.
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <unordered_map>
 #include <unordered_set>
@@ -594,6 +595,55 @@ rlt_status rlt_decode_step(rlt_model* m, void* state, int B, const void* e, cons
                            (uint8_t*)ws, st);
     if (s == RLT_OK) it->second.t = t;
     return s;
+}
+
+// ---------------------------------------------------------------- decode step without allocation
+//
+// Scratch for rlt_decode_step_noalloc: a file-scope device array that every GPU which loads
+// this library holds until the process exits.  Its device address is looked up once per
+// device (cudaGetSymbolAddress with that device current); host code never passes the
+// array's host-side name to a kernel.
+}  // extern "C"
+
+namespace {
+constexpr size_t NOALLOC_SCRATCH_BYTES = size_t(32) << 20;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+
+constexpr int NOALLOC_MAX_DEVICES = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[NOALLOC_MAX_DEVICES] = {};
+
+rlt_status noalloc_scratch_for_current_device(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return RLT_ECUDA;
+    if (dev < 0 || dev >= NOALLOC_MAX_DEVICES) return RLT_EUNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return RLT_ECUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return RLT_OK;
+}
+}  // namespace
+
+extern "C" {
+
+rlt_status rlt_decode_step_noalloc(rlt_model* m, void* state, int B, const void* e, const void* M, int T_alloc,
+                                   const int32_t* next_tok, float tau, float* logp_tok, float* lse,
+                                   float* logp_full, void* stream) {
+    if (!m || B < 1) return RLT_EINVAL;
+    size_t need = rlt_decode_workspace_bytes(m, B);
+    if (need == 0) return RLT_EINVAL;
+    if (need > NOALLOC_SCRATCH_BYTES) return RLT_EUNSUPPORTED;   // batch too large for the static scratch
+    void* scratch = nullptr;
+    rlt_status st = noalloc_scratch_for_current_device(&scratch);
+    if (st != RLT_OK) return st;
+    // Every workspace buffer of a step is fully written before it is read, so nothing in the
+    // shared scratch has to start at zero.
+    return rlt_decode_step(m, state, B, e, M, T_alloc, next_tok, tau, logp_tok, lse, logp_full, scratch,
+                           NOALLOC_SCRATCH_BYTES, stream);
 }
 
 size_t rlt_replay_workspace_bytes(const rlt_model* m, int B, int T) {

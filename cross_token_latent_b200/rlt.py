@@ -58,6 +58,10 @@ _EXPORTS = {
                                        ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_float,
                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                        ctypes.c_size_t, ctypes.c_void_p]),
+    "rlt_decode_step_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
+                                               ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_float,
+                                               ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                               ctypes.c_void_p]),
     "rlt_replay_workspace_bytes": (ctypes.c_size_t, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int]),
     "rlt_replay": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
                                   ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -243,6 +247,16 @@ class RLTModel:
         _check(lib().rlt_decode_step(self.handle, _ptr(state.buf), B, _ptr(e), _ptr(M), e.shape[1], _ptr(next_tok),
                                      float(tau), _ptr(logp_tok), _ptr(lse), _ptr(logp_full), _ptr(ws), ws.numel(),
                                      _stream()), "rlt_decode_step")
+
+    def decode_step_noalloc(self, state: RLTState, e: torch.Tensor, M: torch.Tensor,
+                            next_tok: torch.Tensor | None = None, tau: float = 1.0,
+                            logp_tok: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                            logp_full: torch.Tensor | None = None) -> None:
+        """rlt_decode_step without a caller workspace: the step's scratch is the library's static
+        device array (see include/rlt.h for its size limit and the rules on overlapping calls)."""
+        _check(lib().rlt_decode_step_noalloc(self.handle, _ptr(state.buf), state.B, _ptr(e), _ptr(M), e.shape[1],
+                                             _ptr(next_tok), float(tau), _ptr(logp_tok), _ptr(lse), _ptr(logp_full),
+                                             _stream()), "rlt_decode_step_noalloc")
 
     def replay(self, tokens: torch.Tensor, prompt_len, tau: float = 1.0, want_logp: bool = False,
                want_state: bool = False):

@@ -177,6 +177,27 @@ rlt_status rlt_decode_step(rlt_model* m, void* state, int B, const void* e, cons
                            float* lse, float* logp_full, void* ws, size_t ws_bytes,
                            void* stream);
 
+/* Allocation-free variant of rlt_decode_step (no counterpart in the paper; a library
+ * convenience).  Some callers cannot allocate device memory at all: code that runs inside a
+ * host runtime which owns the whole device pool and hands out no allocator, or serving loops
+ * that must never enter an allocator once they are running.  This entry point takes the same
+ * arguments as rlt_decode_step minus the workspace: the step's scratch lives in one
+ * file-scope device array of 32 MiB (33554432 bytes) that every GPU which loads the library
+ * holds until the process exits.  The caller still passes the
+ * state, e, M and every output buffer.
+ *   - The first call on a device looks up the array's device address (once per device, with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the one array, and it keeps whatever the last call left there (no step
+ *     needs any of it to start at zero).  Calls that overlap on the GPU race on it: issue them
+ *     on one stream, or order them with events, one at a time.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine.
+ * Errors: RLT_EUNSUPPORTED when rlt_decode_workspace_bytes(m, B) exceeds the array (checked
+ * on the host before anything is launched); otherwise those of rlt_decode_step, plus
+ * RLT_ECUDA if the array's address cannot be obtained. */
+rlt_status rlt_decode_step_noalloc(rlt_model* m, void* state, int B, const void* e, const void* M,
+                                   int T_alloc, const int32_t* next_tok, float tau,
+                                   float* logp_tok, float* lse, float* logp_full, void* stream);
+
 /* ---------------------------------------------------------------- exact replay */
 
 /* Workspace bytes rlt_replay needs for B sequences of T tokens (e, M, a state and the
