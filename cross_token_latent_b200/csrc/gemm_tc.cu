@@ -163,22 +163,51 @@ __device__ __forceinline__ void epilogue16(Epi epi, const EpiArgs& ea, int m, in
     }
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int SPLIT>
 struct TcShape {
     static constexpr int B_BYTES = BN * BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int TMEM_COLS = BN < 32 ? 32 : BN;
-    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
+    // split-K: the owner CTA of a row band receives every rank's partial rows here
+    static constexpr int ROWS_PER_OWNER = BM / SPLIT;
+    static constexpr int RECV_BYTES = SPLIT > 1 ? BM * BN * 4 : 0;
+    static constexpr int SMEM = STAGES * STAGE_BYTES + RECV_BYTES + 1024 + 256;
 };
 
-template <int BN, int STAGES>
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory"); }
+__device__ __forceinline__ void cluster_arrive_release() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait_acquire() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
+// Store 16 floats into the shared memory of cluster CTA `rank` at the address that `local`
+// has in this CTA (distributed shared memory).
+__device__ __forceinline__ void dsmem_store16(const float* local, uint32_t rank, const float* v) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+#pragma unroll
+    for (int j = 0; j < 16; j += 4)
+        asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(remote + 4 * j), "f"(v[j]),
+                     "f"(v[j + 1]), "f"(v[j + 2]), "f"(v[j + 3])
+                     : "memory");
+}
+
+// SPLIT > 1: the grid's z dimension splits the k-blocks over a cluster of SPLIT CTAs that
+// compute the same output tile.  Each CTA accumulates its share in its own TMEM, then sends
+// every partial row to the CTA that owns the row band (BM / SPLIT rows per rank) through
+// distributed shared memory; the owner adds the SPLIT partials in rank order (the same order
+// for every element and every run) and applies the epilogue.
+template <int BN, int STAGES, int SPLIT>
 __global__ void __launch_bounds__(128, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW, int M, int N, int K,
           Epi epi, EpiArgs ea, DevHeader* hdr) {
-    using S = TcShape<BN, STAGES>;
+    using S = TcShape<BN, STAGES, SPLIT>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES);
+    float* recv = reinterpret_cast<float*>(smem + STAGES * S::STAGE_BYTES);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES + S::RECV_BYTES);
     uint64_t* empty = full + STAGES;
     uint64_t* done = empty + STAGES;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
@@ -186,8 +215,13 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
-    const int nkb = (K + BK - 1) / BK;
+    const int nkb_all = (K + BK - 1) / BK;
+    const uint32_t rank = SPLIT > 1 ? cluster_rank() : 0;
+    const int per = (nkb_all + SPLIT - 1) / SPLIT;
+    const int kb0 = min(nkb_all, (int)rank * per);
+    const int nkb = min(nkb_all, kb0 + per) - kb0;
     pdl_trigger();
+    if constexpr (SPLIT > 1) cluster_arrive_relaxed();     // peers may write here once all have started
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -218,19 +252,19 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         for (int kb = 0; kb < pre; ++kb) {
             uint8_t* a = smem + kb * S::STAGE_BYTES;
             mbar_expect_tx(&full[kb], S::STAGE_BYTES);
-            tma_load_2d(a + A_BYTES, &tmW, &full[kb], kb * BK, n0);
+            tma_load_2d(a + A_BYTES, &tmW, &full[kb], (kb0 + kb) * BK, n0);
         }
         pdl_wait();
         for (int kb = 0; kb < pre; ++kb)
-            tma_load_2d(smem + kb * S::STAGE_BYTES, &tmA, &full[kb], kb * BK, m0);
+            tma_load_2d(smem + kb * S::STAGE_BYTES, &tmA, &full[kb], (kb0 + kb) * BK, m0);
         for (int kb = pre; kb < nkb; ++kb) {
             int s = kb % STAGES;
             uint32_t ph = (kb / STAGES) & 1;
             if (!mbar_wait(&empty[s], ph ^ 1, &abort_flag)) { abort_flag = 1; break; }
             uint8_t* a = smem + s * S::STAGE_BYTES;
             mbar_expect_tx(&full[s], S::STAGE_BYTES);
-            tma_load_2d(a, &tmA, &full[s], kb * BK, m0);
-            tma_load_2d(a + A_BYTES, &tmW, &full[s], kb * BK, n0);
+            tma_load_2d(a, &tmA, &full[s], (kb0 + kb) * BK, m0);
+            tma_load_2d(a + A_BYTES, &tmW, &full[s], (kb0 + kb) * BK, n0);
         }
     } else if (warp == 1 && lane == 0) {
         // MMA issuer
@@ -247,26 +281,71 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                 umma(tmem, da + 2 * k, dw + 2 * k, idesc, (kb | k) != 0);
             umma_commit(&empty[s]);
         }
-        umma_commit(done);
+        if (nkb > 0) umma_commit(done);
     }
     __syncwarp();
     pdl_wait();
 
-    // epilogue: thread owns output row m0 + 32*warp + lane
-    bool ok = mbar_wait(done, 0, &abort_flag);
+    // epilogue: thread owns output row m0 + 32*warp + lane (a split rank with no k-blocks has
+    // issued no MMA and contributes zeros)
+    bool ok = nkb == 0 ? true : mbar_wait(done, 0, &abort_flag);
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
-    if (ok) {
-        const int m = m0 + warp * 32 + lane;
-        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    if constexpr (SPLIT == 1) {
+        if (ok) {
+            const int m = m0 + warp * 32 + lane;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 16) {
-            float v[16];
-            tmem_ld16(lane_base + c, v);
-            int n = n0 + c;
-            if (m < M && n < N) epilogue16(epi, ea, m, n, min(16, N - n), v);
+            for (int c = 0; c < BN; c += 16) {
+                float v[16];
+                tmem_ld16(lane_base + c, v);
+                int n = n0 + c;
+                if (m < M && n < N) epilogue16(epi, ea, m, n, min(16, N - n), v);
+            }
         }
-    } else if (lane == 0) {
+    } else {
+        // send this warp's 32 partial rows to the owner of their band
+        const int row = warp * 32 + lane;                        // row within the tile
+        const uint32_t owner = (uint32_t)(row / S::ROWS_PER_OWNER);
+        const int row_local = row - (int)owner * S::ROWS_PER_OWNER;
+        cluster_wait_acquire();                                  // every CTA of the cluster has started
+        if (ok) {
+#pragma unroll 1
+            for (int c = 0; c < BN; c += 16) {
+                float v[16];
+                if (nkb > 0) {
+                    tmem_ld16(lane_base + c, v);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) v[j] = 0.f;
+                }
+                dsmem_store16(recv + ((size_t)rank * S::ROWS_PER_OWNER + row_local) * BN + c, owner, v);
+            }
+        }
+        cluster_arrive_release();
+        cluster_wait_acquire();                                  // all partials have landed
+        if (ok && owner == rank) {
+            const int m = m0 + row;
+#pragma unroll 1
+            for (int c = 0; c < BN; c += 16) {
+                float v[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] = 0.f;
+                for (int src = 0; src < SPLIT; ++src) {
+                    const float4* p = reinterpret_cast<const float4*>(
+                        recv + ((size_t)src * S::ROWS_PER_OWNER + row_local) * BN + c);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        float4 q = p[j];
+                        v[4 * j] += q.x; v[4 * j + 1] += q.y; v[4 * j + 2] += q.z; v[4 * j + 3] += q.w;
+                    }
+                }
+                int n = n0 + c;
+                if (m < M && n < N) epilogue16(epi, ea, m, n, min(16, N - n), v);
+            }
+        }
+    }
+    if (!ok && lane == 0) {
         abort_flag = 1;
         raise_flag(hdr, ERR_TIMEOUT);
     }
@@ -341,60 +420,105 @@ bool cached_map(CUtensorMap* map, const void* ptr, int rows, int cols, int ld, i
     return true;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int SPLIT>
 cudaError_t run_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K, const EpiArgs& ea,
                    DevHeader* hdr) {
-    using S = TcShape<BN, STAGES>;
+    using S = TcShape<BN, STAGES, SPLIT>;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
+        cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN, STAGES, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             S::SMEM);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
     CUtensorMap ta, tw;
     if (!cached_map(&ta, A, M, K, lda, BM) || !cached_map(&tw, W, N, K, K, BN)) return cudaErrorInvalidValue;
-    dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
-    return launch_k(L, k_gemm_tc<BN, STAGES>, grid, 128, S::SMEM, ta, tw, M, N, K, epi, ea, hdr);
+    dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, SPLIT);
+    if constexpr (SPLIT == 1) {
+        return launch_k(L, k_gemm_tc<BN, STAGES, 1>, grid, 128, S::SMEM, ta, tw, M, N, K, epi, ea, hdr);
+    } else {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = grid;
+        cfg.blockDim = dim3(128);
+        cfg.dynamicSmemBytes = S::SMEM;
+        cfg.stream = L.stream;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 1;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = SPLIT;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        *L.count += 1;
+        return cudaLaunchKernelEx(&cfg, k_gemm_tc<BN, STAGES, SPLIT>, ta, tw, M, N, K, epi, ea, hdr);
+    }
 }
 
-// Tile variants: (BN, stages) and how many CTAs fit on one SM (shared memory bound).
+// Tile variants: (BN, stages, k-split over a cluster) and how many CTAs fit on one SM.
 struct TcVariant {
-    int bn, stages, per_sm;
+    int bn, stages, per_sm, split;
 };
 constexpr TcVariant VARIANTS[] = {
-    {32, 5, 2},    // 100 KB
-    {64, 4, 2},    //  96 KB
-    {128, 3, 2},   //  96 KB
-    {128, 5, 1},   // 160 KB
-    {256, 4, 1},   // 192 KB
+    {32, 5, 2, 1},     // 100 KB
+    {64, 4, 2, 1},     //  96 KB
+    {128, 3, 2, 1},    //  96 KB
+    {128, 5, 1, 1},    // 160 KB
+    {256, 4, 1, 1},    // 192 KB
+    {128, 4, 1, 2},    // 128 KB + 64 KB partials
+    {128, 4, 1, 4},
+    {64, 4, 1, 2},     //  96 KB + 32 KB partials
+    {64, 4, 1, 4},
 };
 constexpr int N_VARIANTS = sizeof(VARIANTS) / sizeof(VARIANTS[0]);
 
 cudaError_t run_variant(int v, Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                         const EpiArgs& ea, DevHeader* hdr) {
     switch (v) {
-        case 0: return run_tc<32, 5>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 1: return run_tc<64, 4>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 2: return run_tc<128, 3>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 3: return run_tc<128, 5>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 4: return run_tc<256, 4>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 0: return run_tc<32, 5, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 1: return run_tc<64, 4, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 2: return run_tc<128, 3, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 3: return run_tc<128, 5, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 4: return run_tc<256, 4, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 5: return run_tc<128, 4, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 6: return run_tc<128, 4, 4>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 7: return run_tc<64, 4, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 8: return run_tc<64, 4, 4>(L, epi, A, lda, W, M, N, K, ea, hdr);
     }
     return cudaErrorInvalidValue;
 }
 
-// One output tile per CTA and a latency-bound k-loop at decode sizes: the widest tile whose
-// grid still fits in one wave of co-resident CTAs wins; grids larger than a wave use the
+// At decode sizes one CTA per output tile leaves a latency-bound k-loop: the widest
+// unsplit tile whose grid fits in one wave (and keeps at least half the SMs busy) with at most
+// 16 k-blocks per CTA wins; otherwise the k-blocks are split over a cluster so that the grid
+// fills one wave with as few k-blocks per CTA as possible.  Grids larger than a wave use the
 // widest tile.
-int pick_variant(int M, int N) {
+int pick_variant(int M, int N, int K) {
     long long mt = (M + BM - 1) / BM;
-    for (int v = N_VARIANTS - 1; v >= 0; --v) {
+    int nkb = (K + BK - 1) / BK;
+    for (int v = 4; v >= 0; --v) {
         const TcVariant& t = VARIANTS[v];
         long long tiles = mt * ((N + t.bn - 1) / t.bn);
-        if (tiles <= 148LL * t.per_sm && tiles >= 74) return v;
+        if (tiles <= 148LL * t.per_sm && tiles >= 74 && nkb <= 16) return v;
     }
     long long tiles256 = mt * ((N + 255) / 256);
     if (tiles256 > 148) return 4;
-    return 0;
+    int best = -1;
+    long long best_ctas = 0;
+    for (int v = 5; v < N_VARIANTS; ++v) {
+        const TcVariant& t = VARIANTS[v];
+        long long ctas = mt * ((N + t.bn - 1) / t.bn) * t.split;
+        if (ctas > 148 || t.split > nkb) continue;
+        if (ctas > best_ctas) { best = v; best_ctas = ctas; }
+    }
+    if (best >= 0 && best_ctas >= 64) return best;
+    // fall back to the unsplit tile with the most CTAs within a wave
+    for (int v = 0; v <= 4; ++v) {
+        const TcVariant& t = VARIANTS[v];
+        if (mt * ((N + t.bn - 1) / t.bn) <= 148LL * t.per_sm) return v;
+    }
+    return 4;
 }
 
 }  // namespace
@@ -409,7 +533,7 @@ bool gemm_tc_supported(const void* A, int lda, const void* W, int K) {
 
 cudaError_t launch_gemm_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                            const EpiArgs& ea, DevHeader* hdr, int variant) {
-    int v = (variant >= 0 && variant < N_VARIANTS) ? variant : pick_variant(M, N);
+    int v = (variant >= 0 && variant < N_VARIANTS) ? variant : pick_variant(M, N, K);
     return run_variant(v, L, epi, A, lda, W, M, N, K, ea, hdr);
 }
 

@@ -49,8 +49,6 @@ def make(workload: str, seqs: list[int], steps: int, tag: str, s_every: int = 16
     s_keep = []
     for t in range(1, steps + 1):
         st, logp = ora.step(st, e[:, t - 1], M, wl.tau)
-        z_lse = (ora.head(st.s, wl.tau) - logp)  # not used: lse from the definition below
-        del z_lse
         zt = ora._lin(ora.rnd(st.s), ora.w["unembed"]) / wl.tau
         mx = zt.max(-1, keepdims=True)
         lse[:, t - 1] = (mx + np.log(np.exp(zt - mx).sum(-1, keepdims=True)))[:, 0]

@@ -27,7 +27,7 @@ def model():
     return build_model(TINY.model, max_pos=8)
 
 
-@pytest.mark.parametrize("kernel", [0, 2, 3, 4, 5, 6])
+@pytest.mark.parametrize("kernel", [0, 2, 3, 4, 5, 6, 7, 8, 9, 10])
 @pytest.mark.parametrize("M,N,K", SHAPES)
 def test_tcgen05_gemm_matches_float64(model, M, N, K, kernel):
     g = torch.Generator().manual_seed(M * 7919 + N * 31 + K)
@@ -45,10 +45,11 @@ def test_tcgen05_gemm_matches_float64(model, M, N, K, kernel):
         assert bool(((c_simt - ref).abs() <= 1e-4 * bound + 1e-6).all())
 
 
-def test_tcgen05_gemm_is_deterministic(model):
+@pytest.mark.parametrize("kernel", [0, 7, 8, 9, 10])
+def test_tcgen05_gemm_is_deterministic(model, kernel):
     g = torch.Generator().manual_seed(5)
     A = torch.randn(512, 1024, generator=g).to(torch.bfloat16)
     W = torch.randn(3072, 1024, generator=g).to(torch.bfloat16)
-    a = model.gemm_bf16(A, W)
-    b = model.gemm_bf16(A, W)
+    a = model.gemm_bf16(A, W, kernel=kernel)
+    b = model.gemm_bf16(A, W, kernel=kernel)
     assert torch.equal(a, b)
