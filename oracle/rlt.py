@@ -154,7 +154,11 @@ class RLTOracle:
         return round_bf16(x) if self.bf16 else x
 
     def _lin(self, x: np.ndarray, W: np.ndarray) -> np.ndarray:
-        return x @ W.T
+        """The linear map y = x W^T over the last axis.  For a few rows the product is taken
+        as (W x^T)^T, which BLAS runs several times faster for the same result."""
+        x2 = x.reshape(-1, x.shape[-1])
+        y = (W @ x2.T).T if x2.shape[0] <= 64 else x2 @ W.T
+        return y.reshape(*x.shape[:-1], W.shape[0])
 
     def _heads(self, x: np.ndarray) -> np.ndarray:
         return x.reshape(*x.shape[:-1], self.cfg.n_heads, self.cfg.head_dim)
