@@ -1,0 +1,333 @@
+// Encoder causal self-attention on the sm_100a tensor cores (bf16, head_dim 64 or 128).
+//
+// One CTA computes 128 queries of one (sequence, head) against the causal key range in tiles
+// of 128 keys, flash-attention style, with every operand K-major in the 128-byte swizzle
+// layout that TMA writes:
+//   warp 4, lane 0  TMA producer: the Q tile once, then K and V^T tiles into two stages;
+//   warp 5, lane 0  MMA issuer: S = Q K^T into TMEM columns [0, 128), then O += P V into TMEM
+//                   columns [128, 128 + head_dim) once the softmax warps have written P;
+//   warp 5          allocates / frees the 256 TMEM columns;
+//   warps 0-3       softmax: thread r owns query row r (TMEM lane r): causal mask on the
+//                   diagonal tile, running max, exp2, P rounded to bf16 into shared memory (the
+//                   row sum is taken over the rounded values, so P V / sum stays a convex
+//                   combination), rescale of O in TMEM when the max grows, and the epilogue
+//                   O / sum -> bf16.
+// V is stored transposed per (sequence, head) ([head_dim][T_pad], keys contiguous) so that it
+// is a K-major B operand like the others.  Every mbarrier wait is bounded.
+#include <cudaTypedefs.h>
+
+#include "kernels.cuh"
+#include "sm100.cuh"
+
+namespace rlt {
+
+namespace {
+
+constexpr int QT = 128;   // queries per CTA (UMMA M)
+constexpr int KT = 128;   // keys per tile (UMMA N of S and K of P V)
+
+template <int HD>
+struct FaShape {
+    static constexpr int ATOMS = HD / 64;                 // 64-element swizzle atoms along head_dim
+    static constexpr int Q_BYTES = QT * HD * 2;
+    static constexpr int K_BYTES = KT * HD * 2;
+    static constexpr int V_BYTES = HD * KT * 2;           // V^T tile: HD rows x 128 keys
+    static constexpr int P_BYTES = QT * KT * 2;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + Q_BYTES;         // 2 stages
+    static constexpr int OFF_V = OFF_K + 2 * K_BYTES;     // 2 stages
+    static constexpr int OFF_P = OFF_V + 2 * V_BYTES;
+    static constexpr int OFF_BAR = OFF_P + P_BYTES;
+    static constexpr int SMEM = OFF_BAR + 256 + 1024;
+    static constexpr int TMEM_COLS = 256;
+    static constexpr uint32_t S_COL = 0, O_COL = 128;
+};
+
+template <int HD>
+__global__ void __launch_bounds__(192, 1)
+k_enc_fa_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+            const __grid_constant__ CUtensorMap tmV, bf16* __restrict__ o, int B, int Tn, int H, float qscale,
+            DevHeader* hdr) {
+    using S = FaShape<HD>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
+    uint64_t* kv_full = q_full + 1;       // [2]
+    uint64_t* kv_empty = kv_full + 2;     // [2]
+    uint64_t* s_full = kv_empty + 2;
+    uint64_t* p_full = s_full + 1;
+    uint64_t* o_done = p_full + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
+    __shared__ int abort_flag;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_qt = (Tn + QT - 1) / QT;
+    const int qt = n_qt - 1 - (int)blockIdx.x;            // longest causal ranges first
+    const int bh = blockIdx.y;
+    const int q0 = qt * QT;
+    const int nt = qt + 1;                                 // key tiles 0..qt
+    pdl_trigger();
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(p_full, 128);
+        mbar_init(o_done, 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 5) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(S::TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 4) {
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(&tmQ) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(&tmK) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(&tmV) : "memory");
+            pdl_wait();
+            mbar_expect_tx(q_full, S::Q_BYTES);
+#pragma unroll
+            for (int a = 0; a < S::ATOMS; ++a) tma_load_3d(smem + S::OFF_Q + a * QT * 128, &tmQ, q_full, 64 * a, q0, bh);
+            for (int j = 0; j < nt; ++j) {
+                int s = j & 1;
+                uint32_t ph = (j >> 1) & 1;
+                if (!mbar_wait(&kv_empty[s], ph ^ 1, &abort_flag)) { abort_flag = 1; break; }
+                mbar_expect_tx(&kv_full[s], S::K_BYTES + S::V_BYTES);
+                uint8_t* kb = smem + S::OFF_K + s * S::K_BYTES;
+                uint8_t* vb = smem + S::OFF_V + s * S::V_BYTES;
+#pragma unroll
+                for (int a = 0; a < S::ATOMS; ++a) tma_load_3d(kb + a * KT * 128, &tmK, &kv_full[s], 64 * a, j * KT, bh);
+#pragma unroll
+                for (int a = 0; a < 2; ++a) tma_load_3d(vb + a * HD * 128, &tmV, &kv_full[s], j * KT + 64 * a, 0, bh);
+            }
+        }
+    } else if (warp == 5) {
+        if (lane == 0) {
+            constexpr uint32_t id_s = idesc_bf16(QT, KT), id_o = idesc_bf16(QT, HD);
+            const uint32_t tS = tmem + S::S_COL, tO = tmem + S::O_COL;
+            bool ok = mbar_wait(q_full, 0, &abort_flag) && mbar_wait(&kv_full[0], 0, &abort_flag);
+            if (ok) {
+                tc_fence_after();
+#pragma unroll
+                for (int a = 0; a < S::ATOMS; ++a) {
+                    uint64_t dq = sdesc_sw128(smem + S::OFF_Q + a * QT * 128);
+                    uint64_t dk = sdesc_sw128(smem + S::OFF_K + a * KT * 128);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) umma(tS, dq + 2 * k, dk + 2 * k, id_s, (a | k) != 0);
+                }
+                umma_commit(s_full);
+            }
+            for (int j = 0; ok && j < nt; ++j) {
+                int s = j & 1;
+                if (!mbar_wait(p_full, j & 1, &abort_flag)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                    uint64_t dp = sdesc_sw128(smem + S::OFF_P + a * QT * 128);
+                    uint64_t dv = sdesc_sw128(smem + S::OFF_V + s * S::V_BYTES + a * HD * 128);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) umma(tO, dp + 2 * k, dv + 2 * k, id_o, (j | a | k) != 0);
+                }
+                umma_commit(&kv_empty[s]);
+                umma_commit(o_done);
+                if (j + 1 < nt) {
+                    int s1 = (j + 1) & 1;
+                    if (!mbar_wait(&kv_full[s1], ((j + 1) >> 1) & 1, &abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int a = 0; a < S::ATOMS; ++a) {
+                        uint64_t dq = sdesc_sw128(smem + S::OFF_Q + a * QT * 128);
+                        uint64_t dk = sdesc_sw128(smem + S::OFF_K + s1 * S::K_BYTES + a * KT * 128);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) umma(tS, dq + 2 * k, dk + 2 * k, id_s, (a | k) != 0);
+                    }
+                    umma_commit(s_full);
+                }
+            }
+            if (!ok) abort_flag = 1;
+        }
+    } else {
+        // softmax warps: thread r owns query row r of the tile
+        const int r = threadIdx.x;                        // 0..127
+        const int q = q0 + r;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const uint32_t tS = tmem + S::S_COL + lane_off, tO = tmem + S::O_COL + lane_off;
+        uint8_t* P = smem + S::OFF_P;
+        float m = -1e30f, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nt; ++j) {
+            ok = ok && mbar_wait(s_full, j & 1, &abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            float sv[KT];
+#pragma unroll
+            for (int c = 0; c < KT; c += 32) tmem_ld32(tS + c, sv + c);
+            const bool diag = (j == nt - 1);
+            float mx = m;
+#pragma unroll
+            for (int c = 0; c < KT; ++c) {
+                float v = sv[c] * qscale;
+                if (diag && j * KT + c > q) v = -1e30f;
+                sv[c] = v;
+                mx = fmaxf(mx, v);
+            }
+            const float alpha = exp2f(m - mx);
+            float rowsum = 0.f;
+            // P_j overwrites P_{j-1}: wait until P_{j-1} V_{j-1} has completed (it also makes O final
+            // for the rescale below)
+            if (j > 0) {
+                ok = mbar_wait(o_done, (j - 1) & 1, &abort_flag);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                tc_fence_after();
+            }
+#pragma unroll
+            for (int a = 0; a < 2; ++a) {
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    float p8[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        float p = round_to<bf16>(exp2f(sv[a * 64 + ch * 8 + i] - mx));
+                        p8[i] = p;
+                        rowsum += p;
+                    }
+                    uint8_t* dst = P + a * QT * 128 + r * 128 + ((ch ^ (r & 7)) << 4);
+                    *reinterpret_cast<uint4*>(dst) = Vec16<bf16>::pack(p8);
+                }
+            }
+            l = l * alpha + rowsum;
+            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {     // warp-collective TMEM access
+#pragma unroll 1
+                for (int c = 0; c < HD; c += 32) {
+                    float ov[32];
+                    tmem_ld32(tO + c, ov);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+                    tmem_st32(tO + c, ov);
+                }
+            }
+            m = mx;
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(p_full);
+        }
+        pdl_wait();
+        if (ok) {
+            ok = mbar_wait(o_done, (nt - 1) & 1, &abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+        }
+        if (ok) {
+            tc_fence_after();
+            const float inv = 1.0f / l;
+            const int b = bh / H, h = bh % H;
+            bf16* orow = o + ((long long)b * Tn + q) * H * HD + h * HD;
+#pragma unroll 1
+            for (int c = 0; c < HD; c += 32) {
+                float ov[32];
+                tmem_ld32(tO + c, ov);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) ov[i] *= inv;
+                if (q < Tn) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) st16(orow + c + i, Vec16<bf16>::pack(ov + i));
+                }
+            }
+        } else if (lane == 0) {
+            abort_flag = 1;
+            raise_flag(hdr, ERR_TIMEOUT);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(S::TMEM_COLS));
+    }
+}
+
+// V^T planes: qkv float32 [B*T, 3d] (v at columns 2d + h*hd) -> vt [B][H][hd][Tp] bf16 via a
+// shared-memory tile transpose (32 positions x hd columns per block).
+template <int HD>
+__global__ void __launch_bounds__(256) k_enc_vt(const float* __restrict__ qkv, bf16* __restrict__ vt, int B, int Tn,
+                                                int H, int Tp) {
+    __shared__ float tile[32][HD + 1];
+    pdl_wait();
+    pdl_trigger();
+    const int p0 = blockIdx.x * 32, h = blockIdx.y, b = blockIdx.z;
+    const int d = H * HD;
+    for (int i = threadIdx.x; i < 32 * HD; i += blockDim.x) {
+        int pr = i / HD, c = i % HD;
+        int p = p0 + pr;
+        tile[pr][c] = p < Tn ? qkv[((long long)b * Tn + p) * 3 * d + 2 * d + h * HD + c] : 0.f;
+    }
+    __syncthreads();
+    bf16* base = vt + ((long long)b * H + h) * HD * Tp;
+    for (int i = threadIdx.x; i < 32 * HD; i += blockDim.x) {
+        int c = i / 32, pr = i % 32;
+        int p = p0 + pr;
+        if (p < Tp) base[(long long)c * Tp + p] = __float2bfloat16_rn(tile[pr][c]);
+    }
+}
+
+template <int HD>
+cudaError_t run_fa(Launch L, const bf16* q, const bf16* k, const bf16* vt, bf16* o, int B, int Tn, int H, int Tp,
+                   DevHeader* hdr) {
+    using S = FaShape<HD>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(k_enc_fa_tc<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    const uint64_t BH = (uint64_t)B * H;
+    CUtensorMap tq, tk, tv;
+    uint64_t qdims[3] = {(uint64_t)HD, (uint64_t)Tn, BH};
+    uint64_t qstr[2] = {(uint64_t)HD * 2, (uint64_t)Tn * HD * 2};
+    uint32_t qbox[3] = {64, QT, 1};
+    uint64_t vdims[3] = {(uint64_t)Tn, (uint64_t)HD, BH};
+    uint64_t vstr[2] = {(uint64_t)Tp * 2, (uint64_t)HD * Tp * 2};
+    uint32_t vbox[3] = {64, (uint32_t)HD, 1};
+    if (!tma_map_bf16(&tq, q, 3, qdims, qstr, qbox) || !tma_map_bf16(&tk, k, 3, qdims, qstr, qbox) ||
+        !tma_map_bf16(&tv, vt, 3, vdims, vstr, vbox))
+        return cudaErrorInvalidValue;
+    dim3 grid((Tn + QT - 1) / QT, (unsigned)BH);
+    const float qscale = 1.4426950408889634f / sqrtf((float)HD);
+    return launch_k(L, k_enc_fa_tc<HD>, grid, 192, S::SMEM, tq, tk, tv, o, B, Tn, H, qscale, hdr);
+}
+
+}  // namespace
+
+int enc_vt_pitch(int Tn) { return (Tn + 7) / 8 * 8; }
+
+bool enc_attention_tc_supported(int hd) { return hd == 64 || hd == 128; }
+
+cudaError_t launch_enc_vt(Launch L, const float* qkv, bf16* vt, int B, int Tn, int H, int hd) {
+    dim3 grid((unsigned)((enc_vt_pitch(Tn) + 31) / 32), (unsigned)H, (unsigned)B);
+    int Tp = enc_vt_pitch(Tn);
+    if (hd == 64) return launch_k(L, k_enc_vt<64>, grid, 256, 0, qkv, vt, B, Tn, H, Tp);
+    if (hd == 128) return launch_k(L, k_enc_vt<128>, grid, 256, 0, qkv, vt, B, Tn, H, Tp);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_enc_attention_tc(Launch L, const bf16* q, const bf16* k, const bf16* vt, bf16* o, int B, int Tn,
+                                    int H, int hd, DevHeader* hdr) {
+    int Tp = enc_vt_pitch(Tn);
+    if (hd == 64) return run_fa<64>(L, q, k, vt, o, B, Tn, H, Tp, hdr);
+    if (hd == 128) return run_fa<128>(L, q, k, vt, o, B, Tn, H, Tp, hdr);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace rlt

@@ -178,7 +178,7 @@ __global__ void k_lse_gather(const float* __restrict__ logits, int B, int V, flo
 // thread per (n, h, i < hd/2): rotate the pair (i, i + hd/2) of q and k, round q, k, v.
 template <typename T>
 __global__ void k_enc_qkv_layout(const float* __restrict__ qkv, int B, int Tn, int H, int hd,
-                                 const float2* __restrict__ rope, T* __restrict__ planes) {
+                                 const float2* __restrict__ rope, T* __restrict__ planes, bool write_v) {
     pdl_wait();
     pdl_trigger();
     int half = hd / 2;
@@ -201,8 +201,10 @@ __global__ void k_enc_qkv_layout(const float* __restrict__ qkv, int B, int Tn, i
         planes[o + f + half] = from_f<T>(qa * cs.y + qb * cs.x);
         planes[plane + o + f] = from_f<T>(ka * cs.x - kb * cs.y);
         planes[plane + o + f + half] = from_f<T>(ka * cs.y + kb * cs.x);
-        planes[2 * plane + o + f] = from_f<T>(row[2 * d + f]);
-        planes[2 * plane + o + f + half] = from_f<T>(row[2 * d + f + half]);
+        if (write_v) {
+            planes[2 * plane + o + f] = from_f<T>(row[2 * d + f]);
+            planes[2 * plane + o + f + half] = from_f<T>(row[2 * d + f + half]);
+        }
     }
 }
 
@@ -296,9 +298,9 @@ cudaError_t launch_lse_gather(Launch L, const float* logits, int B, int V, float
 
 template <typename T>
 cudaError_t launch_enc_qkv_layout(Launch L, const float* qkv, int B, int Tn, int H, int hd,
-                                  const float2* rope, T* planes) {
+                                  const float2* rope, T* planes, bool write_v) {
     return launch_k(L, k_enc_qkv_layout<T>, grid_for((long long)B * Tn * H * (hd / 2), 256), 256, 0, qkv, B, Tn, H,
-                    hd, rope, planes);
+                    hd, rope, planes, write_v);
 }
 
 template <typename T>
@@ -323,7 +325,7 @@ cudaError_t launch_state_init(Launch L, const float* s_star, int B, int d, float
     template cudaError_t launch_final_norm<T>(Launch, const float*, int, int, const float*, float,    \
                                               float*, T*, StateHeader*, int);                         \
     template cudaError_t launch_enc_qkv_layout<T>(Launch, const float*, int, int, int, int,           \
-                                                  const float2*, T*);                                 \
+                                                  const float2*, T*, bool);                           \
     template cudaError_t launch_mem_layout<T>(Launch, const float*, int, int, int, int, int, T*);
 RLT_INST(float)
 RLT_INST(bf16)

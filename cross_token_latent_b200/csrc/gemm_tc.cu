@@ -15,10 +15,12 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cstring>
 #include <mutex>
 #include <unordered_map>
 
 #include "kernels.cuh"
+#include "sm100.cuh"
 
 namespace rlt {
 
@@ -27,89 +29,6 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;                       // 64 bf16 = 128 bytes = one swizzle row
 constexpr int A_BYTES = BM * BK * 2;         // 16 KB
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint64_t globaltimer() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// Bounded wait for the phase with the given parity.  False on timeout or abort.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-    if (mbar_try(bar, parity)) return true;
-    uint64_t t0 = globaltimer();
-    while (true) {
-        if (mbar_try(bar, parity)) return true;
-        if (*abort) return false;
-        if (globaltimer() - t0 > WAIT_LIMIT_NS) return false;
-    }
-}
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
-        ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
-        : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// Shared-memory matrix descriptor: K-major operand tile in the 128-byte swizzle layout that
-// TMA writes (8-row groups of 1024 bytes).  Fields: start address >> 4 [0,14), leading byte
-// offset >> 4 [16,30) (unused for this layout), stride byte offset >> 4 [32,46) = 1024 B
-// between 8-row groups, descriptor version 1 [46,48), layout 2 = 128-byte swizzle [61,64).
-__device__ __forceinline__ uint64_t sdesc_sw128(const void* tile) {
-    uint64_t a = smem_u32(tile);
-    return ((a >> 4) & 0x3FFFull) | (1ull << 16) | ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
-}
-// Instruction descriptor of kind::f16: D float32 [4,6)=1, A bf16 [7,10)=1, B bf16 [10,13)=1,
-// both K-major, N >> 3 at [17,23), M >> 4 at [24,29).
-__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
-}
-__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc));
-}
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
-    uint32_t r[16];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-
 // Fused epilogue on 16 consecutive columns n..n+15 of row m (cnt of them inside N).
 __device__ __forceinline__ void epilogue16(Epi epi, const EpiArgs& ea, int m, int n, int cnt, const float* v) {
     switch (epi) {
@@ -173,26 +92,6 @@ struct TcShape {
     static constexpr int RECV_BYTES = SPLIT > 1 ? BM * BN * 4 : 0;
     static constexpr int SMEM = STAGES * STAGE_BYTES + RECV_BYTES + 1024 + 256;
 };
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-__device__ __forceinline__ void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory"); }
-__device__ __forceinline__ void cluster_arrive_release() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
-__device__ __forceinline__ void cluster_wait_acquire() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
-// Store 16 floats into the shared memory of cluster CTA `rank` at the address that `local`
-// has in this CTA (distributed shared memory).
-__device__ __forceinline__ void dsmem_store16(const float* local, uint32_t rank, const float* v) {
-    uint32_t remote;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
-#pragma unroll
-    for (int j = 0; j < 16; j += 4)
-        asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(remote + 4 * j), "f"(v[j]),
-                     "f"(v[j + 1]), "f"(v[j + 2]), "f"(v[j + 3])
-                     : "memory");
-}
 
 // SPLIT > 1: the grid's z dimension splits the k-blocks over a cluster of SPLIT CTAs that
 // compute the same output tile.  Each CTA accumulates its share in its own TMEM, then sends
@@ -419,6 +318,57 @@ bool cached_map(CUtensorMap* map, const void* ptr, int rows, int cols, int ld, i
     cache.emplace(k, *map);
     return true;
 }
+
+}  // namespace
+
+bool tma_map_bf16(CUtensorMap* map, const void* ptr, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+                  const uint32_t* box) {
+    struct Key {
+        const void* p;
+        int rank;
+        uint64_t d[5], s[4];
+        uint32_t b[5];
+        bool operator==(const Key& o) const { return std::memcmp(this, &o, sizeof(Key)) == 0; }
+    };
+    struct Hash {
+        size_t operator()(const Key& k) const {
+            const unsigned char* c = reinterpret_cast<const unsigned char*>(&k);
+            size_t h = 1469598103934665603ull;
+            for (size_t i = 0; i < sizeof(Key); ++i) h = (h ^ c[i]) * 1099511628211ull;
+            return h;
+        }
+    };
+    static std::mutex mu;
+    static std::unordered_map<Key, CUtensorMap, Hash> cache;
+    if (rank < 1 || rank > 5) return false;
+    Key k;
+    std::memset(&k, 0, sizeof(k));
+    k.p = ptr;
+    k.rank = rank;
+    for (int i = 0; i < rank; ++i) { k.d[i] = dims[i]; k.b[i] = box[i]; }
+    for (int i = 0; i + 1 < rank; ++i) k.s[i] = strides_bytes[i];
+    std::lock_guard<std::mutex> g(mu);
+    auto it = cache.find(k);
+    if (it != cache.end()) {
+        *map = it->second;
+        return true;
+    }
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t gd[5], gs[4];
+    cuuint32_t bx[5], es[5];
+    for (int i = 0; i < rank; ++i) { gd[i] = dims[i]; bx[i] = box[i]; es[i] = 1; }
+    for (int i = 0; i + 1 < rank; ++i) gs[i] = strides_bytes[i];
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), gd, gs, bx, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return false;
+    if (cache.size() > 8192) cache.clear();
+    cache.emplace(k, *map);
+    return true;
+}
+
+namespace {
 
 template <int BN, int STAGES, int SPLIT>
 cudaError_t run_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K, const EpiArgs& ea,

@@ -63,10 +63,11 @@ cudaError_t launch_lse_gather(Launch L, const float* logits, int B, int V, float
                               const int32_t* tok, int tok_stride, float* logp_tok, int lp_stride,
                               float* lse, float* logp_full, float* score, const int32_t* prompt_len,
                               int t, DevHeader* hdr);
-// Encoder q/k/v: qkv float32 [B*T, 3d] -> planes T [3][B][H][T][hd], RoPE on q and k.
+// Encoder q/k/v: qkv float32 [B*T, 3d] -> planes T [3][B][H][T][hd], RoPE on q and k; the v
+// plane is skipped when write_v is false (the tensor-core path writes V transposed instead).
 template <typename T>
 cudaError_t launch_enc_qkv_layout(Launch L, const float* qkv, int B, int Tn, int H, int hd,
-                                  const float2* rope, T* planes);
+                                  const float2* rope, T* planes, bool write_v = true);
 // Memory projection output float32 [B*T, 2d] -> M_g T [2][B][H][T_alloc][hd]
 template <typename T>
 cudaError_t launch_mem_layout(Launch L, const float* kv, int B, int Tn, int T_alloc, int H, int hd,
@@ -120,5 +121,14 @@ cudaError_t launch_xattn_decode(Launch L, const float* qc, const T* Mg, long lon
 // Encoder causal self-attention: planes T [3][B][H][T][hd] -> o T [B*T, d]
 template <typename T>
 cudaError_t launch_enc_attention(Launch L, const T* planes, T* o, int B, int Tn, int H, int hd);
+
+// ------------------------------------------------------------------ attention_tc.cu
+// Tensor-core encoder attention (bf16, head_dim 64 or 128): q, k planes [B][H][T][hd] and the
+// transposed values vt [B][H][hd][enc_vt_pitch(T)] -> o [B*T, d].
+bool enc_attention_tc_supported(int hd);
+int enc_vt_pitch(int Tn);
+cudaError_t launch_enc_vt(Launch L, const float* qkv, bf16* vt, int B, int Tn, int H, int hd);
+cudaError_t launch_enc_attention_tc(Launch L, const bf16* q, const bf16* k, const bf16* vt, bf16* o, int B, int Tn,
+                                    int H, int hd, DevHeader* hdr);
 
 }  // namespace rlt

@@ -230,7 +230,9 @@ EncWS enc_ws(const rlt_config& c, int B, int T) {
     w.a = take(N * d * e);
     w.act = take(N * (size_t)c.F * e);
     w.qkv = take(N * 3 * d * 4);
-    w.planes = take(3 * N * d * e);
+    // q and k planes, then v ([B][H][T][hd]) or, on the tensor-core path, v transposed
+    // ([B][H][hd][T_pad])
+    w.planes = take(2 * N * d * e + (size_t)B * c.n_heads * c.head_dim * enc_vt_pitch(T) * e);
     w.att = take(N * d * e);
     w.ews = take(N * d * e);
     w.total = off;
@@ -285,14 +287,24 @@ rlt_status encode_impl(rlt_model* m, const int32_t* tokens, int B, int Tn, int T
     T* att = reinterpret_cast<T*>(ws + w.att);
     T* ews = reinterpret_cast<T*>(ws + w.ews);
     const float2* rope = m->at<float2>(m->lay.rope);
+    const bool use_tc_attn = sizeof(T) == 2 && enc_attention_tc_supported(hd);
     CK(launch_embed<T>(L, tokens, N, m->at<T>(m->lay.embed), c.V, d, h, m->hdr()));
     for (int l = 0; l < c.L_E; ++l) {
         EpiArgs ea; ea.hdr = m->hdr();
         CK(launch_rmsnorm<T>(L, h, N, d, m->at<float>(m->lay.attn_norm[l]), c.rms_eps, a, d, N, N, nullptr));
         ea.out_f32 = qkv; ea.ld_out = 3 * d;
         CK(launch_gemm<T>(L, Epi::StoreF32, a, d, m->at<T>(m->lay.wqkv[l]), N, 3 * d, d, ea));
-        CK(launch_enc_qkv_layout<T>(L, qkv, B, Tn, H, hd, rope, planes));
-        CK(launch_enc_attention<T>(L, planes, att, B, Tn, H, hd));
+        if (use_tc_attn) {
+            bf16* pl = reinterpret_cast<bf16*>(planes);
+            size_t plane = (size_t)N * d;
+            CK(launch_enc_qkv_layout<T>(L, qkv, B, Tn, H, hd, rope, planes, false));
+            CK(launch_enc_vt(L, qkv, pl + 2 * plane, B, Tn, H, hd));
+            CK(launch_enc_attention_tc(L, pl, pl + plane, pl + 2 * plane, reinterpret_cast<bf16*>(att), B, Tn, H, hd,
+                                       m->hdr()));
+        } else {
+            CK(launch_enc_qkv_layout<T>(L, qkv, B, Tn, H, hd, rope, planes));
+            CK(launch_enc_attention<T>(L, planes, att, B, Tn, H, hd));
+        }
         ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = h; ea.ld_out = d;
         CK(launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.wo[l]), N, d, d, ea));
         CK(launch_rmsnorm<T>(L, h, N, d, m->at<float>(m->lay.ffn_norm[l]), c.rms_eps, a, d, N, N, nullptr));

@@ -140,6 +140,24 @@ def test_variant_parity(name, B, T):
     check(cfg, s, lp, s_r, lp_r)
 
 
+@pytest.mark.parametrize("hd,T", [(64, 300), (128, 300), (64, 129), (128, 257)])
+def test_tensor_core_encoder_attention_over_several_key_tiles(hd, T):
+    """bf16 head_dim 64/128 encoders run causal attention on the tensor cores in 128x128 tiles:
+    several query and key tiles, ragged last tiles, online rescaling across tiles."""
+    cfg = replace(TINY.model, dtype="bf16", d=128, n_heads=128 // hd, head_dim=hd, F=256, W=6)
+    w = make_weights(cfg, seed=5)
+    tok = np.random.default_rng([13, hd, T]).integers(0, cfg.V, size=(2, T)).astype(np.int32)
+    model = build_model(cfg, max_pos=T, weights=w)
+    e_r, M_r = RLTOracle(cfg, w).encode(tok)
+    e, M = model.encode(torch.from_numpy(tok).cuda())
+    assert cosine(to_np(e), e_r).min() >= 0.999
+    assert cosine(m_layout(M, T), M_r).min() >= 0.999
+    steps = 40 if T > 200 else T
+    _, _, s, lp, _, _ = gpu_run(model, tok, steps=steps)
+    _, _, s_r, lp_r = RLTOracle(cfg, w).run(tok, steps=steps)
+    check(cfg, s, lp, s_r, lp_r)
+
+
 # ------------------------------------------------------------------ small bf16 workload (full batch)
 
 def test_small_bf16_parity_full_batch():
