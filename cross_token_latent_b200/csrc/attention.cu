@@ -107,71 +107,30 @@ __device__ __forceinline__ void merge_groups(float& m, float& l, float* acc) {
     }
 }
 
-// One CTA of SWA_WARPS warps per (sequence, head).  Thread 0 streams the n = min(t-1, W-1)
-// cached keys and values into shared memory with bulk asynchronous copies, 8 KB of keys (and
-// of values) per chunk through SWA_NBUF buffers (mbarrier-tracked, bounded waits), so a CTA's
-// ring is in flight after one round trip.  Every warp computes q (RoPE at position t-1) and attends over
-// its quarter of each chunk; warp 0 also takes the current token (k_t, v_t rounded to the
-// storage type, as cached).  The warps' partial softmax states are merged through shared
-// memory; then warp 0 writes the output and stores k_t, v_t into ring slot (t-1) mod (W-1) --
-// after every read of the ring, so the slot's old entry (token t-W+1, still in the window) is
-// used first.
+// One CTA of SWA_WARPS warps per (sequence, head).  Every warp computes q and the current
+// k/v (RoPE at position t-1); warp w streams a contiguous share of the n = min(t-1, W-1)
+// cached entries; the warps' partial softmax states are merged through shared memory, then
+// warp 0 writes the output and stores k_t, v_t into ring slot (t-1) mod (W-1) (after every
+// warp has read the ring, so the slot's old entry -- token t-W+1, still in the window -- is
+// used first).
 constexpr int SWA_WARPS = 4;
-constexpr int SWA_CHUNK_BYTES = 8192;
-constexpr int SWA_NBUF = 2;
-constexpr uint64_t SWA_WAIT_NS = 2000000000ull;
-
-__device__ __forceinline__ uint32_t smem_addr(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 
 template <typename T, int HD>
-__global__ void __launch_bounds__(SWA_WARPS * 32) k_swa_decode(const float* __restrict__ qkv,
-                                                               const float2* __restrict__ rope_row,
-                                                               T* __restrict__ ring, T* __restrict__ o,
-                                                               int B, int H, int W, int t, float qscale,
-                                                               DevHeader* hdr) {
+__global__ void __launch_bounds__(SWA_WARPS * 32, 6) k_swa_decode(const float* __restrict__ qkv,
+                                                                  const float2* __restrict__ rope_row,
+                                                                  T* __restrict__ ring, T* __restrict__ o,
+                                                                  int B, int H, int W, int t, float qscale) {
     using G = Geom<T, HD>;
     constexpr int EPL = G::EPL, LPK = G::LPK;
-    constexpr int SWA_CHUNK = SWA_CHUNK_BYTES / (HD * (int)sizeof(T));   // keys per chunk
-    constexpr int CHUNK_ELEMS = SWA_CHUNK * HD;
-    __shared__ __align__(128) T sm_k[SWA_NBUF][CHUNK_ELEMS];
-    __shared__ __align__(128) T sm_v[SWA_NBUF][CHUNK_ELEMS];
-    __shared__ __align__(8) uint64_t full[SWA_NBUF];
     __shared__ float sm_m[SWA_WARPS], sm_l[SWA_WARPS];
     __shared__ __align__(16) float sm_acc[SWA_WARPS][HD];
     __shared__ __align__(16) uint4 sm_kv[2][LPK];      // current k_t, v_t in storage type
-    __shared__ int failed;
     pdl_wait();
     pdl_trigger();
     const int item = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane / LPK, li = lane % LPK;
     const int b = item / H, h = item % H;
     const int d = H * HD, half = HD / 2;
-    const int n = W > 1 ? min(t - 1, W - 1) : 0;
-    const int nchunks = (n + SWA_CHUNK - 1) / SWA_CHUNK;
-    T* Kr = ring + (((long long)b * 2 + 0) * H + h) * (long long)(W > 1 ? W - 1 : 0) * HD;
-    T* Vr = ring + (((long long)b * 2 + 1) * H + h) * (long long)(W > 1 ? W - 1 : 0) * HD;
-
-    auto issue = [&](int c) {      // thread 0: bulk-copy chunk c into buffer c % SWA_NBUF
-        const int buf = c % SWA_NBUF;
-        const int keys = min(SWA_CHUNK, n - c * SWA_CHUNK);
-        const uint32_t bytes = (uint32_t)(keys * HD * sizeof(T));
-        const uint32_t bar = smem_addr(&full[buf]);
-        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(2 * bytes) : "memory");
-        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                     ::"r"(smem_addr(sm_k[buf])), "l"(Kr + (long long)c * CHUNK_ELEMS), "r"(bytes), "r"(bar)
-                     : "memory");
-        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                     ::"r"(smem_addr(sm_v[buf])), "l"(Vr + (long long)c * CHUNK_ELEMS), "r"(bytes), "r"(bar)
-                     : "memory");
-    };
-    if (threadIdx.x == 0) {
-        failed = 0;
-        for (int i = 0; i < SWA_NBUF; ++i)
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&full[i])));
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        for (int c = 0; c < min(nchunks, SWA_NBUF); ++c) issue(c);
-    }
-
     const float* row = qkv + (long long)b * 3 * d + h * HD;
     float q[EPL];
 #pragma unroll
@@ -186,6 +145,7 @@ __global__ void __launch_bounds__(SWA_WARPS * 32) k_swa_decode(const float* __re
 #pragma unroll
     for (int i = 0; i < EPL; ++i) acc[i] = 0.f;
     if (warp == 0) {
+        // the current token: k_t (rotated) and v_t rounded to the storage type, as cached
         float k[EPL], v[EPL];
 #pragma unroll
         for (int i = 0; i < EPL; ++i) {
@@ -208,33 +168,16 @@ __global__ void __launch_bounds__(SWA_WARPS * 32) k_swa_decode(const float* __re
             sm_kv[1][li] = Vec16<T>::pack(v);
         }
     }
-    __syncthreads();                                       // barriers initialised
-    for (int c = 0; c < nchunks; ++c) {
-        const int buf = c % SWA_NBUF;
-        const uint32_t parity = (c / SWA_NBUF) & 1;
-        const uint32_t bar = smem_addr(&full[buf]);
-        uint32_t done = 0;
-        uint64_t t0 = 0;
-        for (int it = 0;; ++it) {
-            asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                         "selp.u32 %0, 1, 0, p;\n\t}"
-                         : "=r"(done) : "r"(bar), "r"(parity) : "memory");
-            if (done) break;
-            uint64_t now;
-            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
-            if (it == 0) t0 = now;
-            else if (now - t0 > SWA_WAIT_NS) break;
-        }
-        if (!done) failed = 1;
-        __syncthreads();
-        if (failed) break;
-        const int keys = min(SWA_CHUNK, n - c * SWA_CHUNK);
-        const int per = (keys + SWA_WARPS - 1) / SWA_WARPS;
-        const int j0 = min(keys, warp * per);
-        const int nj = min(keys, j0 + per) - j0;
-        attend<T, HD, 4, false>(q, sm_k[buf] + j0 * HD, sm_v[buf] + j0 * HD, nj, g, li, m, l, acc);
-        __syncthreads();                                   // buffer consumed by every warp
-        if (threadIdx.x == 0 && c + SWA_NBUF < nchunks) issue(c + SWA_NBUF);
+    T* Kr = nullptr;
+    T* Vr = nullptr;
+    if (W > 1) {
+        Kr = ring + (((long long)b * 2 + 0) * H + h) * (long long)(W - 1) * HD;
+        Vr = ring + (((long long)b * 2 + 1) * H + h) * (long long)(W - 1) * HD;
+        int n = min(t - 1, W - 1);
+        int per = (n + SWA_WARPS - 1) / SWA_WARPS;
+        int j0 = min(n, warp * per);
+        int nj = min(n, j0 + per) - j0;
+        attend<T, HD, 4, true>(q, Kr + (long long)j0 * HD, Vr + (long long)j0 * HD, nj, g, li, m, l, acc);
     }
     merge_groups<T, HD>(m, l, acc);
     if (g == 0) {
@@ -243,10 +186,6 @@ __global__ void __launch_bounds__(SWA_WARPS * 32) k_swa_decode(const float* __re
         if (li == 0) { sm_m[warp] = m; sm_l[warp] = l; }
     }
     __syncthreads();
-    if (failed) {
-        if (threadIdx.x == 0) raise_flag(hdr, ERR_TIMEOUT);
-        return;
-    }
     if (warp != 0 || g != 0) return;
     float mx = NEG_BIG;
 #pragma unroll
@@ -256,10 +195,10 @@ __global__ void __launch_bounds__(SWA_WARPS * 32) k_swa_decode(const float* __re
     for (int i = 0; i < EPL; ++i) out[i] = 0.f;
 #pragma unroll
     for (int w = 0; w < SWA_WARPS; ++w) {
-        float cw = exp2f(sm_m[w] - mx);
-        L += sm_l[w] * cw;
+        float c = exp2f(sm_m[w] - mx);
+        L += sm_l[w] * c;
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) out[i] += sm_acc[w][li * EPL + i] * cw;
+        for (int i = 0; i < EPL; ++i) out[i] += sm_acc[w][li * EPL + i] * c;
     }
     float inv = 1.0f / L;
 #pragma unroll
@@ -385,9 +324,9 @@ inline unsigned blocks_for(long long items) { return (unsigned)((items + WARPS -
 
 template <typename T>
 cudaError_t launch_swa_decode(Launch L, const float* qkv, const float2* rope_row, T* ring, T* o, int B,
-                              int H, int hd, int W, int t, DevHeader* hdr) {
+                              int H, int hd, int W, int t) {
     RLT_HD_DISPATCH(hd, launch_k(L, k_swa_decode<T, HD>, (unsigned)(B * H), SWA_WARPS * 32, 0, qkv, rope_row,
-                                 ring, o, B, H, W, t, qscale_for(hd), hdr));
+                                 ring, o, B, H, W, t, qscale_for(hd)));
 }
 
 template <typename T>
@@ -415,7 +354,7 @@ cudaError_t launch_enc_attention(Launch L, const T* planes, T* o, int B, int Tn,
 
 #define RLT_INST(T)                                                                                    \
     template cudaError_t launch_swa_decode<T>(Launch, const float*, const float2*, T*, T*, int, int,   \
-                                              int, int, int, DevHeader*);                              \
+                                              int, int, int);                                          \
     template cudaError_t launch_xattn_decode<T>(Launch, const float*, const T*, long long, int, int, T*, int, \
                                                 int, int, int, float*);                                \
     template cudaError_t launch_enc_attention<T>(Launch, const T*, T*, int, int, int, int);

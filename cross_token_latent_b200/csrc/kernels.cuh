@@ -111,7 +111,7 @@ cudaError_t launch_gemm_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16
 // the current token; then stores k_t, v_t into ring slot (t-1) mod (W-1).
 template <typename T>
 cudaError_t launch_swa_decode(Launch L, const float* qkv, const float2* rope_row, T* ring, T* o,
-                              int B, int H, int hd, int W, int t, DevHeader* hdr);
+                              int B, int H, int hd, int W, int t);
 // Decoder cross-attention over M_{<=t} (positions 0..t-1) of one memory group: keys of
 // (b, h) at Mg + (b*H + h)*T_alloc*hd, values `plane` elements further.  Splits the keys of
 // each (b, h) into n_splits chunks when n_splits > 1 (partials in `part`).

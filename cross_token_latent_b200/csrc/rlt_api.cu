@@ -375,7 +375,7 @@ rlt_status step_impl(rlt_model* m, uint8_t* state, int B, const T* e, const T* M
         ea.out_f32 = qkv; ea.ld_out = 3 * d;
         CKP(RLT_K_QKV, launch_gemm<T>(L, Epi::StoreF32, A, d, m->at<T>(m->lay.wqkv[l]), B, 3 * d, d, ea));
         CKP(RLT_K_SWA, launch_swa_decode<T>(L, qkv, rope_row, ring + (size_t)l * ring_layer_elems(c, B), att, B, H, hd,
-                                c.W, t, m->hdr()));
+                                c.W, t));
         ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = x; ea.ld_out = d;
         CKP(RLT_K_O, launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.wo[l]), B, d, d, ea));
         // cross-attention to M_{<=t}
