@@ -35,11 +35,10 @@ __device__ __forceinline__ float group_sum(float v) {
 }
 
 // Accumulate keys [0, n) of K/V (row stride HD) into this lane group's running softmax.
-// q is pre-scaled by log2(e)/sqrt(hd).  n must be warp-uniform.  With STREAM the rows are read
-// with the L2 eviction policy `pol` and bypass L1; otherwise with plain loads.
+// q is pre-scaled by log2(e)/sqrt(hd).  n must be warp-uniform.
 template <typename T, int HD, int U, bool STREAM>
 __device__ __forceinline__ void attend(const float* q, const T* __restrict__ K, const T* __restrict__ V,
-                                       int n, int g, int li, float& m, float& l, float* acc, uint64_t pol = 0) {
+                                       int n, int g, int li, float& m, float& l, float* acc) {
     using G = Geom<T, HD>;
     constexpr int EPL = G::EPL, LPK = G::LPK, KPI = G::KPI;
     for (int base = 0; base < n; base += KPI * U) {
@@ -50,8 +49,8 @@ __device__ __forceinline__ void attend(const float* q, const T* __restrict__ K, 
             if (j < n) {
                 const T* kp = K + (long long)j * HD + li * EPL;
                 const T* vp = V + (long long)j * HD + li * EPL;
-                kr[u] = STREAM ? ld16_policy(kp, pol) : ld16(kp);
-                vr[u] = STREAM ? ld16_policy(vp, pol) : ld16(vp);
+                kr[u] = STREAM ? ld16_stream(kp) : ld16(kp);
+                vr[u] = STREAM ? ld16_stream(vp) : ld16(vp);
             } else {
                 kr[u] = make_uint4(0, 0, 0, 0);
                 vr[u] = make_uint4(0, 0, 0, 0);
@@ -178,8 +177,7 @@ __global__ void __launch_bounds__(SWA_WARPS * 32, 6) k_swa_decode(const float* _
         int per = (n + SWA_WARPS - 1) / SWA_WARPS;
         int j0 = min(n, warp * per);
         int nj = min(n, j0 + per) - j0;
-        attend<T, HD, 4, true>(q, Kr + (long long)j0 * HD, Vr + (long long)j0 * HD, nj, g, li, m, l, acc,
-                               l2_policy_evict_first());
+        attend<T, HD, 4, true>(q, Kr + (long long)j0 * HD, Vr + (long long)j0 * HD, nj, g, li, m, l, acc);
     }
     merge_groups<T, HD>(m, l, acc);
     if (g == 0) {
@@ -218,16 +216,13 @@ __global__ void __launch_bounds__(WARPS * 32) k_xattn_decode(const float* __rest
                                                              const T* __restrict__ Mg, long long plane,
                                                              int T_alloc, int t, T* __restrict__ o, int B, int H,
                                                              int n_splits, int chunk, float* __restrict__ part,
-                                                             float qscale, int reverse) {
+                                                             float qscale) {
     using G = Geom<T, HD>;
     constexpr int EPL = G::EPL, LPK = G::LPK;
     pdl_wait();
     pdl_trigger();
     int item = blockIdx.x * WARPS + (threadIdx.x >> 5);
     if (item >= B * H * n_splits) return;
-    // Alternate layers walk the (sequence, head) items in opposite orders, so that a layer starts
-    // with the memory rows the previous layer read last (still in L2 when G = 1).
-    if (reverse) item = B * H * n_splits - 1 - item;
     int lane = threadIdx.x & 31, g = lane / LPK, li = lane % LPK;
     int bh = item / n_splits, sp = item % n_splits;
     int b = bh / H, h = bh % H;
@@ -243,8 +238,7 @@ __global__ void __launch_bounds__(WARPS * 32) k_xattn_decode(const float* __rest
     float m = NEG_BIG, l = 0.f, acc[EPL];
 #pragma unroll
     for (int i = 0; i < EPL; ++i) acc[i] = 0.f;
-    attend<T, HD, 4, true>(q, K + (long long)j0 * HD, V + (long long)j0 * HD, n, g, li, m, l, acc,
-                           l2_policy_evict_last());
+    attend<T, HD, 4, true>(q, K + (long long)j0 * HD, V + (long long)j0 * HD, n, g, li, m, l, acc);
     merge_groups<T, HD>(m, l, acc);
     if (g != 0) return;
     if (n_splits == 1) {
@@ -337,17 +331,17 @@ cudaError_t launch_swa_decode(Launch L, const float* qkv, const float2* rope_row
 
 template <typename T>
 static cudaError_t xattn_main(Launch L, const float* qc, const T* Mg, long long plane, int T_alloc, int t, T* o,
-                              int B, int H, int hd, int n_splits, int chunk, float* part, int reverse) {
+                              int B, int H, int hd, int n_splits, int chunk, float* part) {
     RLT_HD_DISPATCH(hd, launch_k(L, k_xattn_decode<T, HD>, blocks_for((long long)B * H * n_splits), WARPS * 32, 0,
-                                 qc, Mg, plane, T_alloc, t, o, B, H, n_splits, chunk, part, qscale_for(hd), reverse));
+                                 qc, Mg, plane, T_alloc, t, o, B, H, n_splits, chunk, part, qscale_for(hd)));
 }
 
 template <typename T>
 cudaError_t launch_xattn_decode(Launch L, const float* qc, const T* Mg, long long plane, int T_alloc, int t, T* o,
-                                int B, int H, int hd, int n_splits, float* part, int reverse) {
+                                int B, int H, int hd, int n_splits, float* part) {
     if (n_splits < 1) n_splits = 1;
     int chunk = (t + n_splits - 1) / n_splits;
-    cudaError_t e = xattn_main<T>(L, qc, Mg, plane, T_alloc, t, o, B, H, hd, n_splits, chunk, part, reverse);
+    cudaError_t e = xattn_main<T>(L, qc, Mg, plane, T_alloc, t, o, B, H, hd, n_splits, chunk, part);
     if (e != cudaSuccess || n_splits == 1) return e;
     return launch_k(L, k_attn_combine<T>, (unsigned)(B * H), (unsigned)hd, 0, (const float*)part, n_splits, hd, H, o);
 }
@@ -362,7 +356,7 @@ cudaError_t launch_enc_attention(Launch L, const T* planes, T* o, int B, int Tn,
     template cudaError_t launch_swa_decode<T>(Launch, const float*, const float2*, T*, T*, int, int,   \
                                               int, int, int);                                          \
     template cudaError_t launch_xattn_decode<T>(Launch, const float*, const T*, long long, int, int, T*, int, \
-                                                int, int, int, float*, int);                           \
+                                                int, int, int, float*);                                \
     template cudaError_t launch_enc_attention<T>(Launch, const T*, T*, int, int, int, int);
 RLT_INST(float)
 RLT_INST(bf16)

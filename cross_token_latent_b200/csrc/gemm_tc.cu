@@ -101,7 +101,7 @@ struct TcShape {
 template <int BN, int STAGES, int SPLIT>
 __global__ void __launch_bounds__(128, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW, int M, int N, int K,
-          Epi epi, EpiArgs ea, DevHeader* hdr, int w_evict_first) {
+          Epi epi, EpiArgs ea, DevHeader* hdr) {
     using S = TcShape<BN, STAGES, SPLIT>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -147,14 +147,11 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         // (A) loads after it.
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmW) : "memory");
-        // decode-size products read each weight tile a handful of times in one burst: let it be
-        // evicted first; the encoder's products reuse every weight tile across thousands of rows
-        const uint64_t wpol = w_evict_first ? l2_policy_evict_first() : l2_policy_evict_normal();
         const int pre = nkb < STAGES ? nkb : STAGES;
         for (int kb = 0; kb < pre; ++kb) {
             uint8_t* a = smem + kb * S::STAGE_BYTES;
             mbar_expect_tx(&full[kb], S::STAGE_BYTES);
-            tma_load_2d_hint(a + A_BYTES, &tmW, &full[kb], (kb0 + kb) * BK, n0, wpol);
+            tma_load_2d(a + A_BYTES, &tmW, &full[kb], (kb0 + kb) * BK, n0);
         }
         pdl_wait();
         for (int kb = 0; kb < pre; ++kb)
@@ -166,7 +163,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
             uint8_t* a = smem + s * S::STAGE_BYTES;
             mbar_expect_tx(&full[s], S::STAGE_BYTES);
             tma_load_2d(a, &tmA, &full[s], (kb0 + kb) * BK, m0);
-            tma_load_2d_hint(a + A_BYTES, &tmW, &full[s], (kb0 + kb) * BK, n0, wpol);
+            tma_load_2d(a + A_BYTES, &tmW, &full[s], (kb0 + kb) * BK, n0);
         }
     } else if (warp == 1 && lane == 0) {
         // MMA issuer
@@ -387,9 +384,8 @@ cudaError_t run_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int
     CUtensorMap ta, tw;
     if (!cached_map(&ta, A, M, K, lda, BM) || !cached_map(&tw, W, N, K, K, BN)) return cudaErrorInvalidValue;
     dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, SPLIT);
-    const int w_evict_first = M <= 1024 ? 1 : 0;
     if constexpr (SPLIT == 1) {
-        return launch_k(L, k_gemm_tc<BN, STAGES, 1>, grid, 128, S::SMEM, ta, tw, M, N, K, epi, ea, hdr, w_evict_first);
+        return launch_k(L, k_gemm_tc<BN, STAGES, 1>, grid, 128, S::SMEM, ta, tw, M, N, K, epi, ea, hdr);
     } else {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = grid;
@@ -406,7 +402,7 @@ cudaError_t run_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int
         cfg.attrs = attr;
         cfg.numAttrs = 2;
         *L.count += 1;
-        return cudaLaunchKernelEx(&cfg, k_gemm_tc<BN, STAGES, SPLIT>, ta, tw, M, N, K, epi, ea, hdr, w_evict_first);
+        return cudaLaunchKernelEx(&cfg, k_gemm_tc<BN, STAGES, SPLIT>, ta, tw, M, N, K, epi, ea, hdr);
     }
 }
 

@@ -114,11 +114,10 @@ cudaError_t launch_swa_decode(Launch L, const float* qkv, const float2* rope_row
                               int B, int H, int hd, int W, int t);
 // Decoder cross-attention over M_{<=t} (positions 0..t-1) of one memory group: keys of
 // (b, h) at Mg + (b*H + h)*T_alloc*hd, values `plane` elements further.  Splits the keys of
-// each (b, h) into n_splits chunks when n_splits > 1 (partials in `part`).  `reverse` walks
-// the work items in the opposite order (alternate layers, for L2 reuse of a shared memory).
+// each (b, h) into n_splits chunks when n_splits > 1 (partials in `part`).
 template <typename T>
 cudaError_t launch_xattn_decode(Launch L, const float* qc, const T* Mg, long long plane, int T_alloc, int t,
-                                T* o, int B, int H, int hd, int n_splits, float* part, int reverse);
+                                T* o, int B, int H, int hd, int n_splits, float* part);
 // Encoder causal self-attention: planes T [3][B][H][T][hd] -> o T [B*T, d]
 template <typename T>
 cudaError_t launch_enc_attention(Launch L, const T* planes, T* o, int B, int Tn, int H, int hd);

@@ -384,7 +384,7 @@ rlt_status step_impl(rlt_model* m, uint8_t* state, int B, const T* e, const T* M
         CKP(RLT_K_QC, launch_gemm<T>(L, Epi::StoreF32, A, d, m->at<T>(m->lay.wqc[l]), B, d, d, ea));
         const T* Mg = M + (c.G == 1 ? 0 : (size_t)l * group_elems);
         CKP(RLT_K_XATTN, launch_xattn_decode<T>(L, qc, Mg, (long long)B * H * T_alloc * hd, T_alloc, t, att, B, H, hd,
-                                                splits, part, l & 1));
+                                                splits, part));
         ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = x; ea.ld_out = d;
         CKP(RLT_K_OC, launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.woc[l]), B, d, d, ea));
         // SwiGLU FFN (weights of encoder layer l)
