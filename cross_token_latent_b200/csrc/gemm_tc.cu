@@ -186,92 +186,46 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     pdl_wait();
 
     // epilogue: thread owns output row m0 + 32*warp + lane (a split rank with no k-blocks has
-    // issued no MMA and contributes zeros).  For a residual add the row's current values are
-    // loaded before waiting for the MMAs, so the epilogue does not pay one L2 round trip per
-    // column chunk after the main loop.
-    const int row = warp * 32 + lane;                            // row within the tile
-    const int m = m0 + row;
-    constexpr bool kPrefetchable = BN <= 128;
-    float xr[kPrefetchable ? BN : 1];
-    const bool resid = kPrefetchable && epi == Epi::ResidAdd;
-    uint32_t owner = 0;
-    int row_local = row;
-    if constexpr (SPLIT > 1) {
-        owner = (uint32_t)(row / S::ROWS_PER_OWNER);
-        row_local = row - (int)owner * S::ROWS_PER_OWNER;
-    }
-    if constexpr (kPrefetchable) {
-        if (resid && m < M && owner == rank) {
-            const float* xp = ea.out_f32 + (long long)m * ea.ld_out;
-#pragma unroll
-            for (int j = 0; j < BN; j += 4) {
-                int n = n0 + j;
-                if (n + 3 < N) {
-                    float4 q = *reinterpret_cast<const float4*>(xp + n);
-                    xr[j] = q.x; xr[j + 1] = q.y; xr[j + 2] = q.z; xr[j + 3] = q.w;
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) xr[j + i] = (n + i < N) ? xp[n + i] : 0.f;
-                }
-            }
-        }
-    }
-    auto finish16 = [&](int c, const float* v) {             // columns n0 + c .. +15 of row m
-        int n = n0 + c;
-        if (m >= M || n >= N) return;
-        int cnt = min(16, N - n);
-        if constexpr (kPrefetchable) {
-            if (resid) {
-                float* o = ea.out_f32 + (long long)m * ea.ld_out + n;
-                if (cnt == 16) {
-#pragma unroll
-                    for (int j = 0; j < 16; j += 4)
-                        *reinterpret_cast<float4*>(o + j) = make_float4(xr[c + j] + v[j], xr[c + j + 1] + v[j + 1],
-                                                                        xr[c + j + 2] + v[j + 2], xr[c + j + 3] + v[j + 3]);
-                } else {
-                    for (int j = 0; j < cnt; ++j) o[j] = xr[c + j] + v[j];
-                }
-                return;
-            }
-        }
-        epilogue16(epi, ea, m, n, cnt, v);
-    };
+    // issued no MMA and contributes zeros)
     bool ok = nkb == 0 ? true : mbar_wait(done, 0, &abort_flag);
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     if constexpr (SPLIT == 1) {
         if (ok) {
-#pragma unroll
-            for (int c = 0; c < BN; c += 32) {
-                float v[32];
-                tmem_ld32(lane_base + c, v);
-                finish16(c, v);
-                finish16(c + 16, v + 16);
+            const int m = m0 + warp * 32 + lane;
+#pragma unroll 1
+            for (int c = 0; c < BN; c += 16) {
+                float v[16];
+                tmem_ld16(lane_base + c, v);
+                int n = n0 + c;
+                if (m < M && n < N) epilogue16(epi, ea, m, n, min(16, N - n), v);
             }
         }
     } else {
         // send this warp's 32 partial rows to the owner of their band
+        const int row = warp * 32 + lane;                        // row within the tile
+        const uint32_t owner = (uint32_t)(row / S::ROWS_PER_OWNER);
+        const int row_local = row - (int)owner * S::ROWS_PER_OWNER;
         cluster_wait_acquire();                                  // every CTA of the cluster has started
         if (ok) {
 #pragma unroll 1
-            for (int c = 0; c < BN; c += 32) {
-                float v[32];
+            for (int c = 0; c < BN; c += 16) {
+                float v[16];
                 if (nkb > 0) {
-                    tmem_ld32(lane_base + c, v);
+                    tmem_ld16(lane_base + c, v);
                 } else {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = 0.f;
+                    for (int j = 0; j < 16; ++j) v[j] = 0.f;
                 }
-                float* dst = recv + ((size_t)rank * S::ROWS_PER_OWNER + row_local) * BN + c;
-                dsmem_store16(dst, owner, v);
-                dsmem_store16(dst + 16, owner, v + 16);
+                dsmem_store16(recv + ((size_t)rank * S::ROWS_PER_OWNER + row_local) * BN + c, owner, v);
             }
         }
         cluster_arrive_release();
         cluster_wait_acquire();                                  // all partials have landed
         if (ok && owner == rank) {
-#pragma unroll
+            const int m = m0 + row;
+#pragma unroll 1
             for (int c = 0; c < BN; c += 16) {
                 float v[16];
 #pragma unroll
@@ -285,7 +239,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                         v[4 * j] += q.x; v[4 * j + 1] += q.y; v[4 * j + 2] += q.z; v[4 * j + 3] += q.w;
                     }
                 }
-                finish16(c, v);
+                int n = n0 + c;
+                if (m < M && n < N) epilogue16(epi, ea, m, n, min(16, N - n), v);
             }
         }
     }
