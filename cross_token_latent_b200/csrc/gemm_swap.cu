@@ -1,0 +1,306 @@
+// Tensor-core GEMM for few rows (M <= 64), the decode shape of small batches:
+// C[M, N] = A[M, K] x W[N, K]^T computed as C^T = W A^T, so that the weight rows sit on the
+// MMA's M = 128 side and the batch rows on its N side (NB = 16, 32 or 64).  Every CTA then
+// streams its own 128-row slab of W exactly once, and only the small activation panel is
+// re-read by every CTA; the K dimension can be split over a cluster of up to 8 CTAs (partial
+// slabs reduced in rank order through distributed shared memory, as in gemm_tc.cu).
+//
+// Roles as in gemm_tc.cu: warp 0 lane 0 issues TMA loads (weights before the programmatic
+// launch dependency wait, activations after it), warp 1 lane 0 issues tcgen05.mma, warp 2 owns
+// the TMEM allocation, all four warps run the epilogue.  In the epilogue thread r of the CTA
+// owns output column (feature) f0 + r and holds the NB batch rows of that column; adjacent
+// lanes hold the gate/up (or gate/feedback) pairs of the interleaved SwiGLU and merge weights.
+#include <cudaTypedefs.h>
+
+#include "kernels.cuh"
+#include "sm100.cuh"
+
+namespace rlt {
+
+namespace {
+
+constexpr int FM = 128;                      // weight rows (features) per CTA: UMMA M
+constexpr int KB = 64;                       // k-block: one 128-byte swizzle row
+constexpr int W_BYTES = FM * KB * 2;
+
+template <int NB, int STAGES, int SPLIT>
+struct SwShape {
+    static constexpr int X_BYTES = NB * KB * 2;
+    static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
+    static constexpr int TMEM_COLS = NB < 32 ? 32 : NB;
+    static constexpr int ROWS_PER_OWNER = FM / SPLIT;
+    static constexpr int RECV_BYTES = SPLIT > 1 ? FM * NB * 4 : 0;
+    static constexpr int SMEM = STAGES * STAGE_BYTES + RECV_BYTES + 1024 + 256;
+};
+
+// Transposed epilogue: v[j] is output (row mb + j, column n) for j = 0..15.  Every lane of the
+// warp must call it (the pair epilogues exchange values between lanes n and n ^ 1).
+__device__ __forceinline__ void epilogue16_t(Epi epi, const EpiArgs& ea, int n, bool n_ok, int mb, int M,
+                                             const float* v) {
+    switch (epi) {
+        case Epi::StoreF32:
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                if (n_ok && mb + j < M) ea.out_f32[(long long)(mb + j) * ea.ld_out + n] = v[j] * ea.scale;
+            break;
+        case Epi::ResidAdd:
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                if (n_ok && mb + j < M) ea.out_f32[(long long)(mb + j) * ea.ld_out + n] += v[j];
+            break;
+        case Epi::SwiGLU: {     // feature 2c = gate_c, 2c+1 = up_c
+            bf16* o = reinterpret_cast<bf16*>(ea.out_t);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                float up = __shfl_xor_sync(0xffffffffu, v[j], 1);
+                if (n_ok && !(n & 1) && mb + j < M)
+                    o[(long long)(mb + j) * ea.ld_out + n / 2] = __float2bfloat16_rn(siluf_(v[j]) * up);
+            }
+            break;
+        }
+        case Epi::Merge: {      // feature 2c = gate pre-activation, 2c+1 = feedback projection
+            const bf16* e = reinterpret_cast<const bf16*>(ea.merge_e);
+            const int c = n / 2;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                float u = __shfl_xor_sync(0xffffffffu, v[j], 1);
+                if (n_ok && !(n & 1) && mb + j < M) {
+                    long long m = mb + j;
+                    ea.out_f32[m * ea.ld_out + c] =
+                        __bfloat162float(e[m * ea.ld_e + c]) + sigmoidf_(v[j] + ea.bias[c]) * u;
+                }
+            }
+            break;
+        }
+    }
+}
+
+template <int NB, int STAGES, int SPLIT>
+__global__ void __launch_bounds__(128, 1)
+k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, int M, int N, int K,
+            Epi epi, EpiArgs ea, DevHeader* hdr) {
+    using S = SwShape<NB, STAGES, SPLIT>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float* recv = reinterpret_cast<float*>(smem + STAGES * S::STAGE_BYTES);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES + S::RECV_BYTES);
+    uint64_t* empty = full + STAGES;
+    uint64_t* done = empty + STAGES;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    __shared__ int abort_flag;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int f0 = blockIdx.x * FM, b0 = blockIdx.y * NB;
+    const int nkb_all = (K + KB - 1) / KB;
+    const uint32_t rank = SPLIT > 1 ? cluster_rank() : 0;
+    const int per = (nkb_all + SPLIT - 1) / SPLIT;
+    const int kb0 = min(nkb_all, (int)rank * per);
+    const int nkb = min(nkb_all, kb0 + per) - kb0;
+    pdl_trigger();
+    if constexpr (SPLIT > 1) cluster_arrive_relaxed();
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(done, 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 2) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(S::TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0 && lane == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&tmW) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&tmX) : "memory");
+        const int pre = nkb < STAGES ? nkb : STAGES;
+        for (int kb = 0; kb < pre; ++kb) {
+            mbar_expect_tx(&full[kb], S::STAGE_BYTES);
+            tma_load_2d(smem + kb * S::STAGE_BYTES, &tmW, &full[kb], (kb0 + kb) * KB, f0);
+        }
+        pdl_wait();
+        for (int kb = 0; kb < pre; ++kb)
+            tma_load_2d(smem + kb * S::STAGE_BYTES + W_BYTES, &tmX, &full[kb], (kb0 + kb) * KB, b0);
+        for (int kb = pre; kb < nkb; ++kb) {
+            int s = kb % STAGES;
+            uint32_t ph = (kb / STAGES) & 1;
+            if (!mbar_wait(&empty[s], ph ^ 1, &abort_flag)) { abort_flag = 1; break; }
+            uint8_t* st = smem + s * S::STAGE_BYTES;
+            mbar_expect_tx(&full[s], S::STAGE_BYTES);
+            tma_load_2d(st, &tmW, &full[s], (kb0 + kb) * KB, f0);
+            tma_load_2d(st + W_BYTES, &tmX, &full[s], (kb0 + kb) * KB, b0);
+        }
+    } else if (warp == 1 && lane == 0) {
+        constexpr uint32_t idesc = idesc_bf16(FM, NB);
+        for (int kb = 0; kb < nkb; ++kb) {
+            int s = kb % STAGES;
+            uint32_t ph = (kb / STAGES) & 1;
+            if (!mbar_wait(&full[s], ph, &abort_flag)) { abort_flag = 1; break; }
+            tc_fence_after();
+            uint8_t* st = smem + s * S::STAGE_BYTES;
+            uint64_t dw = sdesc_sw128(st), dx = sdesc_sw128(st + W_BYTES);
+#pragma unroll
+            for (int k = 0; k < KB / 16; ++k) umma(tmem, dw + 2 * k, dx + 2 * k, idesc, (kb | k) != 0);
+            umma_commit(&empty[s]);
+        }
+        if (nkb > 0) umma_commit(done);
+    }
+    __syncwarp();
+    pdl_wait();
+
+    // epilogue: thread r owns feature f0 + r, TMEM columns are batch rows b0 .. b0 + NB - 1
+    const int r = warp * 32 + lane;
+    const int n = f0 + r;
+    const bool n_ok = n < N;
+    bool ok = nkb == 0 ? true : mbar_wait(done, 0, &abort_flag);
+    ok = __all_sync(0xffffffffu, ok);
+    tc_fence_after();
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    if constexpr (SPLIT == 1) {
+        if (ok) {
+#pragma unroll 1
+            for (int c = 0; c < NB; c += 16) {
+                float v[16];
+                tmem_ld16(lane_base + c, v);
+                epilogue16_t(epi, ea, n, n_ok, b0 + c, M, v);
+            }
+        }
+    } else {
+        const uint32_t owner = (uint32_t)(r / S::ROWS_PER_OWNER);
+        const int r_local = r - (int)owner * S::ROWS_PER_OWNER;
+        cluster_wait_acquire();                                  // every CTA of the cluster has started
+        if (ok) {
+#pragma unroll 1
+            for (int c = 0; c < NB; c += 16) {
+                float v[16];
+                if (nkb > 0) {
+                    tmem_ld16(lane_base + c, v);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) v[j] = 0.f;
+                }
+                dsmem_store16(recv + ((size_t)rank * S::ROWS_PER_OWNER + r_local) * NB + c, owner, v);
+            }
+        }
+        cluster_arrive_release();
+        cluster_wait_acquire();                                  // all partials have landed
+        // every lane runs the epilogue (the pair epilogues shuffle across lanes); lanes outside
+        // this CTA's band only predicate their stores off
+        if (ok) {
+            const bool mine = owner == rank;
+#pragma unroll 1
+            for (int c = 0; c < NB; c += 16) {
+                float v[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] = 0.f;
+                for (int src = 0; src < SPLIT; ++src) {
+                    const float4* p = reinterpret_cast<const float4*>(
+                        recv + ((size_t)src * S::ROWS_PER_OWNER + r_local) * NB + c);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        float4 q = p[j];
+                        v[4 * j] += q.x; v[4 * j + 1] += q.y; v[4 * j + 2] += q.z; v[4 * j + 3] += q.w;
+                    }
+                }
+                epilogue16_t(epi, ea, n, n_ok && mine, b0 + c, M, v);
+            }
+        }
+    }
+    if (!ok && lane == 0) {
+        abort_flag = 1;
+        raise_flag(hdr, ERR_TIMEOUT);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(S::TMEM_COLS));
+    }
+}
+
+bool map2d(CUtensorMap* map, const void* ptr, int rows, int cols, int ld, int box_rows) {
+    uint64_t dims[2] = {(uint64_t)cols, (uint64_t)rows};
+    uint64_t strides[1] = {(uint64_t)ld * 2};
+    uint32_t box[2] = {(uint32_t)KB, (uint32_t)box_rows};
+    return tma_map_bf16(map, ptr, 2, dims, strides, box);
+}
+
+template <int NB, int STAGES, int SPLIT>
+cudaError_t run_swap(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K, const EpiArgs& ea,
+                     DevHeader* hdr) {
+    using S = SwShape<NB, STAGES, SPLIT>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(k_gemm_swap<NB, STAGES, SPLIT>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    CUtensorMap tw, tx;
+    if (!map2d(&tw, W, N, K, K, FM) || !map2d(&tx, A, M, K, lda, NB)) return cudaErrorInvalidValue;
+    dim3 grid((N + FM - 1) / FM, (M + NB - 1) / NB, SPLIT);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = S::SMEM;
+    cfg.stream = L.stream;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+    if (SPLIT > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = 1;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = SPLIT;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    *L.count += 1;
+    return cudaLaunchKernelEx(&cfg, k_gemm_swap<NB, STAGES, SPLIT>, tw, tx, M, N, K, epi, ea, hdr);
+}
+
+template <int NB>
+cudaError_t run_swap_split(int split, Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
+                           const EpiArgs& ea, DevHeader* hdr) {
+    switch (split) {
+        case 1: return run_swap<NB, 6, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 2: return run_swap<NB, 6, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 4: return run_swap<NB, 6, 4>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 8: return run_swap<NB, 6, 8>(L, epi, A, lda, W, M, N, K, ea, hdr);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+bool gemm_swap_supported(int M) { return M >= 1 && M <= 64; }
+
+cudaError_t launch_gemm_swap(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
+                             const EpiArgs& ea, DevHeader* hdr, int split) {
+    if (!gemm_swap_supported(M)) return cudaErrorInvalidValue;
+    const int nb = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+    if (split <= 0) {
+        // fill one wave of SMs with at least two k-blocks per rank
+        long long base = (long long)((N + FM - 1) / FM) * ((M + nb - 1) / nb);
+        int nkb = (K + KB - 1) / KB;
+        split = 1;
+        for (int s : {2, 4, 8})
+            if (base * s <= 148 && nkb >= 2 * s) split = s;
+    }
+    if (nb == 16) return run_swap_split<16>(split, L, epi, A, lda, W, M, N, K, ea, hdr);
+    if (nb == 32) return run_swap_split<32>(split, L, epi, A, lda, W, M, N, K, ea, hdr);
+    return run_swap_split<64>(split, L, epi, A, lda, W, M, N, K, ea, hdr);
+}
+
+}  // namespace rlt

@@ -105,6 +105,13 @@ int gemm_tc_variants();
 cudaError_t launch_gemm_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                            const EpiArgs& ea, DevHeader* hdr, int variant = -1);
 
+// ------------------------------------------------------------------ gemm_swap.cu
+// Few-row products (1 <= M <= 64) with the weights on the MMA's M side; split = K split over a
+// cluster of 1, 2, 4 or 8 CTAs (0: choose).
+bool gemm_swap_supported(int M);
+cudaError_t launch_gemm_swap(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
+                             const EpiArgs& ea, DevHeader* hdr, int split = 0);
+
 // ------------------------------------------------------------------ attention.cu
 // Decoder sliding-window self-attention for one layer at step t (1-based): RoPE at
 // position t-1 on q/k from qkv [B, 3d]; attends over the min(t-1, W-1) cached entries plus

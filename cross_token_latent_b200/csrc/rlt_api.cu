@@ -730,8 +730,9 @@ uint64_t rlt_launch_count(const rlt_model* m) { return m ? m->launches : 0; }
 
 rlt_status rlt_gemm_bf16(rlt_model* m, const void* A, const void* W, float* C, int M, int N, int K, int kernel,
                          void* stream) {
-    if (!m || !A || !W || !C || M < 1 || N < 1 || K < 1 || kernel < 0 || kernel > 1 + gemm_tc_variants())
-        return RLT_EINVAL;
+    const int n_tc = gemm_tc_variants();
+    if (!m || !A || !W || !C || M < 1 || N < 1 || K < 1 || kernel < 0 || kernel > 1 + n_tc + 5) return RLT_EINVAL;
+    if (kernel > 1 + n_tc && !gemm_swap_supported(M)) return RLT_EINVAL;
     if (!aligned(A, 16) || !aligned(W, 16) || !aligned(C, 16) || K % 8 || N % 4) return RLT_EINVAL;
     Launch L = m->launch(stream);
     EpiArgs ea;
@@ -740,8 +741,16 @@ rlt_status rlt_gemm_bf16(rlt_model* m, const void* A, const void* W, float* C, i
     ea.ld_out = N;
     const bf16* a = reinterpret_cast<const bf16*>(A);
     const bf16* w = reinterpret_cast<const bf16*>(W);
-    CK(kernel == 1 ? launch_gemm_simt<bf16>(L, Epi::StoreF32, a, K, w, M, N, K, ea)
-                   : launch_gemm_tc(L, Epi::StoreF32, a, K, w, M, N, K, ea, m->hdr(), kernel - 2));
+    if (kernel == 0) {
+        CK(launch_gemm<bf16>(L, Epi::StoreF32, a, K, w, M, N, K, ea));
+    } else if (kernel == 1) {
+        CK(launch_gemm_simt<bf16>(L, Epi::StoreF32, a, K, w, M, N, K, ea));
+    } else if (kernel <= 1 + n_tc) {
+        CK(launch_gemm_tc(L, Epi::StoreF32, a, K, w, M, N, K, ea, m->hdr(), kernel - 2));
+    } else {
+        static const int splits[5] = {0, 1, 2, 4, 8};
+        CK(launch_gemm_swap(L, Epi::StoreF32, a, K, w, M, N, K, ea, m->hdr(), splits[kernel - 2 - n_tc]));
+    }
     return RLT_OK;
 }
 

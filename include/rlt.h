@@ -236,7 +236,9 @@ uint64_t rlt_launch_count(const rlt_model* m);
  * the CUDA-core kernel, kernel 2 + v = tensor-core tile variant v (0: 128x32 tiles, 5 stages;
  * 1: 128x64, 4; 2: 128x128, 3; 3: 128x128, 5; 4: 128x256, 4; then K split over a cluster of
  * CTAs with a shared-memory reduction: 5: 128x128 split 2; 6: 128x128 split 4; 7: 128x64
- * split 2; 8: 128x64 split 4).  A, W, C 16-byte aligned, K a multiple of 8, N a multiple of 4.
+ * split 2; 8: 128x64 split 4), kernel 11 + s (M <= 64 only) = the few-row kernel with the
+ * weights on the MMA's M side and K split over a cluster of (s = 0: chosen, 1: 1, 2: 2, 3: 4,
+ * 4: 8) CTAs.  A, W, C 16-byte aligned, K a multiple of 8, N a multiple of 4.
  * Errors: RLT_EINVAL, RLT_ECUDA; a tensor-core wait that times out latches
  * RLT_ETIMEOUT (rlt_last_error). */
 rlt_status rlt_gemm_bf16(rlt_model* m, const void* A, const void* W, float* C, int M, int N, int K,
