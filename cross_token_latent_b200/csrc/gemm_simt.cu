@@ -107,7 +107,7 @@ template <>
 cudaError_t launch_gemm<bf16>(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                               const EpiArgs& ea) {
     if (gemm_tc_supported(A, lda, W, K)) {
-        if (gemm_swap_supported(M)) return launch_gemm_swap(L, epi, A, lda, W, M, N, K, ea, ea.hdr);
+        if (gemm_swap_preferred(M, N, K)) return launch_gemm_swap(L, epi, A, lda, W, M, N, K, ea, ea.hdr);
         return launch_gemm_tc(L, epi, A, lda, W, M, N, K, ea, ea.hdr);
     }
     return launch_gemm_simt<bf16>(L, epi, A, lda, W, M, N, K, ea);

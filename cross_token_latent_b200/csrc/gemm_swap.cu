@@ -286,16 +286,39 @@ cudaError_t run_swap_split(int split, Launch L, Epi epi, const bf16* A, int lda,
 
 bool gemm_swap_supported(int M) { return M >= 1 && M <= 64; }
 
+namespace {
+int swap_nb(int M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
+long long swap_base(int M, int N) {
+    const int nb = swap_nb(M);
+    return (long long)((N + FM - 1) / FM) * ((M + nb - 1) / nb);
+}
+}  // namespace
+
+// Measured on B200 at decode sizes: with at most 32 rows the swapped kernel wins or ties on
+// every projection shape; at 33..64 rows it wins only when the weight matrix alone fills a
+// wave with 128-row tiles (N >= ~6K), while narrower outputs run faster on the row-tile kernel
+// whose 64-wide tiles put twice as many CTAs in flight.  Below four k-blocks the narrow
+// row tiles win as well.
+bool gemm_swap_preferred(int M, int N, int K) {
+    if (!gemm_swap_supported(M)) return false;
+    if ((K + KB - 1) / KB < 4) return false;
+    if (M <= 32) return true;
+    const long long base = swap_base(M, N);
+    return base >= 48 && base <= 148;
+}
+
 cudaError_t launch_gemm_swap(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                              const EpiArgs& ea, DevHeader* hdr, int split) {
     if (!gemm_swap_supported(M)) return cudaErrorInvalidValue;
-    const int nb = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+    const int nb = swap_nb(M);
     if (split <= 0) {
-        // fill one wave of SMs with at least two k-blocks per rank
-        long long base = (long long)((N + FM - 1) / FM) * ((M + nb - 1) / nb);
-        int nkb = (K + KB - 1) / KB;
+        // fill one wave of SMs with at least two k-blocks per rank.  Clusters of 8 are left
+        // out: at one CTA per SM not every GPC holds two of them, so a 128-CTA grid of 8-CTA
+        // clusters runs in two waves (measured 2.2x the time of the 4-way split).
+        const long long base = swap_base(M, N);
+        const int nkb = (K + KB - 1) / KB;
         split = 1;
-        for (int s : {2, 4, 8})
+        for (int s : {2, 4})
             if (base * s <= 148 && nkb >= 2 * s) split = s;
     }
     if (nb == 16) return run_swap_split<16>(split, L, epi, A, lda, W, M, N, K, ea, hdr);

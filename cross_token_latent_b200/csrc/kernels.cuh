@@ -109,6 +109,7 @@ cudaError_t launch_gemm_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16
 // Few-row products (1 <= M <= 64) with the weights on the MMA's M side; split = K split over a
 // cluster of 1, 2, 4 or 8 CTAs (0: choose).
 bool gemm_swap_supported(int M);
+bool gemm_swap_preferred(int M, int N, int K);
 cudaError_t launch_gemm_swap(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                              const EpiArgs& ea, DevHeader* hdr, int split = 0);
 
