@@ -100,6 +100,7 @@ cudaError_t launch_gemm_simt(Launch L, Epi epi, const T* A, int lda, const T* W,
 template <>
 cudaError_t launch_gemm<float>(Launch L, Epi epi, const float* A, int lda, const float* W, int M, int N, int K,
                                const EpiArgs& ea) {
+    if (ea.norm_y || ea.ss_in) return cudaErrorInvalidValue;    // deferred norms: tensor-core paths only
     return launch_gemm_simt<float>(L, epi, A, lda, W, M, N, K, ea);
 }
 
@@ -110,6 +111,7 @@ cudaError_t launch_gemm<bf16>(Launch L, Epi epi, const bf16* A, int lda, const b
         if (gemm_swap_preferred(M, N, K)) return launch_gemm_swap(L, epi, A, lda, W, M, N, K, ea, ea.hdr);
         return launch_gemm_tc(L, epi, A, lda, W, M, N, K, ea, ea.hdr);
     }
+    if (ea.norm_y || ea.ss_in) return cudaErrorInvalidValue;    // deferred norms: tensor-core paths only
     return launch_gemm_simt<bf16>(L, epi, A, lda, W, M, N, K, ea);
 }
 

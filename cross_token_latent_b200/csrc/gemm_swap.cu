@@ -34,26 +34,42 @@ struct SwShape {
 };
 
 // Transposed epilogue: v[j] is output (row mb + j, column n) for j = 0..15.  Every lane of the
-// warp must call it (the pair epilogues exchange values between lanes n and n ^ 1).
-__device__ __forceinline__ void epilogue16_t(Epi epi, const EpiArgs& ea, int n, bool n_ok, int mb, int M,
+// warp must call it (the pair epilogues exchange values between lanes n and n ^ 1, and the
+// deferred-norm partials are reduced across lanes).  `store` says whether this lane writes.
+// Deferred-norm groups: for ResidAdd the 16 output columns of a half-warp (lanes 0 / 16 write
+// the partial), for Merge the 16 output columns of a whole warp (lane 0 writes).
+__device__ __forceinline__ void epilogue16_t(Epi epi, const EpiArgs& ea, int n, bool store, int mb, int M,
                                              const float* v) {
     switch (epi) {
         case Epi::StoreF32:
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-                if (n_ok && mb + j < M) ea.out_f32[(long long)(mb + j) * ea.ld_out + n] = v[j] * ea.scale;
+                if (store && mb + j < M) ea.out_f32[(long long)(mb + j) * ea.ld_out + n] = v[j] * ea.scale;
             break;
         case Epi::ResidAdd:
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-                if (n_ok && mb + j < M) ea.out_f32[(long long)(mb + j) * ea.ld_out + n] += v[j];
+            for (int j = 0; j < 16; ++j) {
+                const long long m = mb + j;
+                float x = 0.f;
+                if (store && m < M) {
+                    x = ea.out_f32[m * ea.ld_out + n] + v[j];
+                    ea.out_f32[m * ea.ld_out + n] = x;
+                    if (ea.norm_y) ea.norm_y[m * ea.ld_out + n] = __float2bfloat16_rn(x * ea.norm_g[n]);
+                }
+                if (ea.norm_y) {
+                    float sq = x * x;
+#pragma unroll
+                    for (int o = 8; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+                    if (store && m < M && (n & 15) == 0) ea.ss_out[m * ea.ss_ld + n / 16] = sq;
+                }
+            }
             break;
         case Epi::SwiGLU: {     // feature 2c = gate_c, 2c+1 = up_c
             bf16* o = reinterpret_cast<bf16*>(ea.out_t);
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 float up = __shfl_xor_sync(0xffffffffu, v[j], 1);
-                if (n_ok && !(n & 1) && mb + j < M)
+                if (store && !(n & 1) && mb + j < M)
                     o[(long long)(mb + j) * ea.ld_out + n / 2] = __float2bfloat16_rn(siluf_(v[j]) * up);
             }
             break;
@@ -63,11 +79,19 @@ __device__ __forceinline__ void epilogue16_t(Epi epi, const EpiArgs& ea, int n, 
             const int c = n / 2;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
+                const long long m = mb + j;
                 float u = __shfl_xor_sync(0xffffffffu, v[j], 1);
-                if (n_ok && !(n & 1) && mb + j < M) {
-                    long long m = mb + j;
-                    ea.out_f32[m * ea.ld_out + c] =
-                        __bfloat162float(e[m * ea.ld_e + c]) + sigmoidf_(v[j] + ea.bias[c]) * u;
+                float x = 0.f;
+                if (store && !(n & 1) && m < M) {
+                    x = __bfloat162float(e[m * ea.ld_e + c]) + sigmoidf_(v[j] + ea.bias[c]) * u;
+                    ea.out_f32[m * ea.ld_out + c] = x;
+                    if (ea.norm_y) ea.norm_y[m * ea.ld_out + c] = __float2bfloat16_rn(x * ea.norm_g[c]);
+                }
+                if (ea.norm_y) {
+                    float sq = x * x;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+                    if (store && m < M && (n & 31) == 0) ea.ss_out[m * ea.ss_ld + c / 16] = sq;
                 }
             }
             break;
@@ -88,6 +112,7 @@ k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
     uint64_t* done = empty + STAGES;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
     __shared__ int abort_flag;
+    __shared__ float rinv_s[NB];        // deferred-norm row scales of this CTA's batch rows
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int f0 = blockIdx.x * FM, b0 = blockIdx.y * NB;
@@ -160,6 +185,18 @@ k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
     const int r = warp * 32 + lane;
     const int n = f0 + r;
     const bool n_ok = n < N;
+    if (ea.ss_in) {
+        // warps 2 and 3 have no main-loop role: they compute the row scales while the MMAs run
+        const int i = threadIdx.x - 64;
+        if (i >= 0 && i < NB) rinv_s[i] = b0 + i < M ? deferred_rinv(ea, b0 + i) : 0.f;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+    }
+    auto scale = [&](int c, float* v) {
+        if (ea.ss_in) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] *= rinv_s[c + j];
+        }
+    };
     bool ok = nkb == 0 ? true : mbar_wait(done, 0, &abort_flag);
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
@@ -170,6 +207,7 @@ k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
             for (int c = 0; c < NB; c += 16) {
                 float v[16];
                 tmem_ld16(lane_base + c, v);
+                scale(c, v);
                 epilogue16_t(epi, ea, n, n_ok, b0 + c, M, v);
             }
         }
@@ -210,6 +248,7 @@ k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
                         v[4 * j] += q.x; v[4 * j + 1] += q.y; v[4 * j + 2] += q.z; v[4 * j + 3] += q.w;
                     }
                 }
+                scale(c, v);
                 epilogue16_t(epi, ea, n, n_ok && mine, b0 + c, M, v);
             }
         }
@@ -311,6 +350,7 @@ cudaError_t launch_gemm_swap(Launch L, Epi epi, const bf16* A, int lda, const bf
                              const EpiArgs& ea, DevHeader* hdr, int split) {
     if (!gemm_swap_supported(M)) return cudaErrorInvalidValue;
     const int nb = swap_nb(M);
+    if (ea.norm_y && split > 4) split = 4;      // a deferred-norm group must stay in one owner band
     if (split <= 0) {
         // fill one wave of SMs with at least two k-blocks per rank.  Clusters of 8 are left
         // out: at one CTA per SM not every GPC holds two of them, so a 128-CTA grid of 8-CTA

@@ -29,8 +29,11 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;                       // 64 bf16 = 128 bytes = one swizzle row
 constexpr int A_BYTES = BM * BK * 2;         // 16 KB
-// Fused epilogue on 16 consecutive columns n..n+15 of row m (cnt of them inside N).
-__device__ __forceinline__ void epilogue16(Epi epi, const EpiArgs& ea, int m, int n, int cnt, const float* v) {
+// Fused epilogue on 16 consecutive columns n..n+15 of row m (cnt of them inside N).  With a
+// deferred norm to produce (ea.norm_y, ResidAdd / Merge only) it also writes bf16(x * g) and
+// returns the sum of squares of the new x values it wrote (0 otherwise).
+__device__ __forceinline__ float epilogue16(Epi epi, const EpiArgs& ea, int m, int n, int cnt, const float* v) {
+    float ss = 0.f;
     switch (epi) {
         case Epi::StoreF32: {
             float* o = ea.out_f32 + (long long)m * ea.ld_out + n;
@@ -47,14 +50,34 @@ __device__ __forceinline__ void epilogue16(Epi epi, const EpiArgs& ea, int m, in
         case Epi::ResidAdd: {
             float* o = ea.out_f32 + (long long)m * ea.ld_out + n;
             if (cnt == 16) {
+                float x[16];
 #pragma unroll
                 for (int j = 0; j < 16; j += 4) {
-                    float4 x = *reinterpret_cast<float4*>(o + j);
-                    x.x += v[j]; x.y += v[j + 1]; x.z += v[j + 2]; x.w += v[j + 3];
-                    *reinterpret_cast<float4*>(o + j) = x;
+                    float4 q = *reinterpret_cast<float4*>(o + j);
+                    q.x += v[j]; q.y += v[j + 1]; q.z += v[j + 2]; q.w += v[j + 3];
+                    *reinterpret_cast<float4*>(o + j) = q;
+                    x[j] = q.x; x[j + 1] = q.y; x[j + 2] = q.z; x[j + 3] = q.w;
+                }
+                if (ea.norm_y) {
+                    float y[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        y[j] = x[j] * ea.norm_g[n + j];
+                        ss += x[j] * x[j];
+                    }
+                    bf16* yo = ea.norm_y + (long long)m * ea.ld_out + n;
+                    st16(yo, Vec16<bf16>::pack(y));
+                    st16(yo + 8, Vec16<bf16>::pack(y + 8));
                 }
             } else {
-                for (int j = 0; j < cnt; ++j) o[j] += v[j];
+                for (int j = 0; j < cnt; ++j) {
+                    float x = o[j] + v[j];
+                    o[j] = x;
+                    if (ea.norm_y) {
+                        ea.norm_y[(long long)m * ea.ld_out + n + j] = __float2bfloat16_rn(x * ea.norm_g[n + j]);
+                        ss += x * x;
+                    }
+                }
             }
             break;
         }
@@ -75,12 +98,42 @@ __device__ __forceinline__ void epilogue16(Epi epi, const EpiArgs& ea, int m, in
             float* o = ea.out_f32 + (long long)m * ea.ld_out;
             for (int j = 0; j + 1 < cnt; j += 2) {
                 int c = (n + j) / 2;
-                o[c] = __bfloat162float(e[c]) + sigmoidf_(v[j] + ea.bias[c]) * v[j + 1];
+                float x = __bfloat162float(e[c]) + sigmoidf_(v[j] + ea.bias[c]) * v[j + 1];
+                o[c] = x;
+                if (ea.norm_y) {
+                    ea.norm_y[(long long)m * ea.ld_out + c] = __float2bfloat16_rn(x * ea.norm_g[c]);
+                    ss += x * x;
+                }
             }
             break;
         }
     }
+    return ss;
 }
+
+// Per-row bookkeeping of a deferred norm around the 16-column epilogue chunks of one row:
+// the consumer's row scale, and the producer's group partial sums (16 output columns per
+// group = 16 GEMM columns, or 32 for the interleaved merge).  Tiles start on multiples of 32
+// columns, so a group never straddles two tiles.
+struct RowNorm {
+    float rinv = 1.f;
+    float acc = 0.f;
+    __device__ __forceinline__ void scale(const EpiArgs& ea, float* v) const {
+        if (ea.ss_in) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] *= rinv;
+        }
+    }
+    __device__ __forceinline__ void add(Epi epi, const EpiArgs& ea, int m, int n, int N, float part) {
+        if (!ea.norm_y) return;
+        acc += part;
+        const int gw = epi == Epi::Merge ? 32 : 16;
+        if ((n + 16) % gw == 0 || n + 16 >= N) {
+            ea.ss_out[(long long)m * ea.ss_ld + n / gw] = acc;
+            acc = 0.f;
+        }
+    }
+};
 
 template <int BN, int STAGES, int SPLIT>
 struct TcShape {
@@ -187,6 +240,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 
     // epilogue: thread owns output row m0 + 32*warp + lane (a split rank with no k-blocks has
     // issued no MMA and contributes zeros)
+    RowNorm rn;
+    if (ea.ss_in && m0 + warp * 32 + lane < M) rn.rinv = deferred_rinv(ea, m0 + warp * 32 + lane);
     bool ok = nkb == 0 ? true : mbar_wait(done, 0, &abort_flag);
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
@@ -199,7 +254,10 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                 float v[16];
                 tmem_ld16(lane_base + c, v);
                 int n = n0 + c;
-                if (m < M && n < N) epilogue16(epi, ea, m, n, min(16, N - n), v);
+                if (m < M && n < N) {
+                    rn.scale(ea, v);
+                    rn.add(epi, ea, m, n, N, epilogue16(epi, ea, m, n, min(16, N - n), v));
+                }
             }
         }
     } else {
@@ -240,7 +298,10 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                     }
                 }
                 int n = n0 + c;
-                if (m < M && n < N) epilogue16(epi, ea, m, n, min(16, N - n), v);
+                if (m < M && n < N) {
+                    rn.scale(ea, v);
+                    rn.add(epi, ea, m, n, N, epilogue16(epi, ea, m, n, min(16, N - n), v));
+                }
             }
         }
     }

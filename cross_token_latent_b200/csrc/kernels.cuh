@@ -88,7 +88,31 @@ struct EpiArgs {
     int ld_e = 0;
     const float* bias = nullptr;    // Merge: gate bias b_g
     DevHeader* hdr = nullptr;       // error flags (tensor-core path: bounded-wait timeouts)
+    // Deferred RMSNorm (tensor-core paths only; the output width is a multiple of 16).
+    // Producer side (ResidAdd, Merge): with norm_y set, the epilogue also writes
+    // norm_y[m][c] = bf16(x_new[m][c] * norm_g[c]) (leading dim ld_out) and, for every group of
+    // 16 consecutive output columns, ss_out[m * ss_ld + c / 16] = sum of x_new^2 over the group
+    // (one writer per group, fixed summation order).
+    bf16* norm_y = nullptr;
+    const float* norm_g = nullptr;
+    float* ss_out = nullptr;
+    // Consumer side: with ss_in set, accumulator row m is multiplied by
+    // 1 / sqrt(sum_{g < ss_n} ss_in[m * ss_ld + g] / norm_n + eps) before the epilogue, i.e. the
+    // GEMM of bf16(x * g) becomes the GEMM of RMSNorm(x) * g.
+    const float* ss_in = nullptr;
+    int ss_ld = 0, ss_n = 0;
+    float norm_n = 1.f, eps = 0.f;
 };
+// 1 / rms of row m from its 16-column group partials (summed in group order).
+__device__ __forceinline__ float deferred_rinv(const EpiArgs& ea, long long m) {
+    const float* p = ea.ss_in + m * ea.ss_ld;
+    float s = 0.f;
+    for (int g = 0; g < ea.ss_n; g += 4) {
+        float4 q = *reinterpret_cast<const float4*>(p + g);
+        s += q.x; s += q.y; s += q.z; s += q.w;
+    }
+    return 1.0f / sqrtf(s / ea.norm_n + ea.eps);
+}
 // Dispatch: bf16 operands go to the tcgen05 kernel (gemm_tc.cu) when TMA can address them,
 // otherwise (and for float32 models) to the CUDA-core kernel.
 template <typename T>

@@ -3,6 +3,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 #include <string>
 #include <unordered_map>
 #include <unordered_set>
@@ -240,7 +241,7 @@ EncWS enc_ws(const rlt_config& c, int B, int T) {
 }
 
 struct DecWS {
-    size_t x, A, qkv, att, qc, act, logits, part, total;
+    size_t x, A, qkv, att, qc, act, logits, part, xn, ss, total;
 };
 DecWS dec_ws(const rlt_config& c, int B) {
     DecWS w;
@@ -255,6 +256,8 @@ DecWS dec_ws(const rlt_config& c, int B) {
     w.act = take((size_t)B * c.F * e);
     w.logits = take((size_t)B * c.V * 4);
     w.part = take((size_t)XATTN_PART_ITEMS * (c.head_dim + 2) * 4);
+    w.xn = take((size_t)B * d * e);               // bf16(x * g) of a deferred norm
+    w.ss = take((size_t)B * (d / 16) * 4);        // its 16-column sum-of-squares partials
     w.total = off;
     return w;
 }
@@ -361,37 +364,69 @@ rlt_status step_impl(rlt_model* m, uint8_t* state, int B, const T* e, const T* M
     size_t group_elems = (size_t)2 * B * H * (size_t)T_alloc * hd;
     int splits = xattn_splits(c, B, t);
 
+    // Deferred RMSNorm (bf16 tensor-core path): the GEMM that updates the residual stream x
+    // also writes bf16(x * g) and per-row sum-of-squares partials, and the GEMM that consumes
+    // the norm scales its accumulator rows by 1 / rms (row scaling commutes with the product),
+    // so the three sublayer norms of a layer need no launches of their own.
+    T* xn = reinterpret_cast<T*>(ws + w.xn);
+    float* ss = reinterpret_cast<float*>(ws + w.ss);
+    const bool fuse = std::is_same<T, bf16>::value && d % 64 == 0 &&
+                      gemm_tc_supported(xn, d, m->at<T>(m->lay.wqkv[0]), d) &&
+                      gemm_tc_supported(A, 2 * d, m->at<T>(m->lay.merge_w), 2 * d) &&
+                      gemm_tc_supported(att, d, m->at<T>(m->lay.wo[0]), d) &&
+                      gemm_tc_supported(act, F, m->at<T>(m->lay.wdown[0]), F);
+    auto norm_out = [&](EpiArgs& ea, const float* g) {
+        if (!fuse) return;
+        ea.norm_y = reinterpret_cast<bf16*>(xn); ea.norm_g = g; ea.ss_out = ss; ea.ss_ld = d / 16;
+    };
+    auto norm_in = [&](EpiArgs& ea) {
+        if (!fuse) return;
+        ea.ss_in = ss; ea.ss_ld = d / 16; ea.ss_n = d / 16; ea.norm_n = (float)d; ea.eps = c.rms_eps;
+    };
+    // the sublayer input: bf16(x * g) under a deferred norm, else RMSNorm(x) * g from its own kernel
+    auto pre_norm = [&](const float* g) -> cudaError_t {
+        return launch_rmsnorm<T>(L, x, B, d, g, c.rms_eps, A, d, B, B, nullptr);
+    };
+    const T* hin = fuse ? xn : A;
+
     // gated merge: x = e_t + sigmoid(W_ge e_t + W_gs s + b_g) * (W_fb s)
     CKP(RLT_K_MERGE, launch_merge_prep<T>(L, e, T_alloc, t, s, A, B, d, sh, m->version, m->hdr()));
     {
         EpiArgs ea; ea.hdr = m->hdr();
         ea.out_f32 = x; ea.ld_out = d; ea.merge_e = A; ea.ld_e = 2 * d; ea.bias = m->at<float>(m->lay.merge_b);
+        norm_out(ea, m->at<float>(m->lay.attn_norm[0]));
         CKP(RLT_K_MERGE, launch_gemm<T>(L, Epi::Merge, A, 2 * d, m->at<T>(m->lay.merge_w), B, 2 * d, 2 * d, ea));
     }
     for (int l = 0; l < c.L_D; ++l) {
         EpiArgs ea; ea.hdr = m->hdr();
         // sliding-window self-attention (weights of encoder layer l)
-        CKP(RLT_K_NORM, launch_rmsnorm<T>(L, x, B, d, m->at<float>(m->lay.attn_norm[l]), c.rms_eps, A, d, B, B, nullptr));
+        if (!fuse) CKP(RLT_K_NORM, pre_norm(m->at<float>(m->lay.attn_norm[l])));
         ea.out_f32 = qkv; ea.ld_out = 3 * d;
-        CKP(RLT_K_QKV, launch_gemm<T>(L, Epi::StoreF32, A, d, m->at<T>(m->lay.wqkv[l]), B, 3 * d, d, ea));
+        norm_in(ea);
+        CKP(RLT_K_QKV, launch_gemm<T>(L, Epi::StoreF32, hin, d, m->at<T>(m->lay.wqkv[l]), B, 3 * d, d, ea));
         CKP(RLT_K_SWA, launch_swa_decode<T>(L, qkv, rope_row, ring + (size_t)l * ring_layer_elems(c, B), att, B, H, hd,
                                 c.W, t));
         ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = x; ea.ld_out = d;
+        norm_out(ea, m->at<float>(m->lay.xattn_norm[l]));
         CKP(RLT_K_O, launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.wo[l]), B, d, d, ea));
         // cross-attention to M_{<=t}
-        CKP(RLT_K_NORM, launch_rmsnorm<T>(L, x, B, d, m->at<float>(m->lay.xattn_norm[l]), c.rms_eps, A, d, B, B, nullptr));
+        if (!fuse) CKP(RLT_K_NORM, pre_norm(m->at<float>(m->lay.xattn_norm[l])));
         ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = qc; ea.ld_out = d;
-        CKP(RLT_K_QC, launch_gemm<T>(L, Epi::StoreF32, A, d, m->at<T>(m->lay.wqc[l]), B, d, d, ea));
+        norm_in(ea);
+        CKP(RLT_K_QC, launch_gemm<T>(L, Epi::StoreF32, hin, d, m->at<T>(m->lay.wqc[l]), B, d, d, ea));
         const T* Mg = M + (c.G == 1 ? 0 : (size_t)l * group_elems);
         CKP(RLT_K_XATTN, launch_xattn_decode<T>(L, qc, Mg, (long long)B * H * T_alloc * hd, T_alloc, t, att, B, H, hd,
                                                 splits, part));
         ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = x; ea.ld_out = d;
+        norm_out(ea, m->at<float>(m->lay.ffn_norm[l]));
         CKP(RLT_K_OC, launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.woc[l]), B, d, d, ea));
         // SwiGLU FFN (weights of encoder layer l)
-        CKP(RLT_K_NORM, launch_rmsnorm<T>(L, x, B, d, m->at<float>(m->lay.ffn_norm[l]), c.rms_eps, A, d, B, B, nullptr));
+        if (!fuse) CKP(RLT_K_NORM, pre_norm(m->at<float>(m->lay.ffn_norm[l])));
         ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_t = act; ea.ld_out = F;
-        CKP(RLT_K_FFN_UP, launch_gemm<T>(L, Epi::SwiGLU, A, d, m->at<T>(m->lay.wgu[l]), B, 2 * F, d, ea));
+        norm_in(ea);
+        CKP(RLT_K_FFN_UP, launch_gemm<T>(L, Epi::SwiGLU, hin, d, m->at<T>(m->lay.wgu[l]), B, 2 * F, d, ea));
         ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = x; ea.ld_out = d;
+        if (l + 1 < c.L_D) norm_out(ea, m->at<float>(m->lay.attn_norm[l + 1]));
         CKP(RLT_K_FFN_DOWN, launch_gemm<T>(L, Epi::ResidAdd, act, F, m->at<T>(m->lay.wdown[l]), B, d, F, ea));
     }
     // split: s_t = RMSNorm(x) becomes the state; the same s_t feeds the head
