@@ -312,11 +312,13 @@ cudaError_t run_swap(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, i
 template <int NB>
 cudaError_t run_swap_split(int split, Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                            const EpiArgs& ea, DevHeader* hdr) {
+    // one CTA per SM: as many stages as fit next to the split partials (~200 KB)
+    constexpr int ST = NB == 16 ? 10 : (NB == 32 ? 9 : 7);
     switch (split) {
-        case 1: return run_swap<NB, 6, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 2: return run_swap<NB, 6, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 4: return run_swap<NB, 6, 4>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 8: return run_swap<NB, 6, 8>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 1: return run_swap<NB, ST, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 2: return run_swap<NB, ST, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 4: return run_swap<NB, ST, 4>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 8: return run_swap<NB, ST, 8>(L, epi, A, lda, W, M, N, K, ea, hdr);
     }
     return cudaErrorInvalidValue;
 }

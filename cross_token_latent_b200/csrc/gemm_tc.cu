@@ -472,30 +472,32 @@ struct TcVariant {
     int bn, stages, per_sm, split;
 };
 constexpr TcVariant VARIANTS[] = {
-    {32, 5, 2, 1},     // 100 KB
-    {64, 4, 2, 1},     //  96 KB
-    {128, 3, 2, 1},    //  96 KB
-    {128, 5, 1, 1},    // 160 KB
+    // Decode-size grids run one CTA per SM, and a CTA's k-loop advances one ring of STAGES
+    // tiles per TMA round trip, so the narrow tiles fill ~200 KB of shared memory with stages.
+    {32, 10, 1, 1},    // 200 KB
+    {64, 8, 1, 1},     // 192 KB
+    {128, 3, 2, 1},    //  96 KB (two CTAs per SM for grids of up to two waves)
+    {128, 6, 1, 1},    // 192 KB
     {256, 4, 1, 1},    // 192 KB
     {128, 4, 1, 2},    // 128 KB + 64 KB partials
     {128, 4, 1, 4},
-    {64, 4, 1, 2},     //  96 KB + 32 KB partials
-    {64, 4, 1, 4},
+    {64, 7, 1, 2},     // 168 KB + 32 KB partials
+    {64, 7, 1, 4},
 };
 constexpr int N_VARIANTS = sizeof(VARIANTS) / sizeof(VARIANTS[0]);
 
 cudaError_t run_variant(int v, Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                         const EpiArgs& ea, DevHeader* hdr) {
     switch (v) {
-        case 0: return run_tc<32, 5, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 1: return run_tc<64, 4, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 0: return run_tc<32, 10, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 1: return run_tc<64, 8, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
         case 2: return run_tc<128, 3, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 3: return run_tc<128, 5, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 3: return run_tc<128, 6, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
         case 4: return run_tc<256, 4, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
         case 5: return run_tc<128, 4, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
         case 6: return run_tc<128, 4, 4>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 7: return run_tc<64, 4, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 8: return run_tc<64, 4, 4>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 7: return run_tc<64, 7, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 8: return run_tc<64, 7, 4>(L, epi, A, lda, W, M, N, K, ea, hdr);
     }
     return cudaErrorInvalidValue;
 }

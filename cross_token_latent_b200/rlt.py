@@ -168,11 +168,13 @@ class RLTModel:
                "rlt_model_create")
         self.handle = h
         self._ws: dict = {}
+        self._destroy = lib().rlt_model_destroy    # held so that teardown at exit still reaches it
 
     def __del__(self):
         h = getattr(self, "handle", None)
-        if h:
-            lib().rlt_model_destroy(h)
+        destroy = getattr(self, "_destroy", None)
+        if h and destroy is not None:
+            destroy(h)
             self.handle = None
 
     # ---------------------------------------------------------------- weights

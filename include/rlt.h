@@ -234,8 +234,8 @@ uint64_t rlt_launch_count(const rlt_model* m);
  * accumulation/output, on the model's stream-ordered error flags.  kernel 0 = the
  * tensor-core (tcgen05 + TMA) kernel and tile shape the library's own projections use for
  * this shape (row tiles, or the few-row kernel below), kernel 1 =
- * the CUDA-core kernel, kernel 2 + v = tensor-core tile variant v (0: 128x32 tiles, 5 stages;
- * 1: 128x64, 4; 2: 128x128, 3; 3: 128x128, 5; 4: 128x256, 4; then K split over a cluster of
+ * the CUDA-core kernel, kernel 2 + v = tensor-core tile variant v (0: 128x32 tiles, 10 stages;
+ * 1: 128x64, 8; 2: 128x128, 3; 3: 128x128, 6; 4: 128x256, 4; then K split over a cluster of
  * CTAs with a shared-memory reduction: 5: 128x128 split 2; 6: 128x128 split 4; 7: 128x64
  * split 2; 8: 128x64 split 4), kernel 11 + s (M <= 64 only) = the few-row kernel with the
  * weights on the MMA's M side and K split over a cluster of (s = 0: chosen, 1: 1, 2: 2, 3: 4,
