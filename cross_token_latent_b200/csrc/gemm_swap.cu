@@ -29,7 +29,8 @@ struct SwShape {
     static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
     static constexpr int TMEM_COLS = NB < 32 ? 32 : NB;
     static constexpr int ROWS_PER_OWNER = FM / SPLIT;
-    static constexpr int RECV_BYTES = SPLIT > 1 ? FM * NB * 4 : 0;
+    static constexpr int RECV_LD = NB + 4;        // padded pitch (floats): lanes fall in different banks
+    static constexpr int RECV_BYTES = SPLIT > 1 ? FM * RECV_LD * 4 : 0;
     static constexpr int SMEM = STAGES * STAGE_BYTES + RECV_BYTES + 1024 + 256;
 };
 
@@ -146,22 +147,25 @@ k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
     if (warp == 0 && lane == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmW) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmX) : "memory");
+        // every CTA reads the same activation k-blocks: rotate the start (as in gemm_tc.cu)
+        const int rot = nkb > 0 ? (int)(blockIdx.x % (unsigned)nkb) : 0;
+        auto kx = [&](int kb) { return (kb0 + (kb + rot) % nkb) * KB; };
         const int pre = nkb < STAGES ? nkb : STAGES;
         for (int kb = 0; kb < pre; ++kb) {
             mbar_expect_tx(&full[kb], S::STAGE_BYTES);
-            tma_load_2d(smem + kb * S::STAGE_BYTES, &tmW, &full[kb], (kb0 + kb) * KB, f0);
+            tma_load_2d(smem + kb * S::STAGE_BYTES, &tmW, &full[kb], kx(kb), f0);
         }
         pdl_wait();
         for (int kb = 0; kb < pre; ++kb)
-            tma_load_2d(smem + kb * S::STAGE_BYTES + W_BYTES, &tmX, &full[kb], (kb0 + kb) * KB, b0);
+            tma_load_2d(smem + kb * S::STAGE_BYTES + W_BYTES, &tmX, &full[kb], kx(kb), b0);
         for (int kb = pre; kb < nkb; ++kb) {
             int s = kb % STAGES;
             uint32_t ph = (kb / STAGES) & 1;
             if (!mbar_wait(&empty[s], ph ^ 1, &abort_flag)) { abort_flag = 1; break; }
             uint8_t* st = smem + s * S::STAGE_BYTES;
             mbar_expect_tx(&full[s], S::STAGE_BYTES);
-            tma_load_2d(st, &tmW, &full[s], (kb0 + kb) * KB, f0);
-            tma_load_2d(st + W_BYTES, &tmX, &full[s], (kb0 + kb) * KB, b0);
+            tma_load_2d(st, &tmW, &full[s], kx(kb), f0);
+            tma_load_2d(st + W_BYTES, &tmX, &full[s], kx(kb), b0);
         }
     } else if (warp == 1 && lane == 0) {
         constexpr uint32_t idesc = idesc_bf16(FM, NB);
@@ -225,7 +229,7 @@ k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
 #pragma unroll
                     for (int j = 0; j < 16; ++j) v[j] = 0.f;
                 }
-                dsmem_store16(recv + ((size_t)rank * S::ROWS_PER_OWNER + r_local) * NB + c, owner, v);
+                dsmem_store16(recv + ((size_t)rank * S::ROWS_PER_OWNER + r_local) * S::RECV_LD + c, owner, v);
             }
         }
         cluster_arrive_release();
@@ -241,7 +245,7 @@ k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
                 for (int j = 0; j < 16; ++j) v[j] = 0.f;
                 for (int src = 0; src < SPLIT; ++src) {
                     const float4* p = reinterpret_cast<const float4*>(
-                        recv + ((size_t)src * S::ROWS_PER_OWNER + r_local) * NB + c);
+                        recv + ((size_t)src * S::ROWS_PER_OWNER + r_local) * S::RECV_LD + c);
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         float4 q = p[j];

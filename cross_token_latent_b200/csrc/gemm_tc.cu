@@ -141,16 +141,18 @@ struct TcShape {
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int TMEM_COLS = BN < 32 ? 32 : BN;
     // split-K: the owner CTA of a row band receives every rank's partial rows here
-    static constexpr int ROWS_PER_OWNER = BM / SPLIT;
-    static constexpr int RECV_BYTES = SPLIT > 1 ? BM * BN * 4 : 0;
+    static constexpr int BAND = BN / SPLIT;          // split-K: output columns each rank owns
+    static constexpr int RECV_LD = BAND + 4;         // padded row pitch (floats) of the partials
+    static constexpr int RECV_BYTES = SPLIT > 1 ? SPLIT * BM * RECV_LD * 4 : 0;
+    static_assert(SPLIT == 1 || BAND % 16 == 0, "column bands are whole 16-column chunks");
     static constexpr int SMEM = STAGES * STAGE_BYTES + RECV_BYTES + 1024 + 256;
 };
 
 // SPLIT > 1: the grid's z dimension splits the k-blocks over a cluster of SPLIT CTAs that
 // compute the same output tile.  Each CTA accumulates its share in its own TMEM, then sends
-// every partial row to the CTA that owns the row band (BM / SPLIT rows per rank) through
-// distributed shared memory; the owner adds the SPLIT partials in rank order (the same order
-// for every element and every run) and applies the epilogue.
+// each column band of its partial tile (BN / SPLIT columns per rank) to the CTA that owns the
+// band through distributed shared memory; the owner adds the SPLIT partials in rank order (the
+// same order for every element and every run) and applies the epilogue with all 128 threads.
 template <int BN, int STAGES, int SPLIT>
 __global__ void __launch_bounds__(128, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW, int M, int N, int K,
@@ -261,10 +263,12 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
             }
         }
     } else {
-        // send this warp's 32 partial rows to the owner of their band
-        const int row = warp * 32 + lane;                        // row within the tile
-        const uint32_t owner = (uint32_t)(row / S::ROWS_PER_OWNER);
-        const int row_local = row - (int)owner * S::ROWS_PER_OWNER;
+        // Column bands: rank r owns output columns [r * BAND, (r + 1) * BAND) of the tile for
+        // all 128 rows, so every thread keeps its row.  It sends each band of its partial row
+        // to that band's owner (rows BAND + 4 floats apart: consecutive lanes fall in different
+        // banks), then adds the SPLIT partials of its own band in rank order (the same order
+        // for every element and every run) and applies the epilogue.
+        const int row = warp * 32 + lane;
         cluster_wait_acquire();                                  // every CTA of the cluster has started
         if (ok) {
 #pragma unroll 1
@@ -276,28 +280,27 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 #pragma unroll
                     for (int j = 0; j < 16; ++j) v[j] = 0.f;
                 }
-                dsmem_store16(recv + ((size_t)rank * S::ROWS_PER_OWNER + row_local) * BN + c, owner, v);
+                dsmem_store16(recv + ((size_t)rank * BM + row) * S::RECV_LD + c % S::BAND, (uint32_t)(c / S::BAND), v);
             }
         }
         cluster_arrive_release();
         cluster_wait_acquire();                                  // all partials have landed
-        if (ok && owner == rank) {
+        if (ok) {
             const int m = m0 + row;
 #pragma unroll 1
-            for (int c = 0; c < BN; c += 16) {
+            for (int c = 0; c < S::BAND; c += 16) {
                 float v[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) v[j] = 0.f;
                 for (int src = 0; src < SPLIT; ++src) {
-                    const float4* p = reinterpret_cast<const float4*>(
-                        recv + ((size_t)src * S::ROWS_PER_OWNER + row_local) * BN + c);
+                    const float4* p = reinterpret_cast<const float4*>(recv + ((size_t)src * BM + row) * S::RECV_LD + c);
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         float4 q = p[j];
                         v[4 * j] += q.x; v[4 * j + 1] += q.y; v[4 * j + 2] += q.z; v[4 * j + 3] += q.w;
                     }
                 }
-                int n = n0 + c;
+                int n = n0 + (int)rank * S::BAND + c;
                 if (m < M && n < N) {
                     rn.scale(ea, v);
                     rn.add(epi, ea, m, n, N, epilogue16(epi, ea, m, n, min(16, N - n), v));
@@ -547,6 +550,8 @@ bool gemm_tc_supported(const void* A, int lda, const void* W, int K) {
 cudaError_t launch_gemm_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                            const EpiArgs& ea, DevHeader* hdr, int variant) {
     int v = (variant >= 0 && variant < N_VARIANTS) ? variant : pick_variant(M, N, K);
+    // a merge's deferred-norm group spans 32 GEMM columns and must stay in one column band
+    if (epi == Epi::Merge && ea.norm_y && VARIANTS[v].split > 1 && VARIANTS[v].bn / VARIANTS[v].split < 32) v = 7;
     return run_variant(v, L, epi, A, lda, W, M, N, K, ea, hdr);
 }
 
