@@ -278,13 +278,15 @@ class RLTModel:
                                 _ptr(st.buf) if st else None, _ptr(ws), ws.numel(), _stream()), "rlt_replay")
         return score, lp, st
 
-    def gemm_bf16(self, A: torch.Tensor, W: torch.Tensor, kernel: int = 0) -> torch.Tensor:
-        """C = A W^T (bf16 in, float32 out) with the library's tensor-core (0) or CUDA-core (1) kernel."""
+    def gemm_bf16(self, A: torch.Tensor, W: torch.Tensor, kernel: int = 0,
+                  out: torch.Tensor | None = None) -> torch.Tensor:
+        """C = A W^T (bf16 in, float32 out) with the kernel id of rlt_gemm_bf16 (0: the library's
+        choice, 1: CUDA cores, 2 + v: row-tile variant v, 11 + s: few-row kernel)."""
         A = A.to(self.device, torch.bfloat16).contiguous()
         W = W.to(self.device, torch.bfloat16).contiguous()
         M, K = A.shape
         N = W.shape[0]
-        C = torch.empty((M, N), dtype=torch.float32, device=self.device)
+        C = torch.empty((M, N), dtype=torch.float32, device=self.device) if out is None else out
         _check(lib().rlt_gemm_bf16(self.handle, _ptr(A), _ptr(W), _ptr(C), M, N, K, kernel, _stream()),
                "rlt_gemm_bf16")
         return C
