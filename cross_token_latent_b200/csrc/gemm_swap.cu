@@ -47,24 +47,29 @@ __device__ __forceinline__ void epilogue16_t(Epi epi, const EpiArgs& ea, int n, 
             for (int j = 0; j < 16; ++j)
                 if (store && mb + j < M) ea.out_f32[(long long)(mb + j) * ea.ld_out + n] = v[j] * ea.scale;
             break;
-        case Epi::ResidAdd:
+        case Epi::ResidAdd: {
+            // all 16 residual loads first: with a runtime row pitch the compiler cannot tell a
+            // store from the next row's load, and would otherwise wait out one round trip per row
+            float x[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) x[j] = (store && mb + j < M) ? ea.out_f32[(long long)(mb + j) * ea.ld_out + n] : 0.f;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const long long m = mb + j;
-                float x = 0.f;
+                x[j] += v[j];
                 if (store && m < M) {
-                    x = ea.out_f32[m * ea.ld_out + n] + v[j];
-                    ea.out_f32[m * ea.ld_out + n] = x;
-                    if (ea.norm_y) ea.norm_y[m * ea.ld_out + n] = __float2bfloat16_rn(x * ea.norm_g[n]);
+                    ea.out_f32[m * ea.ld_out + n] = x[j];
+                    if (ea.norm_y) ea.norm_y[m * ea.ld_out + n] = __float2bfloat16_rn(x[j] * ea.norm_g[n]);
                 }
                 if (ea.norm_y) {
-                    float sq = x * x;
+                    float sq = (store && m < M) ? x[j] * x[j] : 0.f;
 #pragma unroll
                     for (int o = 8; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
                     if (store && m < M && (n & 15) == 0) ea.ss_out[m * ea.ss_ld + n / 16] = sq;
                 }
             }
             break;
+        }
         case Epi::SwiGLU: {     // feature 2c = gate_c, 2c+1 = up_c
             bf16* o = reinterpret_cast<bf16*>(ea.out_t);
 #pragma unroll
@@ -78,13 +83,18 @@ __device__ __forceinline__ void epilogue16_t(Epi epi, const EpiArgs& ea, int n, 
         case Epi::Merge: {      // feature 2c = gate pre-activation, 2c+1 = feedback projection
             const bf16* e = reinterpret_cast<const bf16*>(ea.merge_e);
             const int c = n / 2;
+            const bool lead = store && !(n & 1);
+            const float bias = lead ? ea.bias[c] : 0.f;
+            float ev[16];                       // loads first (see ResidAdd)
+#pragma unroll
+            for (int j = 0; j < 16; ++j) ev[j] = (lead && mb + j < M) ? __bfloat162float(e[(long long)(mb + j) * ea.ld_e + c]) : 0.f;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const long long m = mb + j;
                 float u = __shfl_xor_sync(0xffffffffu, v[j], 1);
                 float x = 0.f;
-                if (store && !(n & 1) && m < M) {
-                    x = __bfloat162float(e[m * ea.ld_e + c]) + sigmoidf_(v[j] + ea.bias[c]) * u;
+                if (lead && m < M) {
+                    x = ev[j] + sigmoidf_(v[j] + bias) * u;
                     ea.out_f32[m * ea.ld_out + c] = x;
                     if (ea.norm_y) ea.norm_y[m * ea.ld_out + c] = __float2bfloat16_rn(x * ea.norm_g[c]);
                 }

@@ -96,6 +96,29 @@ __device__ __forceinline__ float epilogue16(Epi epi, const EpiArgs& ea, int m, i
         case Epi::Merge: {      // columns 2j = gate pre-activation, 2j+1 = feedback projection
             const bf16* e = reinterpret_cast<const bf16*>(ea.merge_e) + (long long)m * ea.ld_e;
             float* o = ea.out_f32 + (long long)m * ea.ld_out;
+            if (cnt == 16) {
+                // output columns c0 .. c0+7 (c0 a multiple of 8): vector loads of e and the bias
+                // before any store
+                const int c0 = n / 2;
+                float ev[8], bv[8], x[8];
+                Vec16<bf16>::unpack(ld16(e + c0), ev);
+                Vec16<float>::unpack(ld16(ea.bias + c0), bv);
+                Vec16<float>::unpack(ld16(ea.bias + c0 + 4), bv + 4);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) x[j] = ev[j] + sigmoidf_(v[2 * j] + bv[j]) * v[2 * j + 1];
+                st16(o + c0, Vec16<float>::pack(x));
+                st16(o + c0 + 4, Vec16<float>::pack(x + 4));
+                if (ea.norm_y) {
+                    float y[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        y[j] = x[j] * ea.norm_g[c0 + j];
+                        ss += x[j] * x[j];
+                    }
+                    st16(ea.norm_y + (long long)m * ea.ld_out + c0, Vec16<bf16>::pack(y));
+                }
+                break;
+            }
             for (int j = 0; j + 1 < cnt; j += 2) {
                 int c = (n + j) / 2;
                 float x = __bfloat162float(e[c]) + sigmoidf_(v[j] + ea.bias[c]) * v[j + 1];
