@@ -29,8 +29,8 @@ struct SwShape {
     static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
     static constexpr int TMEM_COLS = NB < 32 ? 32 : NB;
     static constexpr int ROWS_PER_OWNER = FM / SPLIT;
-    static constexpr int RECV_LD = NB + 4;        // padded pitch (floats): lanes fall in different banks
-    static constexpr int RECV_BYTES = SPLIT > 1 ? FM * RECV_LD * 4 : 0;
+    // the owner's partials, batch-column-major per source rank: [SPLIT][NB][ROWS_PER_OWNER]
+    static constexpr int RECV_BYTES = SPLIT > 1 ? SPLIT * NB * ROWS_PER_OWNER * 4 : 0;
     static constexpr int SMEM = STAGES * STAGE_BYTES + RECV_BYTES + 1024 + 256;
 };
 
@@ -239,7 +239,9 @@ k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
 #pragma unroll
                     for (int j = 0; j < 16; ++j) v[j] = 0.f;
                 }
-                dsmem_store16(recv + ((size_t)rank * S::ROWS_PER_OWNER + r_local) * S::RECV_LD + c, owner, v);
+                // for every batch column the band's consecutive features are contiguous
+                dsmem_store16_strided(recv + ((size_t)rank * NB + c) * S::ROWS_PER_OWNER + r_local,
+                                      S::ROWS_PER_OWNER, owner, v);
             }
         }
         cluster_arrive_release();
@@ -254,13 +256,9 @@ k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
 #pragma unroll
                 for (int j = 0; j < 16; ++j) v[j] = 0.f;
                 for (int src = 0; src < SPLIT; ++src) {
-                    const float4* p = reinterpret_cast<const float4*>(
-                        recv + ((size_t)src * S::ROWS_PER_OWNER + r_local) * S::RECV_LD + c);
+                    const float* p = recv + ((size_t)src * NB + c) * S::ROWS_PER_OWNER + r_local;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        float4 q = p[j];
-                        v[4 * j] += q.x; v[4 * j + 1] += q.y; v[4 * j + 2] += q.z; v[4 * j + 3] += q.w;
-                    }
+                    for (int j = 0; j < 16; ++j) v[j] += p[j * S::ROWS_PER_OWNER];
                 }
                 scale(c, v);
                 epilogue16_t(epi, ea, n, n_ok && mine, b0 + c, M, v);

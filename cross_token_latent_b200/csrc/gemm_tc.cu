@@ -165,8 +165,8 @@ struct TcShape {
     static constexpr int TMEM_COLS = BN < 32 ? 32 : BN;
     // split-K: the owner CTA of a row band receives every rank's partial rows here
     static constexpr int BAND = BN / SPLIT;          // split-K: output columns each rank owns
-    static constexpr int RECV_LD = BAND + 4;         // padded row pitch (floats) of the partials
-    static constexpr int RECV_BYTES = SPLIT > 1 ? SPLIT * BM * RECV_LD * 4 : 0;
+    // the owner's partials, column-major per source rank: [SPLIT][BAND][BM] floats
+    static constexpr int RECV_BYTES = SPLIT > 1 ? SPLIT * BAND * BM * 4 : 0;
     static_assert(SPLIT == 1 || BAND % 16 == 0, "column bands are whole 16-column chunks");
     static constexpr int SMEM = STAGES * STAGE_BYTES + RECV_BYTES + 1024 + 256;
 };
@@ -288,9 +288,10 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     } else {
         // Column bands: rank r owns output columns [r * BAND, (r + 1) * BAND) of the tile for
         // all 128 rows, so every thread keeps its row.  It sends each band of its partial row
-        // to that band's owner (rows BAND + 4 floats apart: consecutive lanes fall in different
-        // banks), then adds the SPLIT partials of its own band in rank order (the same order
-        // for every element and every run) and applies the epilogue.
+        // to that band's owner, column-major (for every column a warp's 32 rows are 128
+        // contiguous bytes, so each remote store instruction is one coalesced transfer), then
+        // adds the SPLIT partials of its own band in rank order (the same order for every
+        // element and every run) and applies the epilogue.
         const int row = warp * 32 + lane;
         cluster_wait_acquire();                                  // every CTA of the cluster has started
         if (ok) {
@@ -303,7 +304,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 #pragma unroll
                     for (int j = 0; j < 16; ++j) v[j] = 0.f;
                 }
-                dsmem_store16(recv + ((size_t)rank * BM + row) * S::RECV_LD + c % S::BAND, (uint32_t)(c / S::BAND), v);
+                dsmem_store16_strided(recv + ((size_t)rank * S::BAND + c % S::BAND) * BM + row, BM,
+                                      (uint32_t)(c / S::BAND), v);
             }
         }
         cluster_arrive_release();
@@ -316,12 +318,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 #pragma unroll
                 for (int j = 0; j < 16; ++j) v[j] = 0.f;
                 for (int src = 0; src < SPLIT; ++src) {
-                    const float4* p = reinterpret_cast<const float4*>(recv + ((size_t)src * BM + row) * S::RECV_LD + c);
+                    const float* p = recv + ((size_t)src * S::BAND + c) * BM + row;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        float4 q = p[j];
-                        v[4 * j] += q.x; v[4 * j + 1] += q.y; v[4 * j + 2] += q.z; v[4 * j + 3] += q.w;
-                    }
+                    for (int j = 0; j < 16; ++j) v[j] += p[j * BM];
                 }
                 int n = n0 + (int)rank * S::BAND + c;
                 if (m < M && n < N) {

@@ -147,16 +147,16 @@ __device__ __forceinline__ uint32_t cluster_rank() {
 __device__ __forceinline__ void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory"); }
 __device__ __forceinline__ void cluster_arrive_release() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait_acquire() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
-// Store 16 floats into the shared memory of cluster CTA `rank` at the address that `local`
-// has in this CTA (distributed shared memory).
-__device__ __forceinline__ void dsmem_store16(const float* local, uint32_t rank, const float* v) {
+// Store 16 floats v[j] into the shared memory of cluster CTA `rank` at the addresses that
+// local + j * stride (floats) have in this CTA (distributed shared memory).  Used with lanes on
+// consecutive `local` addresses, so that each store instruction of a warp is one contiguous
+// transfer.
+__device__ __forceinline__ void dsmem_store16_strided(const float* local, int stride, uint32_t rank, const float* v) {
     uint32_t remote;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
 #pragma unroll
-    for (int j = 0; j < 16; j += 4)
-        asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(remote + 4 * j), "f"(v[j]),
-                     "f"(v[j + 1]), "f"(v[j + 2]), "f"(v[j + 3])
-                     : "memory");
+    for (int j = 0; j < 16; ++j)
+        asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote + 4u * (uint32_t)(j * stride)), "f"(v[j]) : "memory");
 }
 
 
