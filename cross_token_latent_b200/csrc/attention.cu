@@ -34,56 +34,73 @@ __device__ __forceinline__ float group_sum(float v) {
     return v;
 }
 
-// Accumulate keys [0, n) of K/V (row stride HD) into this lane group's running softmax.
+// One round of the key loop: KPI * U keys starting at `base`, one 16-byte piece of a K row and
+// of a V row per lane and key (zeros past n).
+template <typename T, int HD, int U, bool STREAM>
+__device__ __forceinline__ void load_round(const T* __restrict__ K, const T* __restrict__ V, int n, int base, int g,
+                                           int li, uint4* kr, uint4* vr) {
+    using G = Geom<T, HD>;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        int j = base + u * G::KPI + g;
+        if (j < n) {
+            const T* kp = K + (long long)j * HD + li * G::EPL;
+            const T* vp = V + (long long)j * HD + li * G::EPL;
+            kr[u] = STREAM ? ld16_stream(kp) : ld16(kp);
+            vr[u] = STREAM ? ld16_stream(vp) : ld16(vp);
+        } else {
+            kr[u] = make_uint4(0, 0, 0, 0);
+            vr[u] = make_uint4(0, 0, 0, 0);
+        }
+    }
+}
+
+// Fold one loaded round into this lane group's running softmax (m, l, acc).
+template <typename T, int HD, int U>
+__device__ __forceinline__ void consume_round(const float* q, int n, int base, int g, const uint4* kr, const uint4* vr,
+                                              float& m, float& l, float* acc) {
+    using G = Geom<T, HD>;
+    constexpr int EPL = G::EPL, LPK = G::LPK, KPI = G::KPI;
+    float s[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        float kf[EPL];
+        Vec16<T>::unpack(kr[u], kf);
+        float dot = 0.f;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) dot = fmaf(q[i], kf[i], dot);
+        dot = group_sum<LPK>(dot);
+        s[u] = (base + u * KPI + g < n) ? dot : NEG_BIG;
+    }
+    float mx = m;
+#pragma unroll
+    for (int u = 0; u < U; ++u) mx = fmaxf(mx, s[u]);
+    float corr = exp2f(m - mx);
+    l *= corr;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) acc[i] *= corr;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        float p = (base + u * KPI + g < n) ? exp2f(s[u] - mx) : 0.f;
+        l += p;
+        float vf[EPL];
+        Vec16<T>::unpack(vr[u], vf);
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) acc[i] = fmaf(p, vf[i], acc[i]);
+    }
+    m = mx;
+}
+
+// Accumulate keys [base0, n) of K/V (row stride HD) into this lane group's running softmax.
 // q is pre-scaled by log2(e)/sqrt(hd).  n must be warp-uniform.
 template <typename T, int HD, int U, bool STREAM>
 __device__ __forceinline__ void attend(const float* q, const T* __restrict__ K, const T* __restrict__ V,
-                                       int n, int g, int li, float& m, float& l, float* acc) {
+                                       int n, int g, int li, float& m, float& l, float* acc, int base0 = 0) {
     using G = Geom<T, HD>;
-    constexpr int EPL = G::EPL, LPK = G::LPK, KPI = G::KPI;
-    for (int base = 0; base < n; base += KPI * U) {
+    for (int base = base0; base < n; base += G::KPI * U) {
         uint4 kr[U], vr[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            int j = base + u * KPI + g;
-            if (j < n) {
-                const T* kp = K + (long long)j * HD + li * EPL;
-                const T* vp = V + (long long)j * HD + li * EPL;
-                kr[u] = STREAM ? ld16_stream(kp) : ld16(kp);
-                vr[u] = STREAM ? ld16_stream(vp) : ld16(vp);
-            } else {
-                kr[u] = make_uint4(0, 0, 0, 0);
-                vr[u] = make_uint4(0, 0, 0, 0);
-            }
-        }
-        float s[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            float kf[EPL];
-            Vec16<T>::unpack(kr[u], kf);
-            float dot = 0.f;
-#pragma unroll
-            for (int i = 0; i < EPL; ++i) dot = fmaf(q[i], kf[i], dot);
-            dot = group_sum<LPK>(dot);
-            s[u] = (base + u * KPI + g < n) ? dot : NEG_BIG;
-        }
-        float mx = m;
-#pragma unroll
-        for (int u = 0; u < U; ++u) mx = fmaxf(mx, s[u]);
-        float corr = exp2f(m - mx);
-        l *= corr;
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) acc[i] *= corr;
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            float p = (base + u * KPI + g < n) ? exp2f(s[u] - mx) : 0.f;
-            l += p;
-            float vf[EPL];
-            Vec16<T>::unpack(vr[u], vf);
-#pragma unroll
-            for (int i = 0; i < EPL; ++i) acc[i] = fmaf(p, vf[i], acc[i]);
-        }
-        m = mx;
+        load_round<T, HD, U, STREAM>(K, V, n, base, g, li, kr, vr);
+        consume_round<T, HD, U>(q, n, base, g, kr, vr, m, l, acc);
     }
 }
 
@@ -132,6 +149,22 @@ __global__ void __launch_bounds__(SWA_WARPS * 32, 6) k_swa_decode(const float* _
     const int b = item / H, h = item % H;
     const int d = H * HD, half = HD / 2;
     const float* row = qkv + (long long)b * 3 * d + h * HD;
+    // this warp's share of the ring; its first round of loads is issued before q is formed, so
+    // the ring's memory latency overlaps the q / RoPE loads instead of following them
+    T* Kr = nullptr;
+    T* Vr = nullptr;
+    int j0 = 0, nj = 0;
+    if (W > 1) {
+        Kr = ring + (((long long)b * 2 + 0) * H + h) * (long long)(W - 1) * HD;
+        Vr = ring + (((long long)b * 2 + 1) * H + h) * (long long)(W - 1) * HD;
+        int n = min(t - 1, W - 1);
+        int per = (n + SWA_WARPS - 1) / SWA_WARPS;
+        j0 = min(n, warp * per);
+        nj = min(n, j0 + per) - j0;
+    }
+    constexpr int SWA_U = 4;
+    uint4 kr0[SWA_U], vr0[SWA_U];
+    load_round<T, HD, SWA_U, true>(Kr + (long long)j0 * HD, Vr + (long long)j0 * HD, nj, 0, g, li, kr0, vr0);
     float q[EPL];
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
@@ -168,16 +201,10 @@ __global__ void __launch_bounds__(SWA_WARPS * 32, 6) k_swa_decode(const float* _
             sm_kv[1][li] = Vec16<T>::pack(v);
         }
     }
-    T* Kr = nullptr;
-    T* Vr = nullptr;
-    if (W > 1) {
-        Kr = ring + (((long long)b * 2 + 0) * H + h) * (long long)(W - 1) * HD;
-        Vr = ring + (((long long)b * 2 + 1) * H + h) * (long long)(W - 1) * HD;
-        int n = min(t - 1, W - 1);
-        int per = (n + SWA_WARPS - 1) / SWA_WARPS;
-        int j0 = min(n, warp * per);
-        int nj = min(n, j0 + per) - j0;
-        attend<T, HD, 4, true>(q, Kr + (long long)j0 * HD, Vr + (long long)j0 * HD, nj, g, li, m, l, acc);
+    if (nj > 0) {
+        consume_round<T, HD, SWA_U>(q, nj, 0, g, kr0, vr0, m, l, acc);
+        attend<T, HD, SWA_U, true>(q, Kr + (long long)j0 * HD, Vr + (long long)j0 * HD, nj, g, li, m, l, acc,
+                                   Geom<T, HD>::KPI * SWA_U);
     }
     merge_groups<T, HD>(m, l, acc);
     if (g == 0) {

@@ -538,7 +538,12 @@ int pick_variant(int M, int N, int K) {
     for (int v = 4; v >= 0; --v) {
         const TcVariant& t = VARIANTS[v];
         long long tiles = mt * ((N + t.bn - 1) / t.bn);
-        if (tiles <= 148LL * t.per_sm && tiles >= 74 && nkb <= 16) return v;
+        if (tiles <= 148LL * t.per_sm && tiles >= 74 && nkb <= 16) {
+            // 32-wide tiles re-read the activation panel from L2 for every 32 output columns;
+            // 64-wide tiles with K split in two give as many CTAs for half that traffic
+            if (v == 0 && mt * ((N + 63) / 64) * 2 <= 148 && nkb >= 8) return 7;
+            return v;
+        }
     }
     long long tiles256 = mt * ((N + 255) / 256);
     if (tiles256 > 148) return 4;
