@@ -22,6 +22,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 from pathlib import Path
 
@@ -126,7 +127,7 @@ class ClockSampler:
     def __init__(self, gpu_id: str):
         self.gpu_id = gpu_id
         self.proc = None
-        self.out = ROOT / "gpurun_out" / f"clocks_{os.getpid()}.csv"
+        self.out = Path(tempfile.gettempdir()) / f"rlt_bench_clocks_{os.getpid()}.csv"
 
     def __enter__(self):
         try:
