@@ -360,21 +360,24 @@ bool gemm_swap_preferred(int M, int N, int K) {
     return base >= 48 && base <= 148;
 }
 
+// Fill one wave of SMs with at least two k-blocks per rank.  Clusters of 8 are left out: at
+// one CTA per SM not every GPC holds two of them, so a 128-CTA grid of 8-CTA clusters runs in
+// two waves (measured 2.2x the time of the 4-way split).
+int gemm_swap_auto_split(int M, int N, int K) {
+    const long long base = swap_base(M, N);
+    const int nkb = (K + KB - 1) / KB;
+    int split = 1;
+    for (int s : {2, 4})
+        if (base * s <= 148 && nkb >= 2 * s) split = s;
+    return split;
+}
+
 cudaError_t launch_gemm_swap(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                              const EpiArgs& ea, DevHeader* hdr, int split) {
     if (!gemm_swap_supported(M)) return cudaErrorInvalidValue;
     const int nb = swap_nb(M);
     if (ea.norm_y && split > 4) split = 4;      // a deferred-norm group must stay in one owner band
-    if (split <= 0) {
-        // fill one wave of SMs with at least two k-blocks per rank.  Clusters of 8 are left
-        // out: at one CTA per SM not every GPC holds two of them, so a 128-CTA grid of 8-CTA
-        // clusters runs in two waves (measured 2.2x the time of the 4-way split).
-        const long long base = swap_base(M, N);
-        const int nkb = (K + KB - 1) / KB;
-        split = 1;
-        for (int s : {2, 4})
-            if (base * s <= 148 && nkb >= 2 * s) split = s;
-    }
+    if (split <= 0) split = gemm_swap_auto_split(M, N, K);
     if (nb == 16) return run_swap_split<16>(split, L, epi, A, lda, W, M, N, K, ea, hdr);
     if (nb == 32) return run_swap_split<32>(split, L, epi, A, lda, W, M, N, K, ea, hdr);
     return run_swap_split<64>(split, L, epi, A, lda, W, M, N, K, ea, hdr);

@@ -568,6 +568,8 @@ int pick_variant(int M, int N, int K) {
 
 int gemm_tc_variants() { return N_VARIANTS; }
 
+int gemm_tc_pick(int M, int N, int K) { return pick_variant(M, N, K); }
+
 bool gemm_tc_supported(const void* A, int lda, const void* W, int K) {
     // TMA: 16-byte aligned base addresses and row pitches
     return (reinterpret_cast<uintptr_t>(A) % 16 == 0) && (reinterpret_cast<uintptr_t>(W) % 16 == 0) &&

@@ -125,6 +125,8 @@ cudaError_t launch_gemm_simt(Launch L, Epi epi, const T* A, int lda, const T* W,
 // ------------------------------------------------------------------ gemm_tc.cu
 bool gemm_tc_supported(const void* A, int lda, const void* W, int K);
 int gemm_tc_variants();
+// the row-tile variant the library picks for an M x N x K product (host logic only)
+int gemm_tc_pick(int M, int N, int K);
 // variant < 0: pick the tile shape from (M, N); otherwise force tile variant `variant`.
 cudaError_t launch_gemm_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                            const EpiArgs& ea, DevHeader* hdr, int variant = -1);
@@ -134,6 +136,8 @@ cudaError_t launch_gemm_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16
 // cluster of 1, 2, 4 or 8 CTAs (0: choose).
 bool gemm_swap_supported(int M);
 bool gemm_swap_preferred(int M, int N, int K);
+// the K split (1, 2 or 4) the few-row kernel picks when asked to choose (host logic only)
+int gemm_swap_auto_split(int M, int N, int K);
 cudaError_t launch_gemm_swap(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                              const EpiArgs& ea, DevHeader* hdr, int split = 0);
 

@@ -763,6 +763,15 @@ rlt_status rlt_last_error(rlt_model* m, void* stream) {
 
 uint64_t rlt_launch_count(const rlt_model* m) { return m ? m->launches : 0; }
 
+int rlt_gemm_plan(int M, int N, int K) {
+    if (M < 1 || N < 1 || K < 1) return -1;
+    if (gemm_swap_preferred(M, N, K)) {
+        const int s = gemm_swap_auto_split(M, N, K);
+        return 11 + (s == 1 ? 1 : (s == 2 ? 2 : (s == 4 ? 3 : 4)));
+    }
+    return 2 + gemm_tc_pick(M, N, K);
+}
+
 rlt_status rlt_gemm_bf16(rlt_model* m, const void* A, const void* W, float* C, int M, int N, int K, int kernel,
                          void* stream) {
     const int n_tc = gemm_tc_variants();

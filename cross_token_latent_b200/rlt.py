@@ -70,6 +70,7 @@ _EXPORTS = {
     "rlt_launch_count": (ctypes.c_uint64, [ctypes.c_void_p]),
     "rlt_gemm_bf16": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                      ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    "rlt_gemm_plan": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int]),
     "rlt_profile_start": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_uint32]),
     "rlt_profile_stop": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_double),
                                         ctypes.POINTER(ctypes.c_uint64)]),
@@ -96,6 +97,11 @@ def lib() -> ctypes.CDLL:
 
 def exported_names() -> list[str]:
     return list(_EXPORTS)
+
+
+def gemm_plan(M: int, N: int, K: int) -> int:
+    """Kernel id (as rlt_gemm_bf16 numbers them) the library picks for an M x N x K bf16 product."""
+    return lib().rlt_gemm_plan(M, N, K)
 
 
 def _check(code: int, what: str) -> None:

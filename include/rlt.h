@@ -245,6 +245,13 @@ uint64_t rlt_launch_count(const rlt_model* m);
 rlt_status rlt_gemm_bf16(rlt_model* m, const void* A, const void* W, float* C, int M, int N, int K,
                          int kernel, void* stream);
 
+/* The kernel id (numbered as for rlt_gemm_bf16: 2 + v for row-tile variant v, 11 + s for the
+ * few-row kernel with split s = 1: 1, 2: 2, 3: 4) that the library's own projections use for an
+ * M x N x K bf16 product whose operands TMA can address, before any epilogue-specific
+ * adjustment.  Pure host logic: no device, model or stream is touched.  Returns -1 for
+ * non-positive sizes. */
+int rlt_gemm_plan(int M, int N, int K);
+
 /* ---------------------------------------------------------------- kernel timing */
 
 /* Kernel kinds of the decoder step (and the encoder as one kind) for live timing. */
