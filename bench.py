@@ -218,7 +218,15 @@ def oracle_steps_for(wl) -> int:
 
 # ----------------------------------------------------------------------------- reference arm
 
-def run_reference(args, wl, rank: int) -> None:
+def arm_config(wl, B: int, T: int, world: int) -> dict:
+    """The workload description both arms print (the reference arm adds its sample)."""
+    return {"workload": wl.name, "B_per_gpu": B, "T": T, "global_batch": world * B, "seq_len": T,
+            "parallelism": f"replicas x{world} (sequences sharded, no data-path collective)",
+            "l2": "inputs larger than L2 (M, SWA cache and weights stream from HBM every step)",
+            "step": "one full decoder sweep of T lockstep transitions with next-token log-prob gather"}
+
+
+def run_reference(args, wl, rank: int, world: int) -> None:
     if rank != 0:
         return
     steps = oracle_steps_for(wl)
@@ -230,10 +238,10 @@ def run_reference(args, wl, rank: int) -> None:
     value = statistics.median(vals)
     cores = blas_threads()
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * steps / value,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "sample": desc},
+        "config": {**arm_config(wl, wl.B, wl.T, world), "sample": desc},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -289,7 +297,7 @@ def main() -> int:
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
     if args.impl == "reference":
-        run_reference(args, wl, rank)
+        run_reference(args, wl, rank, world)
         return 0
 
     import torch
@@ -449,10 +457,7 @@ def main() -> int:
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": m.dtype, "data": "synthetic",
-            "config": {"workload": wl.name, "B_per_gpu": B, "T": T, "global_batch": world * B, "seq_len": T,
-                       "parallelism": f"replicas x{world} (sequences sharded, no data-path collective)",
-                       "l2": "inputs larger than L2 (M, SWA cache and weights stream from HBM every step)",
-                       "step": "one full decoder sweep of T lockstep transitions with next-token log-prob gather"},
+            "config": arm_config(wl, B, T, world),
             "roofline": roofline, "step_roofline": step_roofline, "cpu_baseline": cpu, "e2e": e2e,
             "replay": replay, "gpu_launches": launches, "clocks": clocks,
             "kernel_breakdown_ms_per_sweep": {k: round(v[0], 3) for k, v in sorted(breakdown.items())},
