@@ -87,6 +87,15 @@ def kind_cost(kind: str, m, B: int, T: int) -> tuple[str, float]:
     return "hbm", 0.0
 
 
+def encode_flops(m, B: int, T: int) -> float:
+    """FLOPs of one rlt_encode over B sequences of T tokens: 2 per weight and token for the
+    encoder layers (q/k/v/o 4d^2, SwiGLU 3dF) and the G memory projections (2d^2 each), plus the
+    causal attention (q k^T and p v: 4 * hd FLOPs per (query, key <= query) pair and head)."""
+    lin = 2.0 * B * T * (m.L_E * (4 * m.d * m.d + 3 * m.d * m.F) + m.G * 2 * m.d * m.d)
+    att = 4.0 * m.L_E * B * m.n_heads * m.head_dim * T * (T + 1) / 2
+    return lin + att
+
+
 def run_roofline_s(m, B: int, T: int, peaks: dict, m_once: bool = False) -> float:
     bw = peaks["hbm_gbs"] * 1e9
     fl = peaks["bf16_tflops"] * 1e12
@@ -432,6 +441,22 @@ def main() -> int:
                "d2h_bytes_per_step": int(lp_host.numel() * 4), "ms_per_step": e_ms,
                "includes": "H2D tokens, rlt_encode, T rlt_decode_step calls, D2H log-probs"}
 
+    # the encoder on its own (the rlt_encode call of the e2e path), tensor-bound
+    enc = None
+    if not args.no_e2e:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        model.encode(tok, out=(e, M))
+        a.record()
+        model.encode(tok, out=(e, M))
+        b.record()
+        torch.cuda.synchronize()
+        enc_ms = max_over_ranks(a.elapsed_time(b), dev)
+        ef = encode_flops(m, B, T)
+        enc_roof_ms = 1e3 * ef / (peaks["bf16_tflops"] * 1e12)
+        enc = {"ms": enc_ms, "tflop": ef / 1e12, "achieved_tflops": ef / (enc_ms / 1e3) / 1e12,
+               "peak_tflops": peaks["bf16_tflops"], "roofline_ms": enc_roof_ms, "frac": enc_roof_ms / enc_ms,
+               "note": "one rlt_encode of the whole batch; FLOPs of the linear maps and the causal attention"}
+
     replay = None
     if not args.no_replay:
         P = torch.full((B,), wl.prompt_len, dtype=torch.int32, device=dev)
@@ -443,8 +468,11 @@ def main() -> int:
         b.record()
         torch.cuda.synchronize()
         r_ms = max_over_ranks(a.elapsed_time(b), dev)
+        r_roof_ms = 1e3 * rr + 1e3 * encode_flops(m, B, T) / (peaks["bf16_tflops"] * 1e12)
         replay = {"value": world * B * T / (r_ms / 1e3), "unit": "tokens/s", "ms": r_ms,
-                  "includes": "rlt_replay: encode + T steps + response scoring"}
+                  "roofline_ms": r_roof_ms, "frac": r_roof_ms / r_ms,
+                  "includes": "rlt_replay: encode + T steps + response scoring",
+                  "roofline_note": "decoder run roofline + encoder FLOPs at the bf16 burst peak"}
     model.check_device_errors()
 
     cpu = None
@@ -459,7 +487,7 @@ def main() -> int:
             "vs_baseline": None, "dtype": m.dtype, "data": "synthetic",
             "config": arm_config(wl, B, T, world),
             "roofline": roofline, "step_roofline": step_roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "replay": replay, "gpu_launches": launches, "clocks": clocks,
+            "replay": replay, "encode": enc, "gpu_launches": launches, "clocks": clocks,
             "kernel_breakdown_ms_per_sweep": {k: round(v[0], 3) for k, v in sorted(breakdown.items())},
         }
         print(json.dumps(line), flush=True)

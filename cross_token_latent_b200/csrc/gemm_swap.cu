@@ -154,13 +154,16 @@ k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    const uint64_t lim = ea.wait_ns;
+    int armed = 0;                     // producer: k-blocks whose loads have been issued
     if (warp == 0 && lane == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmW) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmX) : "memory");
         // every CTA reads the same activation k-blocks: rotate the start (as in gemm_tc.cu)
         const int rot = nkb > 0 ? (int)(blockIdx.x % (unsigned)nkb) : 0;
         auto kx = [&](int kb) { return (kb0 + (kb + rot) % nkb) * KB; };
-        const int pre = nkb < STAGES ? nkb : STAGES;
+        // the bounded-wait self-test (ea.no_loads) issues nothing
+        const int pre = ea.no_loads ? 0 : (nkb < STAGES ? nkb : STAGES);
         for (int kb = 0; kb < pre; ++kb) {
             mbar_expect_tx(&full[kb], S::STAGE_BYTES);
             tma_load_2d(smem + kb * S::STAGE_BYTES, &tmW, &full[kb], kx(kb), f0);
@@ -168,21 +171,24 @@ k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
         pdl_wait();
         for (int kb = 0; kb < pre; ++kb)
             tma_load_2d(smem + kb * S::STAGE_BYTES + W_BYTES, &tmX, &full[kb], kx(kb), b0);
-        for (int kb = pre; kb < nkb; ++kb) {
+        armed = pre;
+        for (int kb = pre; kb < nkb && !ea.no_loads; ++kb) {
             int s = kb % STAGES;
             uint32_t ph = (kb / STAGES) & 1;
-            if (!mbar_wait(&empty[s], ph ^ 1, &abort_flag)) { abort_flag = 1; break; }
+            if (!mbar_wait(&empty[s], ph ^ 1, &abort_flag, lim)) { abort_flag = 1; break; }
             uint8_t* st = smem + s * S::STAGE_BYTES;
             mbar_expect_tx(&full[s], S::STAGE_BYTES);
             tma_load_2d(st, &tmW, &full[s], kx(kb), f0);
             tma_load_2d(st + W_BYTES, &tmX, &full[s], kx(kb), b0);
+            armed = kb + 1;
         }
     } else if (warp == 1 && lane == 0) {
+        // after a timeout the issuer stops but still commits `done` (see gemm_tc.cu)
         constexpr uint32_t idesc = idesc_bf16(FM, NB);
         for (int kb = 0; kb < nkb; ++kb) {
             int s = kb % STAGES;
             uint32_t ph = (kb / STAGES) & 1;
-            if (!mbar_wait(&full[s], ph, &abort_flag)) { abort_flag = 1; break; }
+            if (!mbar_wait(&full[s], ph, &abort_flag, lim)) { abort_flag = 1; break; }
             tc_fence_after();
             uint8_t* st = smem + s * S::STAGE_BYTES;
             uint64_t dw = sdesc_sw128(st), dx = sdesc_sw128(st + W_BYTES);
@@ -211,8 +217,8 @@ k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
             for (int j = 0; j < 16; ++j) v[j] *= rinv_s[c + j];
         }
     };
-    bool ok = nkb == 0 ? true : mbar_wait(done, 0, &abort_flag);
-    ok = __all_sync(0xffffffffu, ok);
+    bool ok = nkb == 0 ? true : mbar_wait(done, 0, nullptr, lim);
+    ok = __syncthreads_and(ok) && abort_flag == 0;      // no partial accumulator is stored
     tc_fence_after();
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     if constexpr (SPLIT == 1) {
@@ -265,9 +271,11 @@ k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
             }
         }
     }
-    if (!ok && lane == 0) {
-        abort_flag = 1;
+    if (!ok && threadIdx.x == 0) {
         raise_flag(hdr, ERR_TIMEOUT);
+        // wait (bounded) for the loads this CTA still has in flight before it exits
+        for (int kb = armed > STAGES ? armed - STAGES : 0; kb < armed; ++kb)
+            mbar_wait(&full[kb % STAGES], (kb / STAGES) & 1, nullptr, lim);
     }
     tc_fence_before();
     __syncthreads();

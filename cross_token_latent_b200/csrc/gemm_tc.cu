@@ -219,13 +219,15 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    const uint64_t lim = ea.wait_ns;
+    int armed = 0;                     // producer: k-blocks whose loads have been issued
     if (warp == 0 && lane == 0) {
         // TMA producer.  Weight tiles do not depend on the previous kernel: the first stages'
         // W loads are issued before the programmatic-launch dependency wait, the activation
-        // (A) loads after it.
+        // (A) loads after it.  The bounded-wait self-test (ea.no_loads) issues nothing.
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmW) : "memory");
-        const int pre = nkb < STAGES ? nkb : STAGES;
+        const int pre = ea.no_loads ? 0 : (nkb < STAGES ? nkb : STAGES);
         for (int kb = 0; kb < pre; ++kb) {
             uint8_t* a = smem + kb * S::STAGE_BYTES;
             mbar_expect_tx(&full[kb], S::STAGE_BYTES);
@@ -234,22 +236,25 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         pdl_wait();
         for (int kb = 0; kb < pre; ++kb)
             tma_load_2d(smem + kb * S::STAGE_BYTES, &tmA, &full[kb], (kb0 + kb) * BK, m0);
-        for (int kb = pre; kb < nkb; ++kb) {
+        armed = pre;
+        for (int kb = pre; kb < nkb && !ea.no_loads; ++kb) {
             int s = kb % STAGES;
             uint32_t ph = (kb / STAGES) & 1;
-            if (!mbar_wait(&empty[s], ph ^ 1, &abort_flag)) { abort_flag = 1; break; }
+            if (!mbar_wait(&empty[s], ph ^ 1, &abort_flag, lim)) { abort_flag = 1; break; }
             uint8_t* a = smem + s * S::STAGE_BYTES;
             mbar_expect_tx(&full[s], S::STAGE_BYTES);
             tma_load_2d(a, &tmA, &full[s], (kb0 + kb) * BK, m0);
             tma_load_2d(a + A_BYTES, &tmW, &full[s], (kb0 + kb) * BK, n0);
+            armed = kb + 1;
         }
     } else if (warp == 1 && lane == 0) {
-        // MMA issuer
+        // MMA issuer.  After a timeout it stops issuing but still commits `done`, which then
+        // tracks the MMAs already issued, so that none is in flight when TMEM is freed.
         constexpr uint32_t idesc = idesc_bf16(BM, BN);
         for (int kb = 0; kb < nkb; ++kb) {
             int s = kb % STAGES;
             uint32_t ph = (kb / STAGES) & 1;
-            if (!mbar_wait(&full[s], ph, &abort_flag)) { abort_flag = 1; break; }
+            if (!mbar_wait(&full[s], ph, &abort_flag, lim)) { abort_flag = 1; break; }
             tc_fence_after();
             uint8_t* a = smem + s * S::STAGE_BYTES;
             uint64_t da = sdesc_sw128(a), dw = sdesc_sw128(a + A_BYTES);
@@ -267,8 +272,10 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     // issued no MMA and contributes zeros)
     RowNorm rn;
     if (ea.ss_in && m0 + warp * 32 + lane < M) rn.rinv = deferred_rinv(ea, m0 + warp * 32 + lane);
-    bool ok = nkb == 0 ? true : mbar_wait(done, 0, &abort_flag);
-    ok = __all_sync(0xffffffffu, ok);
+    bool ok = nkb == 0 ? true : mbar_wait(done, 0, nullptr, lim);
+    // a producer or issuer that gave up raised abort_flag before this barrier: no thread then
+    // stores a partial accumulator
+    ok = __syncthreads_and(ok) && abort_flag == 0;
     tc_fence_after();
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     if constexpr (SPLIT == 1) {
@@ -330,9 +337,13 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
             }
         }
     }
-    if (!ok && lane == 0) {
-        abort_flag = 1;
-        raise_flag(hdr, ERR_TIMEOUT);
+    if (!ok) {
+        if (threadIdx.x == 0) {
+            raise_flag(hdr, ERR_TIMEOUT);
+            // wait (bounded) for the loads this CTA still has in flight before it exits
+            for (int kb = armed > STAGES ? armed - STAGES : 0; kb < armed; ++kb)
+                mbar_wait(&full[kb % STAGES], (kb / STAGES) & 1, nullptr, lim);
+        }
     }
     tc_fence_before();
     __syncthreads();

@@ -88,6 +88,11 @@ struct EpiArgs {
     int ld_e = 0;
     const float* bias = nullptr;    // Merge: gate bias b_g
     DevHeader* hdr = nullptr;       // error flags (tensor-core path: bounded-wait timeouts)
+    // Tensor-core kernels: limit of every mbarrier wait (%globaltimer nanoseconds).  no_loads is
+    // the bounded-wait self-test: the kernel issues no TMA load and no MMA, so its first wait
+    // runs out after wait_ns and the launch latches ERR_TIMEOUT without writing any output.
+    unsigned long long wait_ns = 2000000000ull;
+    int no_loads = 0;
     // Deferred RMSNorm (tensor-core paths only; the output width is a multiple of 16).
     // Producer side (ResidAdd, Merge): with norm_y set, the epilogue also writes
     // norm_y[m][c] = bf16(x_new[m][c] * norm_g[c]) (leading dim ld_out) and, for every group of

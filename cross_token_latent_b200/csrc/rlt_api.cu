@@ -147,6 +147,7 @@ struct rlt_model {
     std::vector<std::string> required;
     std::unordered_map<const void*, StateInfo> states;
     uint64_t launches = 0;
+    int device = -1;            // the CUDA device that holds the arena
 
     DevHeader* hdr() const { return reinterpret_cast<DevHeader*>(arena); }
     template <typename T> T* at(size_t off) const { return reinterpret_cast<T*>(arena + off); }
@@ -487,7 +488,13 @@ rlt_status rlt_model_create(const rlt_config* cfg, void* arena, size_t arena_byt
     if (!cfg || !out || !arena || !config_ok(*cfg) || !aligned(arena)) return RLT_EINVAL;
     Layout lay = make_layout(*cfg);
     if (arena_bytes < lay.total) return RLT_EINVAL;
+    cudaPointerAttributes pa;
+    if (cudaPointerGetAttributes(&pa, arena) != cudaSuccess || pa.type != cudaMemoryTypeDevice) {
+        cudaGetLastError();
+        return RLT_EINVAL;
+    }
     rlt_model* m = new rlt_model();
+    m->device = pa.device;
     m->cfg = *cfg;
     m->lay = lay;
     m->arena = reinterpret_cast<uint8_t*>(arena);
@@ -660,9 +667,7 @@ constexpr int NOALLOC_MAX_DEVICES = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[NOALLOC_MAX_DEVICES] = {};
 
-rlt_status noalloc_scratch_for_current_device(void** out) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) return RLT_ECUDA;
+rlt_status noalloc_scratch_for_device(int dev, void** out) {
     if (dev < 0 || dev >= NOALLOC_MAX_DEVICES) return RLT_EUNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
     if (!g_noalloc_ptr[dev]) {
@@ -684,8 +689,12 @@ rlt_status rlt_decode_step_noalloc(rlt_model* m, void* state, int B, const void*
     size_t need = rlt_decode_workspace_bytes(m, B);
     if (need == 0) return RLT_EINVAL;
     if (need > NOALLOC_SCRATCH_BYTES) return RLT_EUNSUPPORTED;   // batch too large for the static scratch
+    // the scratch looked up below belongs to the current device: it must be the model's
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return RLT_ECUDA;
+    if (dev != m->device) return RLT_EINVAL;
     void* scratch = nullptr;
-    rlt_status st = noalloc_scratch_for_current_device(&scratch);
+    rlt_status st = noalloc_scratch_for_device(dev, &scratch);
     if (st != RLT_OK) return st;
     // Every workspace buffer of a step is fully written before it is read, so nothing in the
     // shared scratch has to start at zero.
@@ -790,6 +799,31 @@ rlt_status rlt_gemm_bf16(rlt_model* m, const void* A, const void* W, float* C, i
     } else if (kernel == 1) {
         CK(launch_gemm_simt<bf16>(L, Epi::StoreF32, a, K, w, M, N, K, ea));
     } else if (kernel <= 1 + n_tc) {
+        CK(launch_gemm_tc(L, Epi::StoreF32, a, K, w, M, N, K, ea, m->hdr(), kernel - 2));
+    } else {
+        static const int splits[5] = {0, 1, 2, 4, 8};
+        CK(launch_gemm_swap(L, Epi::StoreF32, a, K, w, M, N, K, ea, m->hdr(), splits[kernel - 2 - n_tc]));
+    }
+    return RLT_OK;
+}
+
+rlt_status rlt_selftest_wait_timeout(rlt_model* m, const void* A, const void* W, float* C, int M, int N, int K,
+                                     int kernel, uint64_t wait_ns, void* stream) {
+    const int n_tc = gemm_tc_variants();
+    if (!m || !A || !W || !C || M < 1 || N < 1 || K < 1 || kernel < 2 || kernel > 1 + n_tc + 5) return RLT_EINVAL;
+    if (kernel > 1 + n_tc && !gemm_swap_supported(M)) return RLT_EINVAL;
+    if (!aligned(A, 16) || !aligned(W, 16) || !aligned(C, 16) || K % 8 || N % 4) return RLT_EINVAL;
+    if (wait_ns < 1000 || wait_ns > 2000000000ull) return RLT_EINVAL;
+    Launch L = m->launch(stream);
+    EpiArgs ea;
+    ea.hdr = m->hdr();
+    ea.out_f32 = C;
+    ea.ld_out = N;
+    ea.wait_ns = wait_ns;
+    ea.no_loads = 1;
+    const bf16* a = reinterpret_cast<const bf16*>(A);
+    const bf16* w = reinterpret_cast<const bf16*>(W);
+    if (kernel <= 1 + n_tc) {
         CK(launch_gemm_tc(L, Epi::StoreF32, a, K, w, M, N, K, ea, m->hdr(), kernel - 2));
     } else {
         static const int splits[5] = {0, 1, 2, 4, 8};

@@ -37,14 +37,16 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait for the phase with the given parity.  False on timeout or abort.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// Bounded wait for the phase with the given parity.  False on timeout (limit_ns of
+// %globaltimer) or when *abort is set (abort may be NULL).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns = WAIT_LIMIT_NS) {
     if (mbar_try(bar, parity)) return true;
     uint64_t t0 = globaltimer();
     while (true) {
         if (mbar_try(bar, parity)) return true;
-        if (*abort) return false;
-        if (globaltimer() - t0 > WAIT_LIMIT_NS) return false;
+        if (abort && *abort) return false;
+        if (globaltimer() - t0 > limit_ns) return false;
     }
 }
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {

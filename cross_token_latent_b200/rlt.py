@@ -71,6 +71,9 @@ _EXPORTS = {
     "rlt_gemm_bf16": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                      ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "rlt_gemm_plan": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "rlt_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                 ctypes.c_uint64, ctypes.c_void_p]),
     "rlt_profile_start": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_uint32]),
     "rlt_profile_stop": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_double),
                                         ctypes.POINTER(ctypes.c_uint64)]),
@@ -296,6 +299,15 @@ class RLTModel:
         _check(lib().rlt_gemm_bf16(self.handle, _ptr(A), _ptr(W), _ptr(C), M, N, K, kernel, _stream()),
                "rlt_gemm_bf16")
         return C
+
+    def selftest_wait_timeout(self, A: torch.Tensor, W: torch.Tensor, C: torch.Tensor, kernel: int,
+                              wait_ns: int) -> None:
+        """Launch tensor-core kernel `kernel` in its no-load self-test mode (every wait bounded by
+        wait_ns); the next last_error() reports RLT_ETIMEOUT."""
+        M, K = A.shape
+        N = W.shape[0]
+        _check(lib().rlt_selftest_wait_timeout(self.handle, _ptr(A), _ptr(W), _ptr(C), M, N, K, kernel,
+                                               int(wait_ns), _stream()), "rlt_selftest_wait_timeout")
 
     def profile_start(self, kinds=None) -> None:
         """Bracket every launch of the given kernel kinds (names of KERNEL_KINDS) with CUDA events."""

@@ -84,7 +84,8 @@ size_t rlt_weights_bytes(const rlt_config* cfg);
 /* Create a model handle over a caller-owned device arena of at least
  * rlt_weights_bytes(cfg) bytes.  The arena must stay allocated until
  * rlt_model_destroy.  Fills the rotary table and clears the device header on
- * `stream`.  Errors: RLT_EINVAL (bad config, NULL, small or misaligned arena),
+ * `stream`.  The device that holds the arena is the model's device.  Errors: RLT_EINVAL
+ * (bad config, NULL, small or misaligned arena, or an arena that is not device memory),
  * RLT_ECUDA. */
 rlt_status rlt_model_create(const rlt_config* cfg, void* arena, size_t arena_bytes,
                             void* stream, rlt_model** out);
@@ -191,6 +192,8 @@ rlt_status rlt_decode_step(rlt_model* m, void* state, int B, const void* e, cons
  *     needs any of it to start at zero).  Calls that overlap on the GPU race on it: issue them
  *     on one stream, or order them with events, one at a time.
  *   - It calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - The calling thread's current device must be the one that holds the model's arena (the
+ *     array used is the current device's copy); otherwise the call returns RLT_EINVAL.
  * Errors: RLT_EUNSUPPORTED when rlt_decode_workspace_bytes(m, B) exceeds the array (checked
  * on the host before anything is launched); otherwise those of rlt_decode_step, plus
  * RLT_ECUDA if the array's address cannot be obtained. */
@@ -251,6 +254,18 @@ rlt_status rlt_gemm_bf16(rlt_model* m, const void* A, const void* W, float* C, i
  * adjustment.  Pure host logic: no device, model or stream is touched.  Returns -1 for
  * non-positive sizes. */
 int rlt_gemm_plan(int M, int N, int K);
+
+/* Self-test of the bounded device waits (no counterpart on the pages: a library check of its
+ * own failure detection).  Launches tensor-core kernel `kernel` (an id of rlt_gemm_bf16 >= 2)
+ * on the shape M x N x K in a mode that issues no TMA load and no MMA, with every mbarrier
+ * wait bounded by `wait_ns` nanoseconds (1e3 .. 2e9).  The kernel's first wait therefore
+ * runs out; each CTA latches RLT_ETIMEOUT in the model's device flags, frees its tensor
+ * memory and returns without writing C.  The next rlt_last_error() reports RLT_ETIMEOUT and
+ * clears it; the model and the CUDA context stay usable.  A, W and C must satisfy
+ * rlt_gemm_bf16's rules (they are described to TMA but never read or written).
+ * Errors: RLT_EINVAL, RLT_ECUDA. */
+rlt_status rlt_selftest_wait_timeout(rlt_model* m, const void* A, const void* W, float* C, int M, int N, int K,
+                                     int kernel, uint64_t wait_ns, void* stream);
 
 /* ---------------------------------------------------------------- kernel timing */
 

@@ -54,3 +54,20 @@ def test_shared_memory_bound_is_stricter_only_for_a_shared_memory():
     b = bench.run_roofline_s(per_layer.model, per_layer.B, per_layer.T, PEAKS)
     b1 = bench.run_roofline_s(per_layer.model, per_layer.B, per_layer.T, PEAKS, m_once=True)
     assert b1 == b
+
+
+# encoder FLOPs of each workload, derived by hand (linear maps + causal attention), in TFLOP
+EXPECTED_ENCODE_TF = {"300m-12+12-b512": 227.0, "replay-24+24-b64": 402.0, "ref-48+48-b32": 754.0,
+                      "ref-48+48-b1": 23.6}
+
+
+@pytest.mark.parametrize("name", sorted(EXPECTED_ENCODE_TF))
+def test_encode_flops_match_the_derived_table(name):
+    wl = WORKLOADS[name]
+    assert bench.encode_flops(wl.model, wl.B, wl.T) / 1e12 == pytest.approx(EXPECTED_ENCODE_TF[name], rel=4e-3)
+
+
+def test_encode_flops_of_one_token_is_two_per_weight_plus_its_self_attention():
+    m = WORKLOADS["tiny-f32"].model
+    per_weight = 2.0 * (m.L_E * (4 * m.d * m.d + 3 * m.d * m.F) + m.G * 2 * m.d * m.d)
+    assert bench.encode_flops(m, 1, 1) == per_weight + 4.0 * m.L_E * m.d

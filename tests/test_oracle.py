@@ -4,6 +4,7 @@ Each test fixes the oracle to a closed form, an invariant the pages state, a
 library routine, or a brute-force textbook pass, chosen so that a dropped term,
 a wrong sign, a wrong index or a transposed operand fails at least one of them.
 """
+import math
 from dataclasses import replace
 
 import numpy as np
@@ -201,6 +202,126 @@ def test_gate_limits():
     np.testing.assert_allclose(opened.merge(e_t, s), e_t + s @ w["merge_fb"].astype(np.float64).T, atol=1e-13)
     zero_fb = RLTOracle(TINY_M, no_feedback(w))
     np.testing.assert_array_equal(zero_fb.merge(e_t, s), e_t)
+
+
+def _expit(x: float) -> float:
+    return 1.0 / (1.0 + math.exp(-x))
+
+
+def _merge_model(ge=None, gs=None, fb=None, bias=None, cls=RLTOracle):
+    """TINY with chosen merge weights (others as drawn); returns (oracle, d)."""
+    w = make_weights(TINY_M)
+    d = TINY_M.d
+    for name, val in (("merge_ge", ge), ("merge_gs", gs), ("merge_fb", fb), ("merge_bias", bias)):
+        if val is not None:
+            w[name] = np.asarray(val, np.float32)
+    return cls(TINY_M, w), d
+
+
+def test_merge_interior_gate_reads_e_and_feedback_reads_s(cls=RLTOracle):
+    """Gate weights on e only (W_gs = 0), feedback the identity: x0_i = e_i + expit((W_ge e)_i) s_i,
+    computed here element by element.  A gate fed s instead of e, or a feedback applied to e,
+    gives different values."""
+    rng = np.random.default_rng(11)
+    d = TINY_M.d
+    ge = rng.standard_normal((d, d)) * 0.3
+    o, _ = _merge_model(ge=ge, gs=np.zeros((d, d)), fb=np.eye(d), bias=np.zeros(d), cls=cls)
+    e_t, s = rng.standard_normal((2, d)), rng.standard_normal((2, d))
+    got = o.merge(e_t, s)
+    ge32 = ge.astype(np.float32).astype(np.float64)
+    for b in range(2):
+        for i in range(d):
+            pre = sum(ge32[i, j] * e_t[b, j] for j in range(d))
+            assert abs(got[b, i] - (e_t[b, i] + _expit(pre) * s[b, i])) < 1e-12
+
+
+def test_merge_interior_state_gate_and_feedback_projection(cls=RLTOracle):
+    """W_ge = 0: x0_i = e_i + expit((W_gs s)_i + b_i) (W_fb s)_i with a nonzero bias and a dense
+    W_fb, element by element.  A bias outside the sigmoid or dropped, or W_fb applied to e,
+    gives different values."""
+    rng = np.random.default_rng(12)
+    d = TINY_M.d
+    gs = rng.standard_normal((d, d)) * 0.3
+    fb = rng.standard_normal((d, d)) * 0.3
+    bias = rng.standard_normal(d)
+    o, _ = _merge_model(ge=np.zeros((d, d)), gs=gs, fb=fb, bias=bias, cls=cls)
+    e_t, s = rng.standard_normal((2, d)), rng.standard_normal((2, d))
+    got = o.merge(e_t, s)
+    gs32, fb32, b32 = (a.astype(np.float32).astype(np.float64) for a in (gs, fb, bias))
+    for b in range(2):
+        for i in range(d):
+            g = _expit(sum(gs32[i, j] * s[b, j] for j in range(d)) + b32[i])
+            u = sum(fb32[i, j] * s[b, j] for j in range(d))
+            assert abs(got[b, i] - (e_t[b, i] + g * u)) < 1e-12
+
+
+def test_merge_interior_single_entry_weights_fix_every_index(cls=RLTOracle):
+    """One nonzero entry per merge matrix pins which input component reaches which output:
+    W_ge[0, 1] = 2, W_gs[0, 2] = -1, W_fb[0, 3] = 1.5, bias b_0 = log 3 (so the gate of an
+    all-zero pre-activation is 3/4).  Output 0 is e_0 + expit(2 e_1 - s_2 + log 3) * 1.5 s_3;
+    every other output i has gate expit(b_i) = 1/2 times a zero feedback, i.e. e_i.  A
+    transposed operand moves the nonzero terms to other components."""
+    d = TINY_M.d
+    ge, gs, fb = np.zeros((d, d)), np.zeros((d, d)), np.zeros((d, d))
+    ge[0, 1], gs[0, 2], fb[0, 3] = 2.0, -1.0, 1.5
+    bias = np.zeros(d)
+    bias[0] = math.log(3.0)
+    o, _ = _merge_model(ge=ge, gs=gs, fb=fb, bias=bias, cls=cls)
+    rng = np.random.default_rng(13)
+    e_t, s = rng.standard_normal((3, d)), rng.standard_normal((3, d))
+    got = o.merge(e_t, s)
+    b0 = float(np.float32(math.log(3.0)))
+    for b in range(3):
+        want0 = e_t[b, 0] + _expit(2.0 * e_t[b, 1] - s[b, 2] + b0) * 1.5 * s[b, 3]
+        assert abs(got[b, 0] - want0) < 1e-12
+        np.testing.assert_array_equal(got[b, 1:], e_t[b, 1:])
+    # with every weight zero the gate is expit(b_0) = 3/4 on a zero feedback: x0 = e
+    o0, _ = _merge_model(ge=np.zeros((d, d)), gs=np.zeros((d, d)), fb=np.eye(d), bias=bias, cls=cls)
+    got0 = o0.merge(e_t, s)
+    np.testing.assert_allclose(got0[:, 0], e_t[:, 0] + 0.75 * s[:, 0], atol=1e-7)
+    np.testing.assert_allclose(got0[:, 1:], e_t[:, 1:] + 0.5 * s[:, 1:], atol=1e-15)
+
+
+class _SwappedGateInputs(RLTOracle):       # s_{t-1} fed to W_ge and e_t to W_gs
+    def merge(self, e_t, s_prev):
+        s_in = self.rnd(s_prev)
+        g = 1 / (1 + np.exp(-(s_in @ self.w["merge_ge"].T + e_t @ self.w["merge_gs"].T + self.w["merge_bias"])))
+        return e_t + g * (s_in @ self.w["merge_fb"].T)
+
+
+class _FeedbackOnE(RLTOracle):             # W_fb applied to e_t
+    def merge(self, e_t, s_prev):
+        s_in = self.rnd(s_prev)
+        g = 1 / (1 + np.exp(-(e_t @ self.w["merge_ge"].T + s_in @ self.w["merge_gs"].T + self.w["merge_bias"])))
+        return e_t + g * (e_t @ self.w["merge_fb"].T)
+
+
+class _BiasOutsideGate(RLTOracle):         # b_g added after the sigmoid
+    def merge(self, e_t, s_prev):
+        s_in = self.rnd(s_prev)
+        g = 1 / (1 + np.exp(-(e_t @ self.w["merge_ge"].T + s_in @ self.w["merge_gs"].T))) + self.w["merge_bias"]
+        return e_t + g * (s_in @ self.w["merge_fb"].T)
+
+
+class _TransposedFeedback(RLTOracle):      # W_fb^T instead of W_fb
+    def merge(self, e_t, s_prev):
+        s_in = self.rnd(s_prev)
+        g = 1 / (1 + np.exp(-(e_t @ self.w["merge_ge"].T + s_in @ self.w["merge_gs"].T + self.w["merge_bias"])))
+        return e_t + g * (s_in @ self.w["merge_fb"])
+
+
+@pytest.mark.parametrize("wrong", [_SwappedGateInputs, _FeedbackOnE, _BiasOutsideGate, _TransposedFeedback])
+def test_merge_pins_catch_planted_mistakes(wrong):
+    """Each plausible mistake, planted in a copy of the oracle, fails at least one merge pin."""
+    failed = 0
+    for pin in (test_merge_interior_gate_reads_e_and_feedback_reads_s,
+                test_merge_interior_state_gate_and_feedback_projection,
+                test_merge_interior_single_entry_weights_fix_every_index):
+        try:
+            pin(cls=wrong)
+        except AssertionError:
+            failed += 1
+    assert failed >= 1
 
 
 # ---------------------------------------------------------------- head

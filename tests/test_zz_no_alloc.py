@@ -14,21 +14,23 @@ import torch
 
 from cross_token_latent_b200 import RLTError
 from workloads import TINY, SMALL, make_tokens, make_weights
-from gpu_util import build_model, cosine, to_np
+from gpu_util import build_model, to_np
 
 pytestmark = pytest.mark.gpu
 
 CASES = {
-    # model, batch, tolerance on log-probs, on s (float32: max abs; bf16: cosine)
-    "tiny-f32": (TINY.model, 2, 1e-4),
-    "small-bf16": (SMALL.model, 64, 5e-2),
-    "tiny-bf16-wide-batch": (replace(TINY.model, dtype="bf16", W=5), 300, 5e-2),
+    # model, batch
+    "tiny-f32": (TINY.model, 2),
+    "small-bf16": (SMALL.model, 64),
+    "tiny-bf16-wide-batch": (replace(TINY.model, dtype="bf16", W=5), 300),
 }
 
 
 @pytest.mark.parametrize("name", list(CASES))
 def test_noalloc_step_matches_decode_step_on_two_calls(name):
-    cfg, B, tol = CASES[name]
+    """Both entry points launch the same deterministic kernels on the same inputs; only the
+    scratch address differs, so every output is identical bit for bit."""
+    cfg, B = CASES[name]
     T = 16
     model = build_model(cfg, max_pos=T, weights=make_weights(cfg, seed=4))
     tok = np.random.default_rng([9, B]).integers(0, cfg.V, size=(B, T)).astype(np.int32)
@@ -46,13 +48,9 @@ def test_noalloc_step_matches_decode_step_on_two_calls(name):
             torch.cuda.synchronize()
             out[key] = (to_np(lp), to_np(lse), to_np(full), to_np(st.s()))
         assert model.last_error() == 0
-        (lp_a, lse_a, full_a, s_a), (lp_b, lse_b, full_b, s_b) = out["ref"], out["noalloc"]
-        assert np.abs(full_a - full_b).max() <= tol
-        assert np.abs(lp_a - lp_b).max() <= tol and np.abs(lse_a - lse_b).max() <= tol
-        if cfg.dtype == "f32":
-            assert np.abs(s_a - s_b).max() <= 1e-4
-        else:
-            assert cosine(s_a, s_b).min() >= 0.999
+        for a, b in zip(out["ref"], out["noalloc"]):
+            np.testing.assert_array_equal(a, b)
+        np.testing.assert_array_equal(to_np(st_ref.buf[256:]), to_np(st_na.buf[256:]))   # s and ring
         assert st_na.position == st_ref.position == step + 1
 
 
@@ -65,3 +63,15 @@ def test_noalloc_step_rejects_batches_beyond_the_static_scratch():
     with pytest.raises(RLTError) as ex:
         model.decode_step_noalloc(big, e, M)
     assert ex.value.status == "RLT_EUNSUPPORTED"
+
+
+@pytest.mark.skipif(not torch.cuda.is_available() or torch.cuda.device_count() < 2, reason="needs two devices")
+def test_noalloc_step_rejects_a_current_device_other_than_the_models():
+    cfg = TINY.model
+    model = build_model(cfg, max_pos=8, weights=make_weights(cfg))
+    e, M = model.alloc_encoder_outputs(1, 8)
+    st = model.new_state(1)
+    with torch.cuda.device(1):
+        with pytest.raises(RLTError) as ex:
+            model.decode_step_noalloc(st, e, M)
+    assert ex.value.status == "RLT_EINVAL"
