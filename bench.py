@@ -288,6 +288,8 @@ def main() -> int:
     ap.add_argument("--workload", default=RLT_300M.name, choices=sorted(WORKLOADS))
     ap.add_argument("--T", type=int, default=None, help="override the sweep length (profiling runs only)")
     ap.add_argument("--B", type=int, default=None, help="override the batch (profiling runs only)")
+    ap.add_argument("--option", action="append", default=[], metavar="NAME=VALUE",
+                    help="scheduling option of the model handle (rlt_set_option), repeatable")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-replay", action="store_true")
@@ -322,6 +324,9 @@ def main() -> int:
     m, B, T = wl.model, wl.B, wl.T
 
     model = RLTModel(m, max_pos=T)
+    for opt in args.option:
+        name, value = opt.split("=", 1)
+        model.set_option(name, int(value))
     w = make_weights(m, wl.weight_seed)
     model.load_weights(w)
     del w
@@ -485,7 +490,7 @@ def main() -> int:
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": m.dtype, "data": "synthetic",
-            "config": arm_config(wl, B, T, world),
+            "config": {**arm_config(wl, B, T, world), **({"options": args.option} if args.option else {})},
             "roofline": roofline, "step_roofline": step_roofline, "cpu_baseline": cpu, "e2e": e2e,
             "replay": replay, "encode": enc, "gpu_launches": launches, "clocks": clocks,
             "kernel_breakdown_ms_per_sweep": {k: round(v[0], 3) for k, v in sorted(breakdown.items())},

@@ -144,97 +144,102 @@ __global__ void __launch_bounds__(SWA_WARPS * 32, 6) k_swa_decode(const float* _
     __shared__ __align__(16) uint4 sm_kv[2][LPK];      // current k_t, v_t in storage type
     pdl_wait();
     pdl_trigger();
-    const int item = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane / LPK, li = lane % LPK;
-    const int b = item / H, h = item % H;
     const int d = H * HD, half = HD / 2;
-    const float* row = qkv + (long long)b * 3 * d + h * HD;
-    // this warp's share of the ring; its first round of loads is issued before q is formed, so
-    // the ring's memory latency overlaps the q / RoPE loads instead of following them
-    T* Kr = nullptr;
-    T* Vr = nullptr;
-    int j0 = 0, nj = 0;
-    if (W > 1) {
-        Kr = ring + (((long long)b * 2 + 0) * H + h) * (long long)(W - 1) * HD;
-        Vr = ring + (((long long)b * 2 + 1) * H + h) * (long long)(W - 1) * HD;
-        int n = min(t - 1, W - 1);
-        int per = (n + SWA_WARPS - 1) / SWA_WARPS;
-        j0 = min(n, warp * per);
-        nj = min(n, j0 + per) - j0;
-    }
-    constexpr int SWA_U = 4;
-    uint4 kr0[SWA_U], vr0[SWA_U];
-    load_round<T, HD, SWA_U, true>(Kr + (long long)j0 * HD, Vr + (long long)j0 * HD, nj, 0, g, li, kr0, vr0);
-    float q[EPL];
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-        int c = li * EPL + i;
-        int cp = c < half ? c + half : c - half;
-        float2 cs = rope_row[c % half];
-        float qa = row[c], qp = row[cp];
-        q[i] = (c < half ? qa * cs.x - qp * cs.y : qp * cs.y + qa * cs.x) * qscale;
-    }
-    float m = NEG_BIG, l = 0.f, acc[EPL];
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) acc[i] = 0.f;
-    if (warp == 0) {
-        // the current token: k_t (rotated) and v_t rounded to the storage type, as cached
-        float k[EPL], v[EPL];
+    // one (sequence, head) item per iteration; the grid is at most one item per CTA and may be
+    // capped below that (then each CTA takes items blockIdx.x, blockIdx.x + gridDim.x, ...)
+    for (int item = blockIdx.x; item < B * H; item += gridDim.x) {
+        const int b = item / H, h = item % H;
+        const float* row = qkv + (long long)b * 3 * d + h * HD;
+        // this warp's share of the ring; its first round of loads is issued before q is formed,
+        // so the ring's memory latency overlaps the q / RoPE loads instead of following them
+        T* Kr = nullptr;
+        T* Vr = nullptr;
+        int j0 = 0, nj = 0;
+        if (W > 1) {
+            Kr = ring + (((long long)b * 2 + 0) * H + h) * (long long)(W - 1) * HD;
+            Vr = ring + (((long long)b * 2 + 1) * H + h) * (long long)(W - 1) * HD;
+            int n = min(t - 1, W - 1);
+            int per = (n + SWA_WARPS - 1) / SWA_WARPS;
+            j0 = min(n, warp * per);
+            nj = min(n, j0 + per) - j0;
+        }
+        constexpr int SWA_U = 4;
+        uint4 kr0[SWA_U], vr0[SWA_U];
+        load_round<T, HD, SWA_U, true>(Kr + (long long)j0 * HD, Vr + (long long)j0 * HD, nj, 0, g, li, kr0, vr0);
+        float q[EPL];
 #pragma unroll
         for (int i = 0; i < EPL; ++i) {
             int c = li * EPL + i;
             int cp = c < half ? c + half : c - half;
             float2 cs = rope_row[c % half];
-            float ka = row[d + c], kp = row[d + cp];
-            k[i] = round_to<T>(c < half ? ka * cs.x - kp * cs.y : kp * cs.y + ka * cs.x);
-            v[i] = round_to<T>(row[2 * d + c]);
+            float qa = row[c], qp = row[cp];
+            q[i] = (c < half ? qa * cs.x - qp * cs.y : qp * cs.y + qa * cs.x) * qscale;
         }
-        float sc = 0.f;
+        float m = NEG_BIG, l = 0.f, acc[EPL];
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) sc = fmaf(q[i], k[i], sc);
-        sc = group_sum<LPK>(sc);
+        for (int i = 0; i < EPL; ++i) acc[i] = 0.f;
+        if (warp == 0) {
+            // the current token: k_t (rotated) and v_t rounded to the storage type, as cached
+            float k[EPL], v[EPL];
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) {
+                int c = li * EPL + i;
+                int cp = c < half ? c + half : c - half;
+                float2 cs = rope_row[c % half];
+                float ka = row[d + c], kp = row[d + cp];
+                k[i] = round_to<T>(c < half ? ka * cs.x - kp * cs.y : kp * cs.y + ka * cs.x);
+                v[i] = round_to<T>(row[2 * d + c]);
+            }
+            float sc = 0.f;
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) sc = fmaf(q[i], k[i], sc);
+            sc = group_sum<LPK>(sc);
+            if (g == 0) {
+                m = sc; l = 1.f;
+#pragma unroll
+                for (int i = 0; i < EPL; ++i) acc[i] = v[i];
+                sm_kv[0][li] = Vec16<T>::pack(k);
+                sm_kv[1][li] = Vec16<T>::pack(v);
+            }
+        }
+        if (nj > 0) {
+            consume_round<T, HD, SWA_U>(q, nj, 0, g, kr0, vr0, m, l, acc);
+            attend<T, HD, SWA_U, true>(q, Kr + (long long)j0 * HD, Vr + (long long)j0 * HD, nj, g, li, m, l, acc,
+                                       Geom<T, HD>::KPI * SWA_U);
+        }
+        merge_groups<T, HD>(m, l, acc);
         if (g == 0) {
-            m = sc; l = 1.f;
 #pragma unroll
-            for (int i = 0; i < EPL; ++i) acc[i] = v[i];
-            sm_kv[0][li] = Vec16<T>::pack(k);
-            sm_kv[1][li] = Vec16<T>::pack(v);
+            for (int i = 0; i < EPL; ++i) sm_acc[warp][li * EPL + i] = acc[i];
+            if (li == 0) { sm_m[warp] = m; sm_l[warp] = l; }
         }
-    }
-    if (nj > 0) {
-        consume_round<T, HD, SWA_U>(q, nj, 0, g, kr0, vr0, m, l, acc);
-        attend<T, HD, SWA_U, true>(q, Kr + (long long)j0 * HD, Vr + (long long)j0 * HD, nj, g, li, m, l, acc,
-                                   Geom<T, HD>::KPI * SWA_U);
-    }
-    merge_groups<T, HD>(m, l, acc);
-    if (g == 0) {
+        __syncthreads();                      // every warp has read its share of the ring
+        if (warp == 0 && g == 0) {
+            float mx = NEG_BIG;
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) sm_acc[warp][li * EPL + i] = acc[i];
-        if (li == 0) { sm_m[warp] = m; sm_l[warp] = l; }
-    }
-    __syncthreads();
-    if (warp != 0 || g != 0) return;
-    float mx = NEG_BIG;
+            for (int w = 0; w < SWA_WARPS; ++w) mx = fmaxf(mx, sm_m[w]);
+            float L = 0.f, out[EPL];
 #pragma unroll
-    for (int w = 0; w < SWA_WARPS; ++w) mx = fmaxf(mx, sm_m[w]);
-    float L = 0.f, out[EPL];
+            for (int i = 0; i < EPL; ++i) out[i] = 0.f;
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) out[i] = 0.f;
+            for (int w = 0; w < SWA_WARPS; ++w) {
+                float c = exp2f(sm_m[w] - mx);
+                L += sm_l[w] * c;
 #pragma unroll
-    for (int w = 0; w < SWA_WARPS; ++w) {
-        float c = exp2f(sm_m[w] - mx);
-        L += sm_l[w] * c;
+                for (int i = 0; i < EPL; ++i) out[i] += sm_acc[w][li * EPL + i] * c;
+            }
+            float inv = 1.0f / L;
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) out[i] += sm_acc[w][li * EPL + i] * c;
-    }
-    float inv = 1.0f / L;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) out[i] *= inv;
-    st16(o + (long long)b * d + h * HD + li * EPL, Vec16<T>::pack(out));
-    if (W > 1) {
-        int slot = (t - 1) % (W - 1);
-        st16(Kr + (long long)slot * HD + li * EPL, sm_kv[0][li]);
-        st16(Vr + (long long)slot * HD + li * EPL, sm_kv[1][li]);
+            for (int i = 0; i < EPL; ++i) out[i] *= inv;
+            st16(o + (long long)b * d + h * HD + li * EPL, Vec16<T>::pack(out));
+            if (W > 1) {
+                int slot = (t - 1) % (W - 1);
+                st16(Kr + (long long)slot * HD + li * EPL, sm_kv[0][li]);
+                st16(Vr + (long long)slot * HD + li * EPL, sm_kv[1][li]);
+            }
+        }
+        __syncthreads();                      // shared partials are free for the next item
     }
 }
 
@@ -248,36 +253,39 @@ __global__ void __launch_bounds__(WARPS * 32) k_xattn_decode(const float* __rest
     constexpr int EPL = G::EPL, LPK = G::LPK;
     pdl_wait();
     pdl_trigger();
-    int item = blockIdx.x * WARPS + (threadIdx.x >> 5);
-    if (item >= B * H * n_splits) return;
-    int lane = threadIdx.x & 31, g = lane / LPK, li = lane % LPK;
-    int bh = item / n_splits, sp = item % n_splits;
-    int b = bh / H, h = bh % H;
-    const int d = H * HD;
-    float q[EPL];
-    const float* qr = qc + (long long)b * d + h * HD + li * EPL;
+    const int lane = threadIdx.x & 31, g = lane / LPK, li = lane % LPK;
+    const int n_items = B * H * n_splits;
+    // one (sequence, head, key chunk) item per warp and iteration; a capped grid strides over
+    // the items
+    for (int item = blockIdx.x * WARPS + (threadIdx.x >> 5); item < n_items; item += gridDim.x * WARPS) {
+        int bh = item / n_splits, sp = item % n_splits;
+        int b = bh / H, h = bh % H;
+        const int d = H * HD;
+        float q[EPL];
+        const float* qr = qc + (long long)b * d + h * HD + li * EPL;
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) q[i] = qr[i] * qscale;
-    const T* K = Mg + (long long)bh * T_alloc * HD;
-    const T* V = K + plane;
-    int j0 = sp * chunk;
-    int n = max(0, min(t, j0 + chunk) - j0);
-    float m = NEG_BIG, l = 0.f, acc[EPL];
+        for (int i = 0; i < EPL; ++i) q[i] = qr[i] * qscale;
+        const T* K = Mg + (long long)bh * T_alloc * HD;
+        const T* V = K + plane;
+        int j0 = sp * chunk;
+        int n = max(0, min(t, j0 + chunk) - j0);
+        float m = NEG_BIG, l = 0.f, acc[EPL];
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) acc[i] = 0.f;
-    attend<T, HD, 4, true>(q, K + (long long)j0 * HD, V + (long long)j0 * HD, n, g, li, m, l, acc);
-    merge_groups<T, HD>(m, l, acc);
-    if (g != 0) return;
-    if (n_splits == 1) {
-        float inv = 1.0f / l, out[EPL];
+        for (int i = 0; i < EPL; ++i) acc[i] = 0.f;
+        attend<T, HD, 4, true>(q, K + (long long)j0 * HD, V + (long long)j0 * HD, n, g, li, m, l, acc);
+        merge_groups<T, HD>(m, l, acc);
+        if (g != 0) continue;
+        if (n_splits == 1) {
+            float inv = 1.0f / l, out[EPL];
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) out[i] = acc[i] * inv;
-        st16(o + (long long)b * d + h * HD + li * EPL, Vec16<T>::pack(out));
-    } else {
-        float* pp = part + (long long)item * (HD + 2);
+            for (int i = 0; i < EPL; ++i) out[i] = acc[i] * inv;
+            st16(o + (long long)b * d + h * HD + li * EPL, Vec16<T>::pack(out));
+        } else {
+            float* pp = part + (long long)item * (HD + 2);
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) pp[li * EPL + i] = acc[i];
-        if (li == 0) { pp[HD] = m; pp[HD + 1] = l; }
+            for (int i = 0; i < EPL; ++i) pp[li * EPL + i] = acc[i];
+            if (li == 0) { pp[HD] = m; pp[HD + 1] = l; }
+        }
     }
 }
 
@@ -337,6 +345,12 @@ __global__ void __launch_bounds__(WARPS * 32, 8) k_enc_attn(const T* __restrict_
 
 inline float qscale_for(int hd) { return LOG2E / sqrtf((float)hd); }
 inline unsigned blocks_for(long long items) { return (unsigned)((items + WARPS - 1) / WARPS); }
+// A grid of `blocks` CTAs, capped at L.attn_ctas_per_sm resident CTAs on every SM when set.
+inline unsigned capped(const Launch& L, unsigned blocks) {
+    if (L.attn_ctas_per_sm <= 0) return blocks;
+    const long long cap = (long long)sm_count() * L.attn_ctas_per_sm;
+    return blocks > cap ? (unsigned)cap : blocks;
+}
 
 }  // namespace
 
@@ -352,14 +366,14 @@ inline unsigned blocks_for(long long items) { return (unsigned)((items + WARPS -
 template <typename T>
 cudaError_t launch_swa_decode(Launch L, const float* qkv, const float2* rope_row, T* ring, T* o, int B,
                               int H, int hd, int W, int t) {
-    RLT_HD_DISPATCH(hd, launch_k(L, k_swa_decode<T, HD>, (unsigned)(B * H), SWA_WARPS * 32, 0, qkv, rope_row,
+    RLT_HD_DISPATCH(hd, launch_k(L, k_swa_decode<T, HD>, capped(L, (unsigned)(B * H)), SWA_WARPS * 32, 0, qkv, rope_row,
                                  ring, o, B, H, W, t, qscale_for(hd)));
 }
 
 template <typename T>
 static cudaError_t xattn_main(Launch L, const float* qc, const T* Mg, long long plane, int T_alloc, int t, T* o,
                               int B, int H, int hd, int n_splits, int chunk, float* part) {
-    RLT_HD_DISPATCH(hd, launch_k(L, k_xattn_decode<T, HD>, blocks_for((long long)B * H * n_splits), WARPS * 32, 0,
+    RLT_HD_DISPATCH(hd, launch_k(L, k_xattn_decode<T, HD>, capped(L, blocks_for((long long)B * H * n_splits)), WARPS * 32, 0,
                                  qc, Mg, plane, T_alloc, t, o, B, H, n_splits, chunk, part, qscale_for(hd)));
 }
 

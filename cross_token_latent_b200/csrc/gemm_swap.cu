@@ -314,7 +314,7 @@ cudaError_t run_swap(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, i
     cudaLaunchAttribute attr[2];
     int na = 0;
     attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    attr[na].val.programmaticStreamSerializationAllowed = L.pdl ? 1 : 0;
     ++na;
     if (SPLIT > 1) {
         attr[na].id = cudaLaunchAttributeClusterDimension;

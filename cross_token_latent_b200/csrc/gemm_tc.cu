@@ -495,7 +495,7 @@ cudaError_t run_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = SPLIT;
         attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        attr[1].val.programmaticStreamSerializationAllowed = L.pdl ? 1 : 0;
         cfg.attrs = attr;
         cfg.numAttrs = 2;
         *L.count += 1;

@@ -11,10 +11,31 @@ namespace rlt {
 struct Launch {
     cudaStream_t stream;
     uint64_t* count;
+    // Programmatic dependent launch (see pdl_wait in common.cuh).  Off when two row groups of
+    // a step run on two streams: a kernel launched early would hold its SM resources while it
+    // waits, which the other group's kernels need.
+    bool pdl = true;
+    // Cap on the resident CTAs per SM of the attention kernels (0: none).  With two row groups
+    // the attention of one group leaves room on every SM for the other group's projections.
+    int attn_ctas_per_sm = 0;
 };
 
-// Launch `kernel` on L.stream with programmatic stream serialization (see pdl_wait in
-// common.cuh) and count it.
+// Number of SMs of the current device (queried once per process).
+inline int sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+            n = v;
+        else
+            return 148;
+    }
+    return n;
+}
+
+// Launch `kernel` on L.stream (with programmatic stream serialization unless L.pdl is off)
+// and count it.
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_k(Launch L, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                             Args&&... args) {
@@ -25,7 +46,7 @@ inline cudaError_t launch_k(Launch L, void (*kernel)(KArgs...), dim3 grid, dim3 
     cfg.stream = L.stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[0].val.programmaticStreamSerializationAllowed = L.pdl ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     *L.count += 1;

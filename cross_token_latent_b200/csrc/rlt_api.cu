@@ -20,6 +20,10 @@ constexpr size_t ALIGN = 256;
 inline size_t align_up(size_t x) { return (x + ALIGN - 1) / ALIGN * ALIGN; }
 inline bool aligned(const void* p, size_t a = ALIGN) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Batches of at least this many sequences may run a step as two row groups on two streams
+// (each group then still fills whole 128-row GEMM tiles).
+constexpr int GROUP_MIN_ROWS = 256;
+
 // Cross-attention key-split partials: capacity in (sequence, head, split) work items.
 constexpr long long XATTN_PART_ITEMS = 32768;
 constexpr int XATTN_MAX_SPLITS = 64;
@@ -148,6 +152,33 @@ struct rlt_model {
     std::unordered_map<const void*, StateInfo> states;
     uint64_t launches = 0;
     int device = -1;            // the CUDA device that holds the arena
+    // rlt_set_option values
+    int opt_row_groups = 0;             // 0 auto, 1 one group, 2 two groups (B >= GROUP_MIN_ROWS)
+    int opt_group_attn_cap = 6;         // attention CTAs per SM while two groups run
+    int opt_group_pdl = 0;              // programmatic dependent launch inside a group's chain
+    // two row groups: library-owned streams, forked from and joined back to the caller's stream
+    cudaStream_t gs[2] = {nullptr, nullptr};
+    cudaEvent_t fork_ev = nullptr, join_ev[2] = {nullptr, nullptr};
+
+    ~rlt_model() {
+        for (int i = 0; i < 2; ++i) {
+            if (gs[i]) cudaStreamDestroy(gs[i]);
+            if (join_ev[i]) cudaEventDestroy(join_ev[i]);
+        }
+        if (fork_ev) cudaEventDestroy(fork_ev);
+    }
+    bool group_streams() {
+        if (gs[0]) return true;
+        for (int i = 0; i < 2; ++i) {
+            if (cudaStreamCreateWithFlags(&gs[i], cudaStreamNonBlocking) != cudaSuccess) return false;
+            if (cudaEventCreateWithFlags(&join_ev[i], cudaEventDisableTiming) != cudaSuccess) return false;
+        }
+        return cudaEventCreateWithFlags(&fork_ev, cudaEventDisableTiming) == cudaSuccess;
+    }
+    int row_groups(int B) const {
+        if (opt_row_groups == 1 || B < GROUP_MIN_ROWS || cfg.dtype != RLT_BF16) return 1;
+        return 2;
+    }
 
     DevHeader* hdr() const { return reinterpret_cast<DevHeader*>(arena); }
     template <typename T> T* at(size_t off) const { return reinterpret_cast<T*>(arena + off); }
@@ -242,7 +273,7 @@ EncWS enc_ws(const rlt_config& c, int B, int T) {
 }
 
 struct DecWS {
-    size_t x, A, qkv, att, qc, act, logits, part, xn, ss, total;
+    size_t x, A, qkv, att, qc, act, logits, part, part2, xn, ss, total;
 };
 DecWS dec_ws(const rlt_config& c, int B) {
     DecWS w;
@@ -257,6 +288,8 @@ DecWS dec_ws(const rlt_config& c, int B) {
     w.act = take((size_t)B * c.F * e);
     w.logits = take((size_t)B * c.V * 4);
     w.part = take((size_t)XATTN_PART_ITEMS * (c.head_dim + 2) * 4);
+    // the second row group's key-split partials
+    w.part2 = B >= GROUP_MIN_ROWS ? take((size_t)XATTN_PART_ITEMS * (c.head_dim + 2) * 4) : w.part;
     w.xn = take((size_t)B * d * e);               // bf16(x * g) of a deferred norm
     w.ss = take((size_t)B * (d / 16) * 4);        // its 16-column sum-of-squares partials
     w.total = off;
@@ -343,34 +376,39 @@ struct StepIO {
     bool head = true;
 };
 
+// Rows [b0, b0 + Bg) of a step over a batch of B sequences: every row-indexed buffer is offset
+// by b0; `part` is this row group's key-split buffer; `first` says whether this group checks
+// and advances the state header.
 template <typename T>
-rlt_status step_impl(rlt_model* m, uint8_t* state, int B, const T* e, const T* M, int T_alloc, int t,
-                     const StepIO& io, uint8_t* ws, cudaStream_t st) {
+rlt_status step_rows(rlt_model* m, uint8_t* state, int B, int b0, int Bg, const T* e, const T* M, int T_alloc,
+                     int t, const StepIO& io, uint8_t* ws, float* part, bool first, Launch L) {
     const rlt_config& c = m->cfg;
-    Launch L{st, &m->launches};
     DecWS w = dec_ws(c, B);
     int d = c.d, F = c.F, H = c.n_heads, hd = c.head_dim;
-    StateHeader* sh = reinterpret_cast<StateHeader*>(state);
-    float* s = reinterpret_cast<float*>(state + state_s_off());
-    T* ring = reinterpret_cast<T*>(state + state_ring_off(c, B));
-    float* x = reinterpret_cast<float*>(ws + w.x);
-    T* A = reinterpret_cast<T*>(ws + w.A);
-    float* qkv = reinterpret_cast<float*>(ws + w.qkv);
-    T* att = reinterpret_cast<T*>(ws + w.att);
-    float* qc = reinterpret_cast<float*>(ws + w.qc);
-    T* act = reinterpret_cast<T*>(ws + w.act);
-    float* logits = reinterpret_cast<float*>(ws + w.logits);
-    float* part = reinterpret_cast<float*>(ws + w.part);
+    const size_t rb = (size_t)b0;
+    StateHeader* sh = first ? reinterpret_cast<StateHeader*>(state) : nullptr;
+    float* s = reinterpret_cast<float*>(state + state_s_off()) + rb * d;
+    T* ring = reinterpret_cast<T*>(state + state_ring_off(c, B)) + rb * 2 * H * (size_t)(c.W - 1) * hd;
+    float* x = reinterpret_cast<float*>(ws + w.x) + rb * d;
+    T* A = reinterpret_cast<T*>(ws + w.A) + rb * 2 * d;
+    float* qkv = reinterpret_cast<float*>(ws + w.qkv) + rb * 3 * d;
+    T* att = reinterpret_cast<T*>(ws + w.att) + rb * d;
+    float* qc = reinterpret_cast<float*>(ws + w.qc) + rb * d;
+    T* act = reinterpret_cast<T*>(ws + w.act) + rb * F;
+    float* logits = reinterpret_cast<float*>(ws + w.logits) + rb * c.V;
     const float2* rope_row = m->at<float2>(m->lay.rope) + (size_t)(t - 1) * (hd / 2);
-    size_t group_elems = (size_t)2 * B * H * (size_t)T_alloc * hd;
-    int splits = xattn_splits(c, B, t);
+    const size_t group_elems = (size_t)2 * B * H * (size_t)T_alloc * hd;
+    const long long plane = (long long)B * H * T_alloc * hd;        // keys -> values of one memory group
+    const T* eg = e + rb * T_alloc * d;
+    const T* Mrows = M + rb * H * (size_t)T_alloc * hd;
+    int splits = xattn_splits(c, Bg, t);
 
     // Deferred RMSNorm (bf16 tensor-core path): the GEMM that updates the residual stream x
     // also writes bf16(x * g) and per-row sum-of-squares partials, and the GEMM that consumes
     // the norm scales its accumulator rows by 1 / rms (row scaling commutes with the product),
     // so the three sublayer norms of a layer need no launches of their own.
-    T* xn = reinterpret_cast<T*>(ws + w.xn);
-    float* ss = reinterpret_cast<float*>(ws + w.ss);
+    T* xn = reinterpret_cast<T*>(ws + w.xn) + rb * d;
+    float* ss = reinterpret_cast<float*>(ws + w.ss) + rb * (d / 16);
     const bool fuse = std::is_same<T, bf16>::value && d % 64 == 0 &&
                       gemm_tc_supported(xn, d, m->at<T>(m->lay.wqkv[0]), d) &&
                       gemm_tc_supported(A, 2 * d, m->at<T>(m->lay.merge_w), 2 * d) &&
@@ -386,17 +424,17 @@ rlt_status step_impl(rlt_model* m, uint8_t* state, int B, const T* e, const T* M
     };
     // the sublayer input: bf16(x * g) under a deferred norm, else RMSNorm(x) * g from its own kernel
     auto pre_norm = [&](const float* g) -> cudaError_t {
-        return launch_rmsnorm<T>(L, x, B, d, g, c.rms_eps, A, d, B, B, nullptr);
+        return launch_rmsnorm<T>(L, x, Bg, d, g, c.rms_eps, A, d, Bg, Bg, nullptr);
     };
     const T* hin = fuse ? xn : A;
 
     // gated merge: x = e_t + sigmoid(W_ge e_t + W_gs s + b_g) * (W_fb s)
-    CKP(RLT_K_MERGE, launch_merge_prep<T>(L, e, T_alloc, t, s, A, B, d, sh, m->version, m->hdr()));
+    CKP(RLT_K_MERGE, launch_merge_prep<T>(L, eg, T_alloc, t, s, A, Bg, d, sh, m->version, m->hdr()));
     {
         EpiArgs ea; ea.hdr = m->hdr();
         ea.out_f32 = x; ea.ld_out = d; ea.merge_e = A; ea.ld_e = 2 * d; ea.bias = m->at<float>(m->lay.merge_b);
         norm_out(ea, m->at<float>(m->lay.attn_norm[0]));
-        CKP(RLT_K_MERGE, launch_gemm<T>(L, Epi::Merge, A, 2 * d, m->at<T>(m->lay.merge_w), B, 2 * d, 2 * d, ea));
+        CKP(RLT_K_MERGE, launch_gemm<T>(L, Epi::Merge, A, 2 * d, m->at<T>(m->lay.merge_w), Bg, 2 * d, 2 * d, ea));
     }
     for (int l = 0; l < c.L_D; ++l) {
         EpiArgs ea; ea.hdr = m->hdr();
@@ -404,42 +442,79 @@ rlt_status step_impl(rlt_model* m, uint8_t* state, int B, const T* e, const T* M
         if (!fuse) CKP(RLT_K_NORM, pre_norm(m->at<float>(m->lay.attn_norm[l])));
         ea.out_f32 = qkv; ea.ld_out = 3 * d;
         norm_in(ea);
-        CKP(RLT_K_QKV, launch_gemm<T>(L, Epi::StoreF32, hin, d, m->at<T>(m->lay.wqkv[l]), B, 3 * d, d, ea));
-        CKP(RLT_K_SWA, launch_swa_decode<T>(L, qkv, rope_row, ring + (size_t)l * ring_layer_elems(c, B), att, B, H, hd,
-                                c.W, t));
+        CKP(RLT_K_QKV, launch_gemm<T>(L, Epi::StoreF32, hin, d, m->at<T>(m->lay.wqkv[l]), Bg, 3 * d, d, ea));
+        CKP(RLT_K_SWA, launch_swa_decode<T>(L, qkv, rope_row, ring + (size_t)l * ring_layer_elems(c, B), att, Bg, H,
+                                            hd, c.W, t));
         ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = x; ea.ld_out = d;
         norm_out(ea, m->at<float>(m->lay.xattn_norm[l]));
-        CKP(RLT_K_O, launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.wo[l]), B, d, d, ea));
+        CKP(RLT_K_O, launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.wo[l]), Bg, d, d, ea));
         // cross-attention to M_{<=t}
         if (!fuse) CKP(RLT_K_NORM, pre_norm(m->at<float>(m->lay.xattn_norm[l])));
         ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = qc; ea.ld_out = d;
         norm_in(ea);
-        CKP(RLT_K_QC, launch_gemm<T>(L, Epi::StoreF32, hin, d, m->at<T>(m->lay.wqc[l]), B, d, d, ea));
-        const T* Mg = M + (c.G == 1 ? 0 : (size_t)l * group_elems);
-        CKP(RLT_K_XATTN, launch_xattn_decode<T>(L, qc, Mg, (long long)B * H * T_alloc * hd, T_alloc, t, att, B, H, hd,
-                                                splits, part));
+        CKP(RLT_K_QC, launch_gemm<T>(L, Epi::StoreF32, hin, d, m->at<T>(m->lay.wqc[l]), Bg, d, d, ea));
+        const T* Mg = Mrows + (c.G == 1 ? 0 : (size_t)l * group_elems);
+        CKP(RLT_K_XATTN, launch_xattn_decode<T>(L, qc, Mg, plane, T_alloc, t, att, Bg, H, hd, splits, part));
         ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = x; ea.ld_out = d;
         norm_out(ea, m->at<float>(m->lay.ffn_norm[l]));
-        CKP(RLT_K_OC, launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.woc[l]), B, d, d, ea));
+        CKP(RLT_K_OC, launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.woc[l]), Bg, d, d, ea));
         // SwiGLU FFN (weights of encoder layer l)
         if (!fuse) CKP(RLT_K_NORM, pre_norm(m->at<float>(m->lay.ffn_norm[l])));
         ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_t = act; ea.ld_out = F;
         norm_in(ea);
-        CKP(RLT_K_FFN_UP, launch_gemm<T>(L, Epi::SwiGLU, hin, d, m->at<T>(m->lay.wgu[l]), B, 2 * F, d, ea));
+        CKP(RLT_K_FFN_UP, launch_gemm<T>(L, Epi::SwiGLU, hin, d, m->at<T>(m->lay.wgu[l]), Bg, 2 * F, d, ea));
         ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = x; ea.ld_out = d;
         if (l + 1 < c.L_D) norm_out(ea, m->at<float>(m->lay.attn_norm[l + 1]));
-        CKP(RLT_K_FFN_DOWN, launch_gemm<T>(L, Epi::ResidAdd, act, F, m->at<T>(m->lay.wdown[l]), B, d, F, ea));
+        CKP(RLT_K_FFN_DOWN, launch_gemm<T>(L, Epi::ResidAdd, act, F, m->at<T>(m->lay.wdown[l]), Bg, d, F, ea));
     }
     // split: s_t = RMSNorm(x) becomes the state; the same s_t feeds the head
-    CKP(RLT_K_FINAL, launch_final_norm<T>(L, x, B, d, m->at<float>(m->lay.dec_norm), c.rms_eps, s, A, sh, t));
+    CKP(RLT_K_FINAL, launch_final_norm<T>(L, x, Bg, d, m->at<float>(m->lay.dec_norm), c.rms_eps, s, A, sh, t));
     if (io.head) {
         EpiArgs ea; ea.hdr = m->hdr();
         ea.out_f32 = logits; ea.ld_out = c.V;
-        CKP(RLT_K_HEAD, launch_gemm<T>(L, Epi::StoreF32, A, d, m->at<T>(m->lay.unembed), B, c.V, d, ea));
-        CKP(RLT_K_LSE, launch_lse_gather(L, logits, B, c.V, io.tau, io.tok, io.tok_stride, io.logp_tok, io.lp_stride,
-                             io.lse, io.logp_full, io.score, io.prompt_len, t, m->hdr()));
+        CKP(RLT_K_HEAD, launch_gemm<T>(L, Epi::StoreF32, A, d, m->at<T>(m->lay.unembed), Bg, c.V, d, ea));
+        CKP(RLT_K_LSE, launch_lse_gather(L, logits, Bg, c.V, io.tau, io.tok ? io.tok + rb * io.tok_stride : nullptr,
+                                         io.tok_stride, io.logp_tok ? io.logp_tok + rb * io.lp_stride : nullptr,
+                                         io.lp_stride, io.lse ? io.lse + rb : nullptr,
+                                         io.logp_full ? io.logp_full + rb * c.V : nullptr,
+                                         io.score ? io.score + rb : nullptr,
+                                         io.prompt_len ? io.prompt_len + rb : nullptr, t, m->hdr()));
     }
     return RLT_OK;
+}
+
+// One decoder step of all B sequences.  Large batches run as two row groups, each on a
+// library stream forked from `st` (an event) and joined back into it: while one group's
+// attention streams HBM, the other group's projections run on the tensor cores.  The
+// attention grids of both groups are capped so that every SM keeps room for the other
+// group's GEMM CTAs.
+template <typename T>
+rlt_status step_impl(rlt_model* m, uint8_t* state, int B, const T* e, const T* M, int T_alloc, int t,
+                     const StepIO& io, uint8_t* ws, cudaStream_t st) {
+    DecWS w = dec_ws(m->cfg, B);
+    float* part = reinterpret_cast<float*>(ws + w.part);
+    if (m->row_groups(B) == 1 || !m->group_streams()) {
+        return step_rows<T>(m, state, B, 0, B, e, M, T_alloc, t, io, ws, part, true, Launch{st, &m->launches});
+    }
+    float* part2 = reinterpret_cast<float*>(ws + w.part2);
+    const int B0 = (B / 2 + 127) / 128 * 128;           // group 0: whole 128-row tiles
+    CK(cudaEventRecord(m->fork_ev, st));
+    rlt_status r = RLT_OK;
+    for (int g = 0; g < 2 && r == RLT_OK; ++g) {
+        CK(cudaStreamWaitEvent(m->gs[g], m->fork_ev, 0));
+        Launch L{m->gs[g], &m->launches};
+        L.pdl = m->opt_group_pdl != 0;
+        L.attn_ctas_per_sm = m->opt_group_attn_cap;
+        r = g == 0 ? step_rows<T>(m, state, B, 0, B0, e, M, T_alloc, t, io, ws, part, true, L)
+                   : step_rows<T>(m, state, B, B0, B - B0, e, M, T_alloc, t, io, ws, part2, false, L);
+    }
+    // join both groups back into the caller's stream (also after an error: nothing is left
+    // dangling on the library streams)
+    for (int g = 0; g < 2; ++g) {
+        CK(cudaEventRecord(m->join_ev[g], m->gs[g]));
+        CK(cudaStreamWaitEvent(st, m->join_ev[g], 0));
+    }
+    return r;
 }
 
 template <typename T>
@@ -771,6 +846,24 @@ rlt_status rlt_last_error(rlt_model* m, void* stream) {
 }
 
 uint64_t rlt_launch_count(const rlt_model* m) { return m ? m->launches : 0; }
+
+rlt_status rlt_set_option(rlt_model* m, const char* name, int64_t value) {
+    if (!m || !name) return RLT_EINVAL;
+    const std::string n(name);
+    if (n == "row_groups") {
+        if (value < 0 || value > 2) return RLT_EINVAL;
+        m->opt_row_groups = (int)value;
+    } else if (n == "group_attn_ctas_per_sm") {
+        if (value < 0 || value > 32) return RLT_EINVAL;
+        m->opt_group_attn_cap = (int)value;
+    } else if (n == "group_pdl") {
+        if (value < 0 || value > 1) return RLT_EINVAL;
+        m->opt_group_pdl = (int)value;
+    } else {
+        return RLT_EINVAL;
+    }
+    return RLT_OK;
+}
 
 int rlt_gemm_plan(int M, int N, int K) {
     if (M < 1 || N < 1 || K < 1) return -1;

@@ -74,6 +74,7 @@ _EXPORTS = {
     "rlt_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                                  ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                  ctypes.c_uint64, ctypes.c_void_p]),
+    "rlt_set_option": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_char_p, ctypes.c_int64]),
     "rlt_profile_start": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_uint32]),
     "rlt_profile_stop": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_double),
                                         ctypes.POINTER(ctypes.c_uint64)]),
@@ -200,6 +201,11 @@ class RLTModel:
         _check(lib().rlt_model_commit(self.handle), "rlt_model_commit")
         torch.cuda.current_stream().synchronize()
         self._keep = None
+
+    def set_option(self, name: str, value: int) -> None:
+        """Scheduling option of the handle (rlt_set_option): "row_groups", "group_attn_ctas_per_sm",
+        "group_pdl"."""
+        _check(lib().rlt_set_option(self.handle, name.encode(), int(value)), f"rlt_set_option({name})")
 
     @property
     def version(self) -> int:

@@ -231,6 +231,22 @@ rlt_status rlt_last_error(rlt_model* m, void* stream);
  * points).  Used by benchmarks to count launches inside a timed region. */
 uint64_t rlt_launch_count(const rlt_model* m);
 
+/* Scheduling options of a model handle (no counterpart on the pages; they change how a step is
+ * scheduled on the GPU, never what it computes beyond summation order):
+ *   "row_groups"              0 (default) automatic: a bf16 step of B >= 256 sequences runs as
+ *                             two row groups, each on a library-owned stream forked from and
+ *                             joined back into the caller's stream, so that one group's
+ *                             attention (HBM-bound) overlaps the other group's projections
+ *                             (tensor cores); 1 always one group; 2 same as 0.
+ *   "group_attn_ctas_per_sm"  with two groups, the cap on resident attention CTAs per SM
+ *                             (0 = none; default 6), which leaves every SM room for the other
+ *                             group's GEMM CTAs.
+ *   "group_pdl"               1: programmatic dependent launch inside each group's chain
+ *                             (default 0: an early-launched kernel would hold SM resources the
+ *                             other group needs).
+ * Errors: RLT_EINVAL (unknown name or value out of range). */
+rlt_status rlt_set_option(rlt_model* m, const char* name, int64_t value);
+
 /* ---------------------------------------------------------------- building block */
 
 /* C[M, N] = A[M, K] W[N, K]^T with bf16 operands (row-major, K contiguous) and float32
