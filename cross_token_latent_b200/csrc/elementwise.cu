@@ -175,6 +175,33 @@ __global__ void k_lse_gather(const float* __restrict__ logits, int B, int V, flo
     }
 }
 
+// One warp per row: merge the column-tile (max, sum of exp) partials of the fused head.
+__global__ void k_lse_combine(const float2* __restrict__ part, int n_tiles, const float* __restrict__ z_tok, int B,
+                              int V, const int32_t* __restrict__ tok, int tok_stride, float* logp_tok, int lp_stride,
+                              float* lse_out, float* score, const int32_t* prompt_len, int t, DevHeader* hdr) {
+    pdl_wait();
+    pdl_trigger();
+    const int b = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    if (b >= B) return;
+    const float2* p = part + (long long)b * n_tiles;
+    float mx = -INFINITY;
+    for (int j = lane; j < n_tiles; j += 32) mx = fmaxf(mx, p[j].x);
+    mx = warp_max(mx);
+    float sm = 0.f;
+    for (int j = lane; j < n_tiles; j += 32) sm += p[j].y * expf(p[j].x - mx);
+    sm = warp_sum(sm);
+    if (lane != 0) return;
+    const float lse = mx + logf(sm);
+    if (lse_out) lse_out[b] = lse;
+    if (tok) {
+        int id = tok[(long long)b * tok_stride];
+        if (id < 0 || id >= V) raise_flag(hdr, ERR_BAD_TOKEN);     // the head gathered id 0
+        const float lp = z_tok[b] - lse;
+        if (logp_tok) logp_tok[(long long)b * lp_stride] = lp;
+        if (score && t >= prompt_len[b]) score[b] += lp;
+    }
+}
+
 // thread per (n, h, i < hd/2): rotate the pair (i, i + hd/2) of q and k, round q, k, v.
 template <typename T>
 __global__ void k_enc_qkv_layout(const float* __restrict__ qkv, int B, int Tn, int H, int hd,
@@ -294,6 +321,13 @@ cudaError_t launch_lse_gather(Launch L, const float* logits, int B, int V, float
                               DevHeader* hdr) {
     return launch_k(L, k_lse_gather, B, 512, 0, logits, B, V, tau, tok, tok_stride, logp_tok, lp_stride, lse,
                     logp_full, score, prompt_len, t, hdr);
+}
+
+cudaError_t launch_lse_combine(Launch L, const float2* part, int n_tiles, const float* z_tok, int B, int V,
+                               const int32_t* tok, int tok_stride, float* logp_tok, int lp_stride, float* lse,
+                               float* score, const int32_t* prompt_len, int t, DevHeader* hdr) {
+    return launch_k(L, k_lse_combine, cdiv(B, 8), 256, 0, part, n_tiles, z_tok, B, V, tok, tok_stride, logp_tok,
+                    lp_stride, lse, score, prompt_len, t, hdr);
 }
 
 template <typename T>

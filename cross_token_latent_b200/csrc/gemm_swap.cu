@@ -107,6 +107,8 @@ __device__ __forceinline__ void epilogue16_t(Epi epi, const EpiArgs& ea, int n, 
             }
             break;
         }
+        case Epi::LsePart:      // not produced by this kernel
+            break;
     }
 }
 

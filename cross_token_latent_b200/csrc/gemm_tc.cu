@@ -130,6 +130,8 @@ __device__ __forceinline__ float epilogue16(Epi epi, const EpiArgs& ea, int m, i
             }
             break;
         }
+        case Epi::LsePart:      // handled by the kernel's own epilogue loop
+            break;
     }
     return ss;
 }
@@ -279,7 +281,42 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     tc_fence_after();
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     if constexpr (SPLIT == 1) {
-        if (ok) {
+        if (ok && epi == Epi::LsePart) {
+            // fused head: this row's (max, sum of exp) over the tile's columns of z = acc * scale,
+            // and the gathered z of its target token when the tile holds it; nothing is stored
+            // per logit
+            const int m = m0 + warp * 32 + lane;
+            int tk = -1;
+            if (m < M && ea.lse_tok) {
+                tk = ea.lse_tok[(long long)m * ea.tok_stride];
+                if (tk < 0 || tk >= N) tk = 0;
+            }
+            float mx = -INFINITY, sm = 0.f;
+#pragma unroll 1
+            for (int c = 0; c < BN; c += 16) {
+                float v[16];
+                tmem_ld16(lane_base + c, v);
+                const int n = n0 + c;
+                if (m < M && n < N) {
+                    const int cnt = min(16, N - n);
+                    float cm = -INFINITY;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        v[j] *= ea.scale;
+                        if (j < cnt) cm = fmaxf(cm, v[j]);
+                        if (n + j == tk) ea.z_tok[m] = v[j];
+                    }
+                    if (cm > mx) {
+                        sm *= expf(mx - cm);
+                        mx = cm;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (j < cnt) sm += expf(v[j] - mx);
+                }
+            }
+            if (m < M) ea.lse_part[(long long)m * ea.lse_ld + blockIdx.x] = make_float2(mx, sm);
+        } else if (ok) {
             const int m = m0 + warp * 32 + lane;
 #pragma unroll 1
             for (int c = 0; c < BN; c += 16) {
@@ -585,6 +622,15 @@ bool gemm_tc_supported(const void* A, int lda, const void* W, int K) {
     // TMA: 16-byte aligned base addresses and row pitches
     return (reinterpret_cast<uintptr_t>(A) % 16 == 0) && (reinterpret_cast<uintptr_t>(W) % 16 == 0) &&
            (lda % 8 == 0) && (K % 8 == 0) && encode_fn() != nullptr;
+}
+
+cudaError_t launch_gemm_tc_lse(Launch L, const bf16* A, int lda, const bf16* W, int M, int N, int K, EpiArgs ea,
+                               DevHeader* hdr, int* n_tiles) {
+    int v = pick_variant(M, N, K);
+    if (VARIANTS[v].split > 1) v = 4;                 // the fused head needs whole rows per CTA
+    ea.lse_ld = (N + VARIANTS[v].bn - 1) / VARIANTS[v].bn;
+    *n_tiles = ea.lse_ld;
+    return run_variant(v, L, Epi::LsePart, A, lda, W, M, N, K, ea, hdr);
 }
 
 cudaError_t launch_gemm_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,

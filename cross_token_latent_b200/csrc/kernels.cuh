@@ -84,6 +84,12 @@ cudaError_t launch_lse_gather(Launch L, const float* logits, int B, int V, float
                               const int32_t* tok, int tok_stride, float* logp_tok, int lp_stride,
                               float* lse, float* logp_full, float* score, const int32_t* prompt_len,
                               int t, DevHeader* hdr);
+// Per row b: LSE = log sum_j part.y exp(part.x - max) + max over the n_tiles column-tile
+// partials of the fused head; the gathered log-prob z_tok[b] - LSE, the LSE itself and the
+// score accumulation as in launch_lse_gather (bad token ids latch ERR_BAD_TOKEN).
+cudaError_t launch_lse_combine(Launch L, const float2* part, int n_tiles, const float* z_tok, int B, int V,
+                               const int32_t* tok, int tok_stride, float* logp_tok, int lp_stride, float* lse,
+                               float* score, const int32_t* prompt_len, int t, DevHeader* hdr);
 // Encoder q/k/v: qkv float32 [B*T, 3d] -> planes T [3][B][H][T][hd], RoPE on q and k; the v
 // plane is skipped when write_v is false (the tensor-core path writes V transposed instead).
 template <typename T>
@@ -99,7 +105,7 @@ cudaError_t launch_state_init(Launch L, const float* s_star, int B, int d, float
 
 // ------------------------------------------------------------------ gemm_simt.cu
 // C[M, N] = A[M, K] (leading dim lda) x W[N, K]^T, float32 accumulation, then an epilogue.
-enum class Epi { StoreF32, ResidAdd, SwiGLU, Merge };
+enum class Epi { StoreF32, ResidAdd, SwiGLU, Merge, LsePart };
 struct EpiArgs {
     float* out_f32 = nullptr;   // StoreF32 target / ResidAdd accumulator / Merge output x
     void* out_t = nullptr;      // SwiGLU output (storage type)
@@ -128,6 +134,16 @@ struct EpiArgs {
     const float* ss_in = nullptr;
     int ss_ld = 0, ss_n = 0;
     float norm_n = 1.f, eps = 0.f;
+    // LM head with a fused log-sum-exp (LsePart, row-tile tensor-core kernel without a K
+    // split): with z = acc * scale, the CTA of column tile j writes, for each of its rows m,
+    // lse_part[m * lse_ld + j] = (max of z over the tile's columns, sum of exp(z - max)); the
+    // tile holding column lse_tok[m * tok_stride] (an id outside [0, N) counts as 0) writes
+    // z_tok[m].  No logits are stored.
+    const int32_t* lse_tok = nullptr;
+    int tok_stride = 1;
+    float2* lse_part = nullptr;
+    int lse_ld = 0;
+    float* z_tok = nullptr;
 };
 // 1 / rms of row m from its 16-column group partials (summed in group order).
 __device__ __forceinline__ float deferred_rinv(const EpiArgs& ea, long long m) {
@@ -156,6 +172,12 @@ int gemm_tc_pick(int M, int N, int K);
 // variant < 0: pick the tile shape from (M, N); otherwise force tile variant `variant`.
 cudaError_t launch_gemm_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                            const EpiArgs& ea, DevHeader* hdr, int variant = -1);
+
+// The LM head with the fused log-sum-exp epilogue (Epi::LsePart, M > 64): picks an unsplit
+// row-tile variant, sets ea.lse_ld to its number of column tiles and launches it; *n_tiles
+// receives that number for launch_lse_combine.
+cudaError_t launch_gemm_tc_lse(Launch L, const bf16* A, int lda, const bf16* W, int M, int N, int K, EpiArgs ea,
+                               DevHeader* hdr, int* n_tiles);
 
 // ------------------------------------------------------------------ gemm_swap.cu
 // Few-row products (1 <= M <= 64) with the weights on the MMA's M side; split = K split over a

@@ -469,16 +469,32 @@ rlt_status step_rows(rlt_model* m, uint8_t* state, int B, int b0, int Bg, const 
     }
     // split: s_t = RMSNorm(x) becomes the state; the same s_t feeds the head
     CKP(RLT_K_FINAL, launch_final_norm<T>(L, x, Bg, d, m->at<float>(m->lay.dec_norm), c.rms_eps, s, A, sh, t));
-    if (io.head) {
+    const int32_t* tok = io.tok ? io.tok + rb * io.tok_stride : nullptr;
+    float* lp_tok = io.logp_tok ? io.logp_tok + rb * io.lp_stride : nullptr;
+    float* lse = io.lse ? io.lse + rb : nullptr;
+    float* score = io.score ? io.score + rb : nullptr;
+    const int32_t* plen = io.prompt_len ? io.prompt_len + rb : nullptr;
+    if (io.head && fuse && Bg > 64 && !io.logp_full) {
+        // the head GEMM's epilogue reduces each row tile of logits to (max, sum of exp) partials
+        // and the gathered target logit; a small kernel merges them into LSE and log-probs
+        EpiArgs ea; ea.hdr = m->hdr();
+        ea.scale = 1.0f / io.tau;
+        ea.lse_tok = tok; ea.tok_stride = io.tok_stride;
+        ea.lse_part = reinterpret_cast<float2*>(logits);
+        ea.z_tok = logits + (size_t)Bg * c.V - Bg;      // the last Bg floats of this group's rows
+        int n_tiles = 0;
+        CKP(RLT_K_HEAD, launch_gemm_tc_lse(L, reinterpret_cast<const bf16*>(A), d,
+                                           reinterpret_cast<const bf16*>(m->at<T>(m->lay.unembed)), Bg, c.V, d, ea,
+                                           m->hdr(), &n_tiles));
+        CKP(RLT_K_LSE, launch_lse_combine(L, ea.lse_part, n_tiles, ea.z_tok, Bg, c.V, tok, io.tok_stride, lp_tok,
+                                          io.lp_stride, lse, score, plen, t, m->hdr()));
+    } else if (io.head) {
         EpiArgs ea; ea.hdr = m->hdr();
         ea.out_f32 = logits; ea.ld_out = c.V;
         CKP(RLT_K_HEAD, launch_gemm<T>(L, Epi::StoreF32, A, d, m->at<T>(m->lay.unembed), Bg, c.V, d, ea));
-        CKP(RLT_K_LSE, launch_lse_gather(L, logits, Bg, c.V, io.tau, io.tok ? io.tok + rb * io.tok_stride : nullptr,
-                                         io.tok_stride, io.logp_tok ? io.logp_tok + rb * io.lp_stride : nullptr,
-                                         io.lp_stride, io.lse ? io.lse + rb : nullptr,
-                                         io.logp_full ? io.logp_full + rb * c.V : nullptr,
-                                         io.score ? io.score + rb : nullptr,
-                                         io.prompt_len ? io.prompt_len + rb : nullptr, t, m->hdr()));
+        CKP(RLT_K_LSE, launch_lse_gather(L, logits, Bg, c.V, io.tau, tok, io.tok_stride, lp_tok, io.lp_stride, lse,
+                                         io.logp_full ? io.logp_full + rb * c.V : nullptr, score, plen, t,
+                                         m->hdr()));
     }
     return RLT_OK;
 }
