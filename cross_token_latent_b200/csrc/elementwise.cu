@@ -37,13 +37,13 @@ __global__ void k_rope_table(float2* table, int max_pos, int half, int hd, doubl
 }
 
 template <typename T>
-__global__ void k_embed(const int32_t* __restrict__ tok, int N, const T* __restrict__ embed, int V,
+__global__ void k_embed(const int32_t* __restrict__ tok, int tok_stride, int N, const T* __restrict__ embed, int V,
                         int d, float* __restrict__ h, DevHeader* hdr) {
     pdl_wait();
     pdl_trigger();
     int n = blockIdx.x;
     if (n >= N) return;
-    int id = tok[n];
+    int id = tok[(long long)n * tok_stride];
     if (id < 0 || id >= V) {
         if (threadIdx.x == 0) raise_flag(hdr, ERR_BAD_TOKEN);
         id = 0;
@@ -235,6 +235,44 @@ __global__ void k_enc_qkv_layout(const float* __restrict__ qkv, int B, int Tn, i
     }
 }
 
+// Encoder key/value cache of one layer, cache_l [2][B][H][T_max][hd] (keys after RoPE, both in
+// the storage type, exactly as the token-parallel encoder rounds them).  Thread per
+// (token n, head, pair i < hd/2) of qkv float32 [B*Tn, 3d]; token n of sequence b is position
+// pos0 + n % Tn.  With q_out set (Tn = 1), the rotated query, rounded like the encoder's stored
+// queries, goes to q_out [B, d] float32.
+template <typename T>
+__global__ void k_enc_cache_write(const float* __restrict__ qkv, int B, int Tn, int H, int hd,
+                                  const float2* __restrict__ rope, int pos0, T* __restrict__ cache_l, int T_max,
+                                  float* __restrict__ q_out) {
+    pdl_wait();
+    pdl_trigger();
+    const int half = hd / 2, d = H * hd;
+    const long long total = (long long)B * Tn * H * half;
+    const long long plane = (long long)B * H * T_max * hd;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int f = (int)(i % half);
+        const long long r = i / half;
+        const int h = (int)(r % H);
+        const long long n = r / H;
+        const int b = (int)(n / Tn), p = pos0 + (int)(n % Tn);
+        const float* row = qkv + n * 3 * d + h * hd;
+        const float2 cs = rope[(long long)p * half + f];
+        const long long o = (((long long)b * H + h) * T_max + p) * hd;
+        const float ka = row[d + f], kb = row[d + f + half];
+        cache_l[o + f] = from_f<T>(ka * cs.x - kb * cs.y);
+        cache_l[o + f + half] = from_f<T>(ka * cs.y + kb * cs.x);
+        cache_l[plane + o + f] = from_f<T>(row[2 * d + f]);
+        cache_l[plane + o + f + half] = from_f<T>(row[2 * d + f + half]);
+        if (q_out) {
+            const float qa = row[f], qb = row[f + half];
+            float* qo = q_out + (long long)b * d + h * hd;
+            qo[f] = round_to<T>(qa * cs.x - qb * cs.y);
+            qo[f + half] = round_to<T>(qa * cs.y + qb * cs.x);
+        }
+    }
+}
+
 template <typename T>
 __global__ void k_mem_layout(const float* __restrict__ kv, int B, int Tn, int T_alloc, int H, int hd,
                              T* __restrict__ Mg) {
@@ -292,8 +330,8 @@ cudaError_t launch_rope_table(Launch L, float2* table, int max_pos, int head_dim
 
 template <typename T>
 cudaError_t launch_embed(Launch L, const int32_t* tok, int N, const T* embed, int V, int d, float* h,
-                         DevHeader* hdr) {
-    return launch_k(L, k_embed<T>, N, 128, 0, tok, N, embed, V, d, h, hdr);
+                         DevHeader* hdr, int tok_stride) {
+    return launch_k(L, k_embed<T>, N, 128, 0, tok, tok_stride, N, embed, V, d, h, hdr);
 }
 
 template <typename T>
@@ -343,6 +381,13 @@ cudaError_t launch_mem_layout(Launch L, const float* kv, int B, int Tn, int T_al
                     H, hd, Mg);
 }
 
+template <typename T>
+cudaError_t launch_enc_cache_write(Launch L, const float* qkv, int B, int Tn, int H, int hd, const float2* rope,
+                                   int pos0, T* cache_l, int T_max, float* q_out) {
+    return launch_k(L, k_enc_cache_write<T>, grid_for((long long)B * Tn * H * (hd / 2), 256), 256, 0, qkv, B, Tn, H,
+                    hd, rope, pos0, cache_l, T_max, q_out);
+}
+
 cudaError_t launch_state_init(Launch L, const float* s_star, int B, int d, float* s, StateHeader* sh,
                               uint64_t version) {
     return launch_k(L, k_state_init, grid_for((long long)B * d, 256), 256, 0, s_star, B, d, s, sh, version);
@@ -351,7 +396,7 @@ cudaError_t launch_state_init(Launch L, const float* s_star, int B, int d, float
 #define RLT_INST(T)                                                                                   \
     template cudaError_t launch_pack_rows<T>(Launch, const float*, T*, int, int, int, int, int, int); \
     template cudaError_t launch_embed<T>(Launch, const int32_t*, int, const T*, int, int, float*,     \
-                                         DevHeader*);                                                 \
+                                         DevHeader*, int);                                            \
     template cudaError_t launch_rmsnorm<T>(Launch, const float*, int, int, const float*, float, T*,   \
                                            int, int, int, T*);                                        \
     template cudaError_t launch_merge_prep<T>(Launch, const T*, int, int, const float*, T*, int, int, \
@@ -360,7 +405,9 @@ cudaError_t launch_state_init(Launch L, const float* s_star, int B, int d, float
                                               float*, T*, StateHeader*, int);                         \
     template cudaError_t launch_enc_qkv_layout<T>(Launch, const float*, int, int, int, int,           \
                                                   const float2*, T*, bool);                           \
-    template cudaError_t launch_mem_layout<T>(Launch, const float*, int, int, int, int, int, T*);
+    template cudaError_t launch_mem_layout<T>(Launch, const float*, int, int, int, int, int, T*);       \
+    template cudaError_t launch_enc_cache_write<T>(Launch, const float*, int, int, int, int, const float2*, int, \
+                                                   T*, int, float*);
 RLT_INST(float)
 RLT_INST(bf16)
 #undef RLT_INST

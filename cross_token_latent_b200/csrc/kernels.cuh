@@ -60,10 +60,10 @@ cudaError_t launch_pack_rows(Launch L, const float* src, T* dst, int rows, int c
                              int row_mult, int row_off, int col_off);
 // table[p*half + i] = (cos, sin)(p * base^(-2i/hd)), computed in double precision
 cudaError_t launch_rope_table(Launch L, float2* table, int max_pos, int head_dim, float base);
-// h[n, :] = embed[tok[n], :] in float32
+// h[n, :] = embed[tok[n * tok_stride], :] in float32
 template <typename T>
 cudaError_t launch_embed(Launch L, const int32_t* tok, int N, const T* embed, int V, int d, float* h,
-                         DevHeader* hdr);
+                         DevHeader* hdr, int tok_stride = 1);
 // out[row_map(n), out_col_off + :] = T(RMSNorm(x[n, :]) * gain).  row_map(n) =
 // (n / rows_per_seq) * out_rows_per_seq + n % rows_per_seq; out2 (optional) is a second
 // contiguous T copy with leading dimension d.
@@ -99,6 +99,12 @@ cudaError_t launch_enc_qkv_layout(Launch L, const float* qkv, int B, int Tn, int
 template <typename T>
 cudaError_t launch_mem_layout(Launch L, const float* kv, int B, int Tn, int T_alloc, int H, int hd,
                               T* Mg);
+// Encoder key/value cache of one layer [2][B][H][T_max][hd]: rotated keys and values of the Tn
+// tokens of qkv float32 [B*Tn, 3d] at positions pos0 .. pos0+Tn-1, in the storage type; with
+// q_out (Tn = 1) also the rotated, storage-rounded query as float32 [B, d].
+template <typename T>
+cudaError_t launch_enc_cache_write(Launch L, const float* qkv, int B, int Tn, int H, int hd, const float2* rope,
+                                   int pos0, T* cache_l, int T_max, float* q_out);
 // H_0: s[b, :] = s_star, header (t=0, version, B)
 cudaError_t launch_state_init(Launch L, const float* s_star, int B, int d, float* s, StateHeader* sh,
                               uint64_t version);
@@ -205,6 +211,16 @@ cudaError_t launch_xattn_decode(Launch L, const float* qc, const T* Mg, long lon
 // Encoder causal self-attention: planes T [3][B][H][T][hd] -> o T [B*T, d]
 template <typename T>
 cudaError_t launch_enc_attention(Launch L, const T* planes, T* o, int B, int Tn, int H, int hd);
+
+// ------------------------------------------------------------------ sample.cu
+// Largest vocabulary the sampler handles (its row lives in shared memory).
+int sample_max_vocab();
+// One token per row of logp [B, V] (log-probabilities at the sampling temperature) with the
+// uniform u[b]: top-k / top-p truncation (ties at a boundary kept), inverse CDF over the kept
+// tokens in id order.  tok[b * tok_stride] = the draw, blp[b] (optional) = its log-probability
+// under the truncated, renormalised distribution.
+cudaError_t launch_sample(Launch L, const float* logp, int B, int V, const float* u, int top_k, float top_p,
+                          int32_t* tok, int tok_stride, float* blp);
 
 // ------------------------------------------------------------------ attention_tc.cu
 // Tensor-core encoder attention (bf16, head_dim 64 or 128): q, k planes [B][H][T][hd] and the

@@ -153,8 +153,8 @@ struct rlt_model {
     uint64_t launches = 0;
     int device = -1;            // the CUDA device that holds the arena
     // rlt_set_option values
-    int opt_row_groups = 0;             // 0 auto, 1 one group, 2 two groups (B >= GROUP_MIN_ROWS)
-    int opt_group_attn_cap = 6;         // attention CTAs per SM while two groups run
+    int opt_row_groups = 1;             // 1 one group, 2 two groups when B >= GROUP_MIN_ROWS
+    int opt_attn_cap = 0;               // resident attention CTAs per SM (0: no cap)
     int opt_group_pdl = 0;              // programmatic dependent launch inside a group's chain
     // two row groups: library-owned streams, forked from and joined back to the caller's stream
     cudaStream_t gs[2] = {nullptr, nullptr};
@@ -176,7 +176,7 @@ struct rlt_model {
         return cudaEventCreateWithFlags(&fork_ev, cudaEventDisableTiming) == cudaSuccess;
     }
     int row_groups(int B) const {
-        if (opt_row_groups == 1 || B < GROUP_MIN_ROWS || cfg.dtype != RLT_BF16) return 1;
+        if (opt_row_groups != 2 || B < GROUP_MIN_ROWS || cfg.dtype != RLT_BF16) return 1;
         return 2;
     }
 
@@ -309,9 +309,15 @@ int xattn_splits(const rlt_config& c, int B, int t) {
 }
 
 // ------------------------------------------------------------------ encoder driver
+size_t enc_cache_layer_elems(const rlt_config& c, int B, int T_max) {
+    return (size_t)2 * B * c.n_heads * (size_t)T_max * c.head_dim;
+}
+
+// Token-parallel encoder over Tn tokens of B sequences; with `cache` (capacity T_max) it also
+// stores every layer's rotated keys and values of positions 0..Tn-1 for incremental appends.
 template <typename T>
 rlt_status encode_impl(rlt_model* m, const int32_t* tokens, int B, int Tn, int T_alloc, T* e, T* M,
-                       uint8_t* ws, cudaStream_t st) {
+                       uint8_t* ws, cudaStream_t st, T* cache = nullptr, int T_max = 0) {
     const rlt_config& c = m->cfg;
     Launch L{st, &m->launches};
     EncWS w = enc_ws(c, B, Tn);
@@ -331,6 +337,9 @@ rlt_status encode_impl(rlt_model* m, const int32_t* tokens, int B, int Tn, int T
         CK(launch_rmsnorm<T>(L, h, N, d, m->at<float>(m->lay.attn_norm[l]), c.rms_eps, a, d, N, N, nullptr));
         ea.out_f32 = qkv; ea.ld_out = 3 * d;
         CK(launch_gemm<T>(L, Epi::StoreF32, a, d, m->at<T>(m->lay.wqkv[l]), N, 3 * d, d, ea));
+        if (cache)
+            CK(launch_enc_cache_write<T>(L, qkv, B, Tn, H, hd, rope, 0,
+                                         cache + (size_t)l * enc_cache_layer_elems(c, B, T_max), T_max, nullptr));
         if (use_tc_attn) {
             bf16* pl = reinterpret_cast<bf16*>(planes);
             size_t plane = (size_t)N * d;
@@ -359,6 +368,80 @@ rlt_status encode_impl(rlt_model* m, const int32_t* tokens, int B, int Tn, int T
         CK(launch_gemm<T>(L, Epi::StoreF32, ews, d, m->at<T>(m->lay.mem) + (size_t)g * 2 * d * d, N, 2 * d, d, ea));
         CK(launch_mem_layout<T>(L, qkv, B, Tn, T_alloc, H, hd, M + g * group_elems));
     }
+    return RLT_OK;
+}
+
+// ------------------------------------------------------------------ incremental encoder
+struct AppWS {
+    size_t h, a, act, qkv, q, att, ews, part, total;
+};
+AppWS app_ws(const rlt_config& c, int B) {
+    AppWS w;
+    size_t d = c.d, e = c.dtype == RLT_BF16 ? 2 : 4;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes); return o; };
+    w.h = take((size_t)B * d * 4);
+    w.a = take((size_t)B * d * e);
+    w.act = take((size_t)B * c.F * e);
+    w.qkv = take((size_t)B * 3 * d * 4);
+    w.q = take((size_t)B * d * 4);
+    w.att = take((size_t)B * d * e);
+    w.ews = take((size_t)B * d * e);
+    w.part = take((size_t)XATTN_PART_ITEMS * (c.head_dim + 2) * 4);
+    w.total = off;
+    return w;
+}
+
+// One new token per sequence at position pos: the encoder layers run on B rows, each layer's
+// causal attention reads the cached keys/values of positions 0..pos (the new ones written
+// first), and the new encoder output and memory rows go to e[:, pos] and M[..., pos, :].
+template <typename T>
+rlt_status encode_append_impl(rlt_model* m, const int32_t* tok, int tok_stride, int B, int pos, T* cache, int T_max,
+                              T* e, T* M, int T_alloc, uint8_t* ws, cudaStream_t st) {
+    const rlt_config& c = m->cfg;
+    Launch L{st, &m->launches};
+    AppWS w = app_ws(c, B);
+    const int d = c.d, F = c.F, H = c.n_heads, hd = c.head_dim;
+    float* h = reinterpret_cast<float*>(ws + w.h);
+    T* a = reinterpret_cast<T*>(ws + w.a);
+    T* act = reinterpret_cast<T*>(ws + w.act);
+    float* qkv = reinterpret_cast<float*>(ws + w.qkv);
+    float* q = reinterpret_cast<float*>(ws + w.q);
+    T* att = reinterpret_cast<T*>(ws + w.att);
+    T* ews = reinterpret_cast<T*>(ws + w.ews);
+    float* part = reinterpret_cast<float*>(ws + w.part);
+    const float2* rope = m->at<float2>(m->lay.rope);
+    const long long cplane = (long long)B * H * T_max * hd;
+    const int splits = xattn_splits(c, B, pos + 1);
+    int p = m->prof.begin(RLT_K_ENCODER, st);
+    CK(launch_embed<T>(L, tok, B, m->at<T>(m->lay.embed), c.V, d, h, m->hdr(), tok_stride));
+    for (int l = 0; l < c.L_E; ++l) {
+        T* cache_l = cache + (size_t)l * enc_cache_layer_elems(c, B, T_max);
+        EpiArgs ea; ea.hdr = m->hdr();
+        CK(launch_rmsnorm<T>(L, h, B, d, m->at<float>(m->lay.attn_norm[l]), c.rms_eps, a, d, B, B, nullptr));
+        ea.out_f32 = qkv; ea.ld_out = 3 * d;
+        CK(launch_gemm<T>(L, Epi::StoreF32, a, d, m->at<T>(m->lay.wqkv[l]), B, 3 * d, d, ea));
+        CK(launch_enc_cache_write<T>(L, qkv, B, 1, H, hd, rope, pos, cache_l, T_max, q));
+        CK(launch_xattn_decode<T>(L, q, cache_l, cplane, T_max, pos + 1, att, B, H, hd, splits, part));
+        ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = h; ea.ld_out = d;
+        CK(launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.wo[l]), B, d, d, ea));
+        CK(launch_rmsnorm<T>(L, h, B, d, m->at<float>(m->lay.ffn_norm[l]), c.rms_eps, a, d, B, B, nullptr));
+        ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_t = act; ea.ld_out = F;
+        CK(launch_gemm<T>(L, Epi::SwiGLU, a, d, m->at<T>(m->lay.wgu[l]), B, 2 * F, d, ea));
+        ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = h; ea.ld_out = d;
+        CK(launch_gemm<T>(L, Epi::ResidAdd, act, F, m->at<T>(m->lay.wdown[l]), B, d, F, ea));
+    }
+    // e[:, pos] = RMSNorm(h) (row b lands at b * T_alloc + pos), plus a contiguous copy for M
+    CK(launch_rmsnorm<T>(L, h, B, d, m->at<float>(m->lay.enc_norm), c.rms_eps, e + (size_t)pos * d, d, 1, T_alloc,
+                         ews));
+    const size_t group_elems = (size_t)2 * B * H * (size_t)T_alloc * hd;
+    for (int g = 0; g < c.G; ++g) {
+        EpiArgs ea; ea.hdr = m->hdr();
+        ea.out_f32 = qkv; ea.ld_out = 2 * d;
+        CK(launch_gemm<T>(L, Epi::StoreF32, ews, d, m->at<T>(m->lay.mem) + (size_t)g * 2 * d * d, B, 2 * d, d, ea));
+        CK(launch_mem_layout<T>(L, qkv, B, 1, T_alloc, H, hd, M + g * group_elems + (size_t)pos * hd));
+    }
+    m->prof.end(p, st);
     return RLT_OK;
 }
 
@@ -510,7 +593,9 @@ rlt_status step_impl(rlt_model* m, uint8_t* state, int B, const T* e, const T* M
     DecWS w = dec_ws(m->cfg, B);
     float* part = reinterpret_cast<float*>(ws + w.part);
     if (m->row_groups(B) == 1 || !m->group_streams()) {
-        return step_rows<T>(m, state, B, 0, B, e, M, T_alloc, t, io, ws, part, true, Launch{st, &m->launches});
+        Launch L{st, &m->launches};
+        L.attn_ctas_per_sm = m->opt_attn_cap;
+        return step_rows<T>(m, state, B, 0, B, e, M, T_alloc, t, io, ws, part, true, L);
     }
     float* part2 = reinterpret_cast<float*>(ws + w.part2);
     const int B0 = (B / 2 + 127) / 128 * 128;           // group 0: whole 128-row tiles
@@ -520,7 +605,7 @@ rlt_status step_impl(rlt_model* m, uint8_t* state, int B, const T* e, const T* M
         CK(cudaStreamWaitEvent(m->gs[g], m->fork_ev, 0));
         Launch L{m->gs[g], &m->launches};
         L.pdl = m->opt_group_pdl != 0;
-        L.attn_ctas_per_sm = m->opt_group_attn_cap;
+        L.attn_ctas_per_sm = m->opt_attn_cap;
         r = g == 0 ? step_rows<T>(m, state, B, 0, B0, e, M, T_alloc, t, io, ws, part, true, L)
                    : step_rows<T>(m, state, B, B0, B - B0, e, M, T_alloc, t, io, ws, part2, false, L);
     }
@@ -742,6 +827,62 @@ rlt_status rlt_decode_step(rlt_model* m, void* state, int B, const void* e, cons
     return s;
 }
 
+size_t rlt_encoder_cache_bytes(const rlt_model* m, int B, int T_max) {
+    if (!m || B < 1 || T_max < 1) return 0;
+    return (size_t)m->cfg.L_E * enc_cache_layer_elems(m->cfg, B, T_max) * m->lay.esz;
+}
+
+rlt_status rlt_encode_prefill(rlt_model* m, const int32_t* tokens, int B, int T, int T_alloc, void* e, void* M,
+                              void* enc_cache, int T_max, void* ws, size_t ws_bytes, void* stream) {
+    if (!m || !tokens || !e || !M || !enc_cache || !ws || B < 1 || T < 1 || T > T_alloc || T_alloc > m->cfg.max_pos)
+        return RLT_EINVAL;
+    if (T > T_max || T_max > m->cfg.max_pos) return RLT_EINVAL;
+    if (m->version == 0) return RLT_EINVAL;
+    if (!aligned(e) || !aligned(M) || !aligned(ws) || !aligned(enc_cache) || !aligned(tokens, 4)) return RLT_EINVAL;
+    if (ws_bytes < enc_ws(m->cfg, B, T).total) return RLT_EINVAL;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* w = reinterpret_cast<uint8_t*>(ws);
+    int p = m->prof.begin(RLT_K_ENCODER, st);
+    rlt_status s = m->cfg.dtype == RLT_BF16
+        ? encode_impl<bf16>(m, tokens, B, T, T_alloc, (bf16*)e, (bf16*)M, w, st, (bf16*)enc_cache, T_max)
+        : encode_impl<float>(m, tokens, B, T, T_alloc, (float*)e, (float*)M, w, st, (float*)enc_cache, T_max);
+    m->prof.end(p, st);
+    return s;
+}
+
+size_t rlt_encode_append_workspace_bytes(const rlt_model* m, int B) {
+    if (!m || B < 1) return 0;
+    return app_ws(m->cfg, B).total;
+}
+
+rlt_status rlt_encode_append(rlt_model* m, const int32_t* tokens, int tok_stride, int B, int pos, void* enc_cache,
+                             int T_max, void* e, void* M, int T_alloc, void* ws, size_t ws_bytes, void* stream) {
+    if (!m || !tokens || !enc_cache || !e || !M || !ws || B < 1 || tok_stride < 1 || pos < 0) return RLT_EINVAL;
+    if (pos >= T_max || pos >= T_alloc || T_max > m->cfg.max_pos || T_alloc > m->cfg.max_pos) return RLT_EINVAL;
+    if (m->version == 0) return RLT_EINVAL;
+    if (!aligned(e) || !aligned(M) || !aligned(ws) || !aligned(enc_cache) || !aligned(tokens, 4)) return RLT_EINVAL;
+    if (ws_bytes < app_ws(m->cfg, B).total) return RLT_EINVAL;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* w = reinterpret_cast<uint8_t*>(ws);
+    return m->cfg.dtype == RLT_BF16
+        ? encode_append_impl<bf16>(m, tokens, tok_stride, B, pos, (bf16*)enc_cache, T_max, (bf16*)e, (bf16*)M,
+                                   T_alloc, w, st)
+        : encode_append_impl<float>(m, tokens, tok_stride, B, pos, (float*)enc_cache, T_max, (float*)e, (float*)M,
+                                    T_alloc, w, st);
+}
+
+rlt_status rlt_sample(rlt_model* m, const float* logp, int B, const float* u, int top_k, float top_p,
+                      int32_t* tokens, int tok_stride, float* behaviour_logp, void* stream) {
+    if (!m || !logp || !u || !tokens || B < 1 || tok_stride < 1 || top_k < 0 || !(top_p > 0.f) || top_p > 1.f)
+        return RLT_EINVAL;
+    if (!aligned(logp, 4) || !aligned(u, 4) || !aligned(tokens, 4) || (behaviour_logp && !aligned(behaviour_logp, 4)))
+        return RLT_EINVAL;
+    if (m->cfg.V > sample_max_vocab()) return RLT_EUNSUPPORTED;
+    Launch L = m->launch(stream);
+    CK(launch_sample(L, logp, B, m->cfg.V, u, top_k, top_p, tokens, tok_stride, behaviour_logp));
+    return RLT_OK;
+}
+
 // ---------------------------------------------------------------- decode step without allocation
 //
 // Scratch for rlt_decode_step_noalloc: a file-scope device array that every GPU which loads
@@ -867,11 +1008,11 @@ rlt_status rlt_set_option(rlt_model* m, const char* name, int64_t value) {
     if (!m || !name) return RLT_EINVAL;
     const std::string n(name);
     if (n == "row_groups") {
-        if (value < 0 || value > 2) return RLT_EINVAL;
+        if (value < 1 || value > 2) return RLT_EINVAL;
         m->opt_row_groups = (int)value;
-    } else if (n == "group_attn_ctas_per_sm") {
+    } else if (n == "attn_ctas_per_sm") {
         if (value < 0 || value > 32) return RLT_EINVAL;
-        m->opt_group_attn_cap = (int)value;
+        m->opt_attn_cap = (int)value;
     } else if (n == "group_pdl") {
         if (value < 0 || value > 1) return RLT_EINVAL;
         m->opt_group_pdl = (int)value;

@@ -48,6 +48,16 @@ _EXPORTS = {
     "rlt_encode": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                   ctypes.c_void_p]),
+    "rlt_encoder_cache_bytes": (ctypes.c_size_t, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int]),
+    "rlt_encode_prefill": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                          ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "rlt_encode_append_workspace_bytes": (ctypes.c_size_t, [ctypes.c_void_p, ctypes.c_int]),
+    "rlt_encode_append": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                         ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "rlt_sample": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int,
+                                  ctypes.c_float, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]),
     "rlt_state_bytes": (ctypes.c_size_t, [ctypes.c_void_p, ctypes.c_int]),
     "rlt_state_init": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]),
     "rlt_state_copy": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
@@ -243,6 +253,73 @@ class RLTModel:
         _check(lib().rlt_encode(self.handle, _ptr(tokens), B, T, T_alloc, _ptr(e), _ptr(M), _ptr(ws), ws.numel(),
                                 _stream()), "rlt_encode")
         return e, M
+
+    # ---------------------------------------------------------------- incremental encoder
+    def alloc_encoder_cache(self, B: int, T_max: int) -> torch.Tensor:
+        return torch.empty(lib().rlt_encoder_cache_bytes(self.handle, B, T_max), dtype=torch.uint8,
+                           device=self.device)
+
+    def encode_prefill(self, tokens: torch.Tensor, T_alloc: int, T_max: int | None = None, out=None, cache=None):
+        """rlt_encode_prefill: (e, M, encoder cache) of the first T tokens, capacities T_alloc / T_max."""
+        tokens = tokens.to(device=self.device, dtype=torch.int32).contiguous()
+        B, T = tokens.shape
+        T_max = T_alloc if T_max is None else T_max
+        e, M = out if out is not None else self.alloc_encoder_outputs(B, T_alloc)
+        cache = self.alloc_encoder_cache(B, T_max) if cache is None else cache
+        nb = lib().rlt_encode_workspace_bytes(self.handle, B, T)
+        ws = self._workspace(("enc", B, T), nb)
+        _check(lib().rlt_encode_prefill(self.handle, _ptr(tokens), B, T, T_alloc, _ptr(e), _ptr(M), _ptr(cache), T_max,
+                                        _ptr(ws), ws.numel(), _stream()), "rlt_encode_prefill")
+        return e, M, cache
+
+    def encode_append(self, tokens: torch.Tensor, pos: int, cache: torch.Tensor, T_max: int, e: torch.Tensor,
+                      M: torch.Tensor) -> None:
+        """rlt_encode_append: tokens is an int32 device vector [B] or a column view of a [B, T]
+        matrix (its stride is passed through); the token at position pos is encoded."""
+        B = tokens.shape[0]
+        stride = tokens.stride(0)
+        nb = lib().rlt_encode_append_workspace_bytes(self.handle, B)
+        ws = self._workspace(("app", B), nb)
+        _check(lib().rlt_encode_append(self.handle, _ptr(tokens), stride, B, int(pos), _ptr(cache), int(T_max), _ptr(e),
+                                       _ptr(M), e.shape[1], _ptr(ws), ws.numel(), _stream()), "rlt_encode_append")
+
+    def sample(self, logp: torch.Tensor, u: torch.Tensor, top_k: int = 0, top_p: float = 1.0,
+               out: torch.Tensor | None = None, behaviour_logp: torch.Tensor | None = None) -> torch.Tensor:
+        """rlt_sample: one token per row of logp [B, V] with the uniforms u [B]; `out` may be a
+        column view of a token matrix (its stride is passed through)."""
+        B = logp.shape[0]
+        out = torch.empty(B, dtype=torch.int32, device=self.device) if out is None else out
+        _check(lib().rlt_sample(self.handle, _ptr(logp), B, _ptr(u), int(top_k), float(top_p), _ptr(out),
+                                out.stride(0), _ptr(behaviour_logp), _stream()), "rlt_sample")
+        return out
+
+    def generate(self, prompt: torch.Tensor, n_new: int, uniforms: torch.Tensor, tau: float = 1.0, top_k: int = 0,
+                 top_p: float = 1.0):
+        """Sample n_new tokens after each prompt row (all rows in lockstep): encode the prompt with a
+        cache, step the decoder through it, then repeat [sample x_{t+1} from logp_t, encode it
+        incrementally, step].  uniforms: float device [n_new, B].  Returns (tokens [B, P + n_new]
+        int32, behaviour log-probs [B, n_new], prompt log-probs [B, P - 1] (entry t-1 = log p of
+        x_{t+1}), the state after all P + n_new tokens).  Every step of the loop runs in the
+        library's kernels; nothing is copied to the host."""
+        prompt = prompt.to(device=self.device, dtype=torch.int32).contiguous()
+        B, P = prompt.shape
+        T = P + n_new
+        toks = torch.empty((T, B), dtype=torch.int32, device=self.device)     # row t = x_{t+1}
+        toks[:P] = prompt.t()
+        e, M, cache = self.encode_prefill(prompt, T_alloc=T, T_max=T)
+        st = self.new_state(B)
+        blp = torch.empty((n_new, B), dtype=torch.float32, device=self.device)
+        lp_prompt = torch.zeros((max(P - 1, 0), B), dtype=torch.float32, device=self.device)
+        row = torch.empty((B, self.cfg.V), dtype=torch.float32, device=self.device)
+        for t in range(1, T):                      # step t consumes x_t and predicts x_{t+1}
+            if t < P:
+                self.decode_step(st, e, M, next_tok=toks[t], tau=tau, logp_tok=lp_prompt[t - 1])
+                continue
+            self.decode_step(st, e, M, tau=tau, logp_full=row)
+            self.sample(row, uniforms[t - P], top_k, top_p, out=toks[t], behaviour_logp=blp[t - P])
+            self.encode_append(toks[t], t, cache, T, e, M)
+        self.decode_step(st, e, M, tau=tau)         # the transition of x_T
+        return toks.t().contiguous(), blp.t().contiguous(), lp_prompt.t().contiguous(), st
 
     # ---------------------------------------------------------------- decoder
     def new_state(self, B: int) -> RLTState:

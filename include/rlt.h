@@ -131,6 +131,56 @@ size_t rlt_encode_workspace_bytes(const rlt_model* m, int B, int T);
 rlt_status rlt_encode(rlt_model* m, const int32_t* tokens, int B, int T, int T_alloc,
                       void* e, void* M, void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------- incremental encoder */
+
+/* Bytes of an encoder key/value cache for B sequences of up to T_max tokens:
+ * [L_E, 2, B, n_heads, T_max, head_dim] in the model dtype (keys after the rotary embedding). */
+size_t rlt_encoder_cache_bytes(const rlt_model* m, int B, int T_max);
+
+/* rlt_encode that also keeps the encoder's keys and values of positions 0..T-1 in a
+ * caller-owned cache of capacity T_max (T <= T_max <= max_pos), so that later tokens can be
+ * encoded one at a time (deepsonar teardown, 2.5: one execution semantics for prefill,
+ * generation and replay; the encoder is causal, so a prefix's encoding never changes).
+ * Workspace as for rlt_encode.  Errors: as rlt_encode. */
+rlt_status rlt_encode_prefill(rlt_model* m, const int32_t* tokens, int B, int T, int T_alloc, void* e, void* M,
+                              void* enc_cache, int T_max, void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes of one rlt_encode_append for B sequences. */
+size_t rlt_encode_append_workspace_bytes(const rlt_model* m, int B);
+
+/* Encode one new token per sequence at position pos (0-based; the cache holds positions
+ * 0..pos-1 from rlt_encode_prefill or earlier appends): every encoder layer attends causally
+ * over the cached keys/values plus the new ones, which are added to the cache; the new encoder
+ * output goes to e[:, pos] and its memory projections to M[..., pos, :].  The result equals the
+ * token-parallel encoding of the whole prefix (up to summation order).
+ *   tokens      device int32, token of sequence b at tokens[b * tok_stride] (a column of a
+ *               [B, T] token matrix has tok_stride T)
+ *   enc_cache   the cache of capacity T_max; e, M with row capacity T_alloc, as rlt_encode
+ * Requires pos < T_max <= max_pos and pos < T_alloc <= max_pos.  Out-of-range ids latch
+ * RLT_EDEVICE.  Errors: RLT_EINVAL, RLT_ECUDA. */
+rlt_status rlt_encode_append(rlt_model* m, const int32_t* tokens, int tok_stride, int B, int pos, void* enc_cache,
+                             int T_max, void* e, void* M, int T_alloc, void* ws, size_t ws_bytes, void* stream);
+
+/* Draw the next token of each sequence (news summary, model-RL co-design principle: the
+ * behaviour log-probability is taken under the distribution actually sampled from).
+ *   logp            device float [B, V]: log-probabilities at the sampling temperature, e.g.
+ *                   the logp_full output of rlt_decode_step at that tau
+ *   u               device float [B]: caller-drawn uniforms in [0, 1)
+ *   top_k           keep token i when fewer than top_k tokens are strictly more probable
+ *                   (0: no top-k)
+ *   top_p           in (0, 1]: then keep i when the mass of the strictly more probable tokens
+ *                   is below top_p times the mass top-k kept (1: no top-p); tokens tied at
+ *                   either boundary are all kept
+ *   tokens          device int32 out: the draw of sequence b at tokens[b * tok_stride]: the
+ *                   first token id whose cumulative kept probability, ids in increasing order,
+ *                   exceeds u[b] times the kept total
+ *   behaviour_logp  device float [B] or NULL: log of the draw's probability after truncation
+ *                   and renormalisation
+ * Errors: RLT_EINVAL, RLT_EUNSUPPORTED (V above 49152: the row is staged in shared memory),
+ * RLT_ECUDA. */
+rlt_status rlt_sample(rlt_model* m, const float* logp, int B, const float* u, int top_k, float top_p,
+                      int32_t* tokens, int tok_stride, float* behaviour_logp, void* stream);
+
 /* ---------------------------------------------------------------- decoder state */
 
 /* Bytes of one decoder state H for B sequences: a 256-byte header, s [B, d] float32 and
@@ -233,17 +283,18 @@ uint64_t rlt_launch_count(const rlt_model* m);
 
 /* Scheduling options of a model handle (no counterpart on the pages; they change how a step is
  * scheduled on the GPU, never what it computes beyond summation order):
- *   "row_groups"              0 (default) automatic: a bf16 step of B >= 256 sequences runs as
- *                             two row groups, each on a library-owned stream forked from and
- *                             joined back into the caller's stream, so that one group's
- *                             attention (HBM-bound) overlaps the other group's projections
- *                             (tensor cores); 1 always one group; 2 same as 0.
- *   "group_attn_ctas_per_sm"  with two groups, the cap on resident attention CTAs per SM
- *                             (0 = none; default 6), which leaves every SM room for the other
- *                             group's GEMM CTAs.
- *   "group_pdl"               1: programmatic dependent launch inside each group's chain
- *                             (default 0: an early-launched kernel would hold SM resources the
- *                             other group needs).
+ *   "row_groups"         1 (default): one step is one chain of kernels on the caller's stream;
+ *                        2: a bf16 step of B >= 256 sequences runs as two row groups, each on a
+ *                        library-owned stream forked from and joined back into the caller's
+ *                        stream, so that one group's attention can overlap the other group's
+ *                        projections.
+ *   "attn_ctas_per_sm"   cap on the resident CTAs per SM of the decoder's attention kernels
+ *                        (0, the default: none), leaving room on every SM for projection CTAs
+ *                        that start early (programmatic launch) or run on the other group's
+ *                        stream.
+ *   "group_pdl"          1: programmatic dependent launch inside each row group's chain
+ *                        (default 0: an early-launched kernel would hold SM resources the
+ *                        other group needs).
  * Errors: RLT_EINVAL (unknown name or value out of range). */
 rlt_status rlt_set_option(rlt_model* m, const char* name, int64_t value);
 

@@ -43,6 +43,9 @@ Readings taken where the pages leave a step open (each is a documented choice):
                 are rounded to bfloat16 (round to nearest even).  The residual
                 stream, norms, decoder queries, softmax and its probabilities,
                 s_t, the log-sum-exp and logp stay in full precision.
+  R12 sampling  top-k and top-p keep every token tied at their boundary; the kept tokens
+                are renormalised and sampled by inverse CDF in token-id order with a
+                caller-given uniform (sample_token).
 """
 from __future__ import annotations
 
@@ -107,6 +110,46 @@ def silu(x: np.ndarray) -> np.ndarray:
 
 def sigmoid(x: np.ndarray) -> np.ndarray:
     return 1.0 / (1.0 + np.exp(-x))
+
+
+def sample_token(logp: np.ndarray, u: float, top_k: int = 0, top_p: float = 1.0):
+    """Draw one token from the next-token distribution with a caller-given uniform u in [0, 1)
+    ([teardown] 2.5: generation runs the same transition; [news] model-RL principle: the
+    behaviour log-probability is the one of the distribution actually sampled from).
+
+    logp: log-probabilities of one row at the sampling temperature (log_softmax(z / tau)).
+    Truncation (reading R12): with p = exp(logp), top-k keeps token i when fewer than k tokens
+    are strictly more probable than i (top_k <= 0: no top-k); top-p then keeps i when the
+    probability mass of the tokens strictly more probable than i is below top_p times the mass
+    top-k kept (top_p >= 1: no top-p).  Tokens tied at a boundary are all kept.  The kept
+    tokens are renormalised to total Z and the token is the inverse CDF at u * Z, the kept
+    tokens taken in increasing id order: the first id whose cumulative kept mass exceeds u * Z.
+    Returns (token, behaviour log-probability log(p_token / Z))."""
+    lp = np.asarray(logp, np.float64)
+    p = np.exp(lp)
+    V = p.shape[0]
+    keep = np.ones(V, bool)
+    if top_k > 0:
+        for i in range(V):
+            keep[i] = np.count_nonzero(p > p[i]) < top_k
+    if top_p < 1.0:
+        z1 = p[keep].sum()
+        keep_p = np.zeros(V, bool)
+        for i in range(V):
+            if keep[i]:
+                keep_p[i] = p[keep & (p > p[i])].sum() < top_p * z1
+        keep = keep_p
+    z = p[keep].sum()
+    target = u * z
+    acc = 0.0
+    last = -1
+    for i in range(V):
+        if keep[i]:
+            acc += p[i]
+            last = i
+            if acc > target:
+                return i, float(lp[i] - np.log(z))
+    return last, float(lp[last] - np.log(z))
 
 
 # ----------------------------------------------------------------------------------

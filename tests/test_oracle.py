@@ -12,7 +12,7 @@ import pytest
 import scipy.special
 import torch
 
-from oracle import RLTOracle, round_bf16, rms_norm, rope
+from oracle import RLTOracle, round_bf16, rms_norm, rope, sample_token
 from workloads import TINY, SMALL, make_tokens, make_weights
 import parallel_ref as pref
 
@@ -337,6 +337,67 @@ def test_head_is_log_softmax_at_temperature():
         np.testing.assert_allclose(np.exp(lp).sum(-1), 1.0, atol=1e-12)
     # infinite temperature -> uniform
     np.testing.assert_allclose(o.head(s, 1e12), -np.log(TINY_M.V), atol=1e-9)
+
+
+# ---------------------------------------------------------------- sampler (reading R12)
+
+def _lp(p):
+    return np.log(np.asarray(p, np.float64))
+
+
+def test_sampler_inverse_cdf_on_a_known_distribution():
+    """p = (0.1, 0.2, 0.3, 0.4): the CDF in id order is 0.1, 0.3, 0.6, 1.0, so u picks the first
+    id whose cumulative mass exceeds u; the behaviour log-prob is log p."""
+    lp = _lp([0.1, 0.2, 0.3, 0.4])
+    for u, want in ((0.0, 0), (0.05, 0), (0.11, 1), (0.29, 1), (0.31, 2), (0.59, 2), (0.61, 3), (0.999, 3)):
+        tok, blp = sample_token(lp, u)
+        assert tok == want, (u, tok)
+        assert blp == pytest.approx(math.log([0.1, 0.2, 0.3, 0.4][want]), abs=1e-12)
+
+
+def test_sampler_top_k_and_top_p_renormalise_the_kept_tokens():
+    lp = _lp([0.1, 0.2, 0.3, 0.4])
+    # top-k 2 keeps ids 2, 3 (0.3, 0.4): renormalised CDF 3/7, 1
+    assert sample_token(lp, 0.42, top_k=2) == (2, pytest.approx(math.log(3 / 7), abs=1e-12))
+    assert sample_token(lp, 0.43, top_k=2) == (3, pytest.approx(math.log(4 / 7), abs=1e-12))
+    # top-p 0.5: id 3 has no more-probable mass, id 2 has 0.4 < 0.5, id 1 has 0.7: kept {2, 3}
+    assert sample_token(lp, 0.0, top_p=0.5)[0] == 2
+    assert sample_token(lp, 0.9, top_p=0.5) == (3, pytest.approx(math.log(4 / 7), abs=1e-12))
+    # top-p 0.4: id 2 has exactly 0.4 more-probable mass, not below 0.4: only id 3 is kept
+    assert sample_token(lp, 0.0, top_p=0.4) == (3, pytest.approx(0.0, abs=1e-12))
+    # top-k 3 then top-p 0.5 of the kept mass 0.9: ids 3 (0 < 0.45), 2 (0.4 < 0.45), 1 (0.7): {2, 3}
+    assert sample_token(lp, 0.0, top_k=3, top_p=0.5)[0] == 2
+    # top-k 3 then top-p 0.4 of 0.9 = 0.36: id 2 has 0.4 >= 0.36: only id 3
+    assert sample_token(lp, 0.0, top_k=3, top_p=0.4)[0] == 3
+
+
+def test_sampler_keeps_every_token_tied_at_the_boundary():
+    lp = _lp([0.25, 0.25, 0.25, 0.25])
+    # top-k 1: no token has a strictly more probable one, so all four stay: uniform
+    assert [sample_token(lp, u, top_k=1)[0] for u in (0.1, 0.3, 0.6, 0.9)] == [0, 1, 2, 3]
+    assert sample_token(lp, 0.3, top_k=1)[1] == pytest.approx(math.log(0.25), abs=1e-12)
+    lp2 = _lp([0.1, 0.3, 0.3, 0.3])
+    # top-k 2: the three 0.3 ties stay, 0.1 goes (three tokens are more probable than it)
+    assert sample_token(lp2, 0.0, top_k=2)[0] == 1
+    assert sample_token(lp2, 0.0, top_k=2)[1] == pytest.approx(math.log(1 / 3), abs=1e-12)
+
+
+def test_sampler_frequencies_match_the_truncated_distribution():
+    """Over 20000 evenly spaced uniforms the token counts equal the kept probabilities
+    (renormalised) within one count per token."""
+    rng = np.random.default_rng(21)
+    z = rng.standard_normal(40) * 2
+    lp = z - scipy.special.logsumexp(z)
+    p = np.exp(lp)
+    order = np.argsort(-p)
+    kept = np.zeros(40, bool)
+    kept[order[:7]] = True                       # top-k 7 (no ties in a continuous draw)
+    n = 20000
+    counts = np.zeros(40)
+    for j in range(n):
+        counts[sample_token(lp, (j + 0.5) / n, top_k=7)[0]] += 1
+    want = np.where(kept, p, 0) / p[kept].sum() * n
+    assert np.all(np.abs(counts - want) <= 1.0 + 1e-9)
 
 
 # ---------------------------------------------------------------- replay contract
