@@ -293,6 +293,7 @@ def main() -> int:
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-replay", action="store_true")
+    ap.add_argument("--no-generate", action="store_true")
     ap.add_argument("--nvtx-sample", type=int, default=0,
                     help="profiling runs: wrap this many evenly spaced steps of the first timed sweep in an NVTX "
                          "range 'sample' (for ncu --nvtx-include sample/); skips the breakdown sweep")
@@ -478,6 +479,29 @@ def main() -> int:
                   "roofline_ms": r_roof_ms, "frac": r_roof_ms / r_ms,
                   "includes": "rlt_replay: encode + T steps + response scoring",
                   "roofline_note": "decoder run roofline + encoder FLOPs at the bf16 burst peak"}
+    # the generation loop: prompt of T/2 tokens, then T/2 sampled ones (prefill with an encoder
+    # cache, decoder steps over the prompt, then [decode with the full row, sample, encode the
+    # draw incrementally] per new token); tokens/s counts the sampled tokens of all sequences
+    gen = None
+    if not args.no_generate and T >= 4:
+        P = T // 2
+        n_new = T - P
+        g = torch.Generator(device=dev).manual_seed(1234)
+        u = torch.rand((n_new, B), generator=g, device=dev)
+        prompt = tok[:, :P].contiguous()
+        model.generate(prompt, n_new, u, tau=wl.tau, top_k=50, top_p=0.95)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        model.generate(prompt, n_new, u, tau=wl.tau, top_k=50, top_p=0.95)
+        b.record()
+        torch.cuda.synchronize()
+        g_ms = max_over_ranks(a.elapsed_time(b), dev)
+        gen = {"value": world * B * n_new / (g_ms / 1e3), "unit": "generated tokens/s", "ms": g_ms,
+               "prompt": P, "new_tokens": n_new, "top_k": 50, "top_p": 0.95,
+               "includes": "rlt_encode_prefill, P decoder steps, then per new token: rlt_decode_step with the "
+                           "full log-prob row, rlt_sample, rlt_encode_append"}
+        model.release_workspaces()
     model.check_device_errors()
 
     cpu = None
@@ -492,7 +516,7 @@ def main() -> int:
             "vs_baseline": None, "dtype": m.dtype, "data": "synthetic",
             "config": {**arm_config(wl, B, T, world), **({"options": args.option} if args.option else {})},
             "roofline": roofline, "step_roofline": step_roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "replay": replay, "encode": enc, "gpu_launches": launches, "clocks": clocks,
+            "replay": replay, "encode": enc, "generate": gen, "gpu_launches": launches, "clocks": clocks,
             "kernel_breakdown_ms_per_sweep": {k: round(v[0], 3) for k, v in sorted(breakdown.items())},
         }
         print(json.dumps(line), flush=True)

@@ -134,9 +134,10 @@ constexpr int SWA_WARPS = 4;
 
 template <typename T, int HD>
 __global__ void __launch_bounds__(SWA_WARPS * 32, 6) k_swa_decode(const float* __restrict__ qkv,
-                                                                  const float2* __restrict__ rope_row,
+                                                                  const float2* __restrict__ rope,
                                                                   T* __restrict__ ring, T* __restrict__ o,
-                                                                  int B, int H, int W, int t, float qscale) {
+                                                                  int B, int H, int W, const int32_t* __restrict__ pos,
+                                                                  int max_t, float qscale) {
     using G = Geom<T, HD>;
     constexpr int EPL = G::EPL, LPK = G::LPK;
     __shared__ float sm_m[SWA_WARPS], sm_l[SWA_WARPS];
@@ -150,6 +151,10 @@ __global__ void __launch_bounds__(SWA_WARPS * 32, 6) k_swa_decode(const float* _
     // capped below that (then each CTA takes items blockIdx.x, blockIdx.x + gridDim.x, ...)
     for (int item = blockIdx.x; item < B * H; item += gridDim.x) {
         const int b = item / H, h = item % H;
+        // this sequence's step t: it has consumed pos[b] tokens (clamped to the bound the host
+        // checked, so that a corrupt state cannot address outside the rotary table)
+        const int t = min(max(pos[b] + 1, 1), max_t);
+        const float2* rope_row = rope + (long long)(t - 1) * half;
         const float* row = qkv + (long long)b * 3 * d + h * HD;
         // this warp's share of the ring; its first round of loads is issued before q is formed,
         // so the ring's memory latency overlaps the q / RoPE loads instead of following them
@@ -246,7 +251,8 @@ __global__ void __launch_bounds__(SWA_WARPS * 32, 6) k_swa_decode(const float* _
 template <typename T, int HD>
 __global__ void __launch_bounds__(WARPS * 32) k_xattn_decode(const float* __restrict__ qc,
                                                              const T* __restrict__ Mg, long long plane,
-                                                             int T_alloc, int t, T* __restrict__ o, int B, int H,
+                                                             int T_alloc, int t, const int32_t* __restrict__ pos,
+                                                             T* __restrict__ o, int B, int H,
                                                              int n_splits, int chunk, float* __restrict__ part,
                                                              float qscale) {
     using G = Geom<T, HD>;
@@ -267,8 +273,10 @@ __global__ void __launch_bounds__(WARPS * 32) k_xattn_decode(const float* __rest
         for (int i = 0; i < EPL; ++i) q[i] = qr[i] * qscale;
         const T* K = Mg + (long long)bh * T_alloc * HD;
         const T* V = K + plane;
+        // keys 0 .. tb-1: tb = t for every sequence, or pos[b] + 1 (at most t) per sequence
+        const int tb = pos ? min(max(pos[b] + 1, 1), t) : t;
         int j0 = sp * chunk;
-        int n = max(0, min(t, j0 + chunk) - j0);
+        int n = max(0, min(tb, j0 + chunk) - j0);
         float m = NEG_BIG, l = 0.f, acc[EPL];
 #pragma unroll
         for (int i = 0; i < EPL; ++i) acc[i] = 0.f;
@@ -364,25 +372,25 @@ inline unsigned capped(const Launch& L, unsigned blocks) {
     }
 
 template <typename T>
-cudaError_t launch_swa_decode(Launch L, const float* qkv, const float2* rope_row, T* ring, T* o, int B,
-                              int H, int hd, int W, int t) {
-    RLT_HD_DISPATCH(hd, launch_k(L, k_swa_decode<T, HD>, capped(L, (unsigned)(B * H)), SWA_WARPS * 32, 0, qkv, rope_row,
-                                 ring, o, B, H, W, t, qscale_for(hd)));
+cudaError_t launch_swa_decode(Launch L, const float* qkv, const float2* rope, T* ring, T* o, int B,
+                              int H, int hd, int W, const int32_t* pos, int max_t) {
+    RLT_HD_DISPATCH(hd, launch_k(L, k_swa_decode<T, HD>, capped(L, (unsigned)(B * H)), SWA_WARPS * 32, 0, qkv, rope,
+                                 ring, o, B, H, W, pos, max_t, qscale_for(hd)));
 }
 
 template <typename T>
-static cudaError_t xattn_main(Launch L, const float* qc, const T* Mg, long long plane, int T_alloc, int t, T* o,
-                              int B, int H, int hd, int n_splits, int chunk, float* part) {
+static cudaError_t xattn_main(Launch L, const float* qc, const T* Mg, long long plane, int T_alloc, int t,
+                              const int32_t* pos, T* o, int B, int H, int hd, int n_splits, int chunk, float* part) {
     RLT_HD_DISPATCH(hd, launch_k(L, k_xattn_decode<T, HD>, capped(L, blocks_for((long long)B * H * n_splits)), WARPS * 32, 0,
-                                 qc, Mg, plane, T_alloc, t, o, B, H, n_splits, chunk, part, qscale_for(hd)));
+                                 qc, Mg, plane, T_alloc, t, pos, o, B, H, n_splits, chunk, part, qscale_for(hd)));
 }
 
 template <typename T>
 cudaError_t launch_xattn_decode(Launch L, const float* qc, const T* Mg, long long plane, int T_alloc, int t, T* o,
-                                int B, int H, int hd, int n_splits, float* part) {
+                                int B, int H, int hd, int n_splits, float* part, const int32_t* pos) {
     if (n_splits < 1) n_splits = 1;
     int chunk = (t + n_splits - 1) / n_splits;
-    cudaError_t e = xattn_main<T>(L, qc, Mg, plane, T_alloc, t, o, B, H, hd, n_splits, chunk, part);
+    cudaError_t e = xattn_main<T>(L, qc, Mg, plane, T_alloc, t, pos, o, B, H, hd, n_splits, chunk, part);
     if (e != cudaSuccess || n_splits == 1) return e;
     return launch_k(L, k_attn_combine<T>, (unsigned)(B * H), (unsigned)hd, 0, (const float*)part, n_splits, hd, H, o);
 }
@@ -395,9 +403,9 @@ cudaError_t launch_enc_attention(Launch L, const T* planes, T* o, int B, int Tn,
 
 #define RLT_INST(T)                                                                                    \
     template cudaError_t launch_swa_decode<T>(Launch, const float*, const float2*, T*, T*, int, int,   \
-                                              int, int, int);                                          \
+                                              int, int, const int32_t*, int);                          \
     template cudaError_t launch_xattn_decode<T>(Launch, const float*, const T*, long long, int, int, T*, int, \
-                                                int, int, int, float*);                                \
+                                                int, int, int, float*, const int32_t*);                \
     template cudaError_t launch_enc_attention<T>(Launch, const T*, T*, int, int, int, int);
 RLT_INST(float)
 RLT_INST(bf16)

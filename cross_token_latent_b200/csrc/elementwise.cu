@@ -57,7 +57,7 @@ __global__ void k_embed(const int32_t* __restrict__ tok, int tok_stride, int N, 
 template <typename T>
 __global__ void k_rmsnorm(const float* __restrict__ x, int N, int d, const float* __restrict__ gain,
                           float eps, T* __restrict__ out, int out_ld, int rows_per_seq,
-                          int out_rows_per_seq, T* __restrict__ out2) {
+                          int out_rows_per_seq, T* __restrict__ out2, const int32_t* __restrict__ row_pos) {
     pdl_wait();
     pdl_trigger();
     int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -71,7 +71,8 @@ __global__ void k_rmsnorm(const float* __restrict__ x, int N, int d, const float
     }
     ss = warp_sum(ss);
     float r = 1.0f / sqrtf(ss / d + eps);
-    long long orow = (long long)(warp / rows_per_seq) * out_rows_per_seq + warp % rows_per_seq;
+    long long orow = row_pos ? (long long)warp * out_rows_per_seq + min(max(row_pos[warp], 0), out_rows_per_seq - 1)
+                             : (long long)(warp / rows_per_seq) * out_rows_per_seq + warp % rows_per_seq;
     T* o = out + orow * out_ld;
     T* o2 = out2 ? out2 + (long long)warp * d : nullptr;
     for (int c = lane; c < d / 4; c += 32) {
@@ -87,17 +88,23 @@ __global__ void k_rmsnorm(const float* __restrict__ x, int N, int d, const float
 }
 
 template <typename T>
-__global__ void k_merge_prep(const T* __restrict__ e, int T_alloc, int t, const float* __restrict__ s,
-                             T* __restrict__ A, int B, int d, const StateHeader* sh, uint64_t version,
-                             DevHeader* hdr) {
+__global__ void k_merge_prep(const T* __restrict__ e, int T_alloc, const int32_t* __restrict__ pos,
+                             const float* __restrict__ s, T* __restrict__ A, int B, int d, const StateHeader* sh,
+                             uint64_t version, DevHeader* hdr) {
     pdl_wait();
     pdl_trigger();
     int b = blockIdx.x;
     if (b == 0 && threadIdx.x == 0 && sh) {
-        if (sh->magic != STATE_MAGIC || sh->t != t - 1 || sh->version != version)
-            raise_flag(hdr, ERR_STATE_MISMATCH);
+        if (sh->magic != STATE_MAGIC || sh->version != version) raise_flag(hdr, ERR_STATE_MISMATCH);
     }
-    const T* er = e + ((long long)b * T_alloc + (t - 1)) * d;
+    // e_t of this sequence's step t = pos[b] + 1 is row pos[b]; a position outside the
+    // capacity the host checked means the state was changed behind the library's back
+    int p = pos[b];
+    if (p < 0 || p >= T_alloc) {
+        if (threadIdx.x == 0) raise_flag(hdr, ERR_STATE_MISMATCH);
+        p = min(max(p, 0), T_alloc - 1);
+    }
+    const T* er = e + ((long long)b * T_alloc + p) * d;
     T* ar = A + (long long)b * 2 * d;
     const float* sr = s + (long long)b * d;
     for (int c = threadIdx.x; c < d; c += blockDim.x) {
@@ -108,13 +115,15 @@ __global__ void k_merge_prep(const T* __restrict__ e, int T_alloc, int t, const 
 
 template <typename T>
 __global__ void k_final_norm(const float* __restrict__ x, int B, int d, const float* __restrict__ gain,
-                             float eps, float* __restrict__ s, T* __restrict__ hs, StateHeader* sh, int t) {
+                             float eps, float* __restrict__ s, T* __restrict__ hs, StateHeader* sh, int t,
+                             int32_t* __restrict__ pos) {
     pdl_wait();
     pdl_trigger();
     int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     int lane = threadIdx.x & 31;
     if (warp == 0 && lane == 0 && sh) sh->t = t;
     if (warp >= B) return;
+    if (lane == 0) pos[warp] += 1;                 // one more token consumed
     const float* xr = x + (long long)warp * d;
     float ss = 0.f;
     for (int c = lane; c < d; c += 32) ss += xr[c] * xr[c];
@@ -131,7 +140,7 @@ __global__ void k_final_norm(const float* __restrict__ x, int B, int d, const fl
 __global__ void k_lse_gather(const float* __restrict__ logits, int B, int V, float tau,
                              const int32_t* __restrict__ tok, int tok_stride, float* logp_tok,
                              int lp_stride, float* lse_out, float* logp_full, float* score,
-                             const int32_t* prompt_len, int t, DevHeader* hdr) {
+                             const int32_t* prompt_len, const int32_t* __restrict__ pos, DevHeader* hdr) {
     pdl_wait();
     pdl_trigger();
     int b = blockIdx.x;
@@ -166,7 +175,7 @@ __global__ void k_lse_gather(const float* __restrict__ logits, int B, int V, flo
             if (id < 0 || id >= V) { raise_flag(hdr, ERR_BAD_TOKEN); id = 0; }
             float lp = z[id] / tau - lse;
             if (logp_tok) logp_tok[(long long)b * lp_stride] = lp;
-            if (score && t >= prompt_len[b]) score[b] += lp;
+            if (score && pos[b] >= prompt_len[b]) score[b] += lp;     // pos[b] = this step's t
         }
     }
     if (logp_full) {
@@ -178,7 +187,8 @@ __global__ void k_lse_gather(const float* __restrict__ logits, int B, int V, flo
 // One warp per row: merge the column-tile (max, sum of exp) partials of the fused head.
 __global__ void k_lse_combine(const float2* __restrict__ part, int n_tiles, const float* __restrict__ z_tok, int B,
                               int V, const int32_t* __restrict__ tok, int tok_stride, float* logp_tok, int lp_stride,
-                              float* lse_out, float* score, const int32_t* prompt_len, int t, DevHeader* hdr) {
+                              float* lse_out, float* score, const int32_t* prompt_len,
+                              const int32_t* __restrict__ pos, DevHeader* hdr) {
     pdl_wait();
     pdl_trigger();
     const int b = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
@@ -198,7 +208,7 @@ __global__ void k_lse_combine(const float2* __restrict__ part, int n_tiles, cons
         if (id < 0 || id >= V) raise_flag(hdr, ERR_BAD_TOKEN);     // the head gathered id 0
         const float lp = z_tok[b] - lse;
         if (logp_tok) logp_tok[(long long)b * lp_stride] = lp;
-        if (score && t >= prompt_len[b]) score[b] += lp;
+        if (score && pos[b] >= prompt_len[b]) score[b] += lp;          // pos[b] = this step's t
     }
 }
 
@@ -242,8 +252,8 @@ __global__ void k_enc_qkv_layout(const float* __restrict__ qkv, int B, int Tn, i
 // queries, goes to q_out [B, d] float32.
 template <typename T>
 __global__ void k_enc_cache_write(const float* __restrict__ qkv, int B, int Tn, int H, int hd,
-                                  const float2* __restrict__ rope, int pos0, T* __restrict__ cache_l, int T_max,
-                                  float* __restrict__ q_out) {
+                                  const float2* __restrict__ rope, int pos0, const int32_t* __restrict__ row_pos,
+                                  T* __restrict__ cache_l, int T_max, float* __restrict__ q_out) {
     pdl_wait();
     pdl_trigger();
     const int half = hd / 2, d = H * hd;
@@ -255,7 +265,8 @@ __global__ void k_enc_cache_write(const float* __restrict__ qkv, int B, int Tn, 
         const long long r = i / half;
         const int h = (int)(r % H);
         const long long n = r / H;
-        const int b = (int)(n / Tn), p = pos0 + (int)(n % Tn);
+        const int b = (int)(n / Tn);
+        const int p = row_pos ? min(max(row_pos[b], 0), T_max - 1) : pos0 + (int)(n % Tn);
         const float* row = qkv + n * 3 * d + h * hd;
         const float2 cs = rope[(long long)p * half + f];
         const long long o = (((long long)b * H + h) * T_max + p) * hd;
@@ -275,7 +286,7 @@ __global__ void k_enc_cache_write(const float* __restrict__ qkv, int B, int Tn, 
 
 template <typename T>
 __global__ void k_mem_layout(const float* __restrict__ kv, int B, int Tn, int T_alloc, int H, int hd,
-                             T* __restrict__ Mg) {
+                             T* __restrict__ Mg, const int32_t* __restrict__ row_pos) {
     pdl_wait();
     pdl_trigger();
     int d = H * hd;
@@ -285,20 +296,27 @@ __global__ void k_mem_layout(const float* __restrict__ kv, int B, int Tn, int T_
          i += (long long)gridDim.x * blockDim.x) {
         int c = (int)(i % (2 * d));
         long long n = i / (2 * d);
-        int b = (int)(n / Tn), p = (int)(n % Tn);
+        int b = (int)(n / Tn);
+        int p = row_pos ? min(max(row_pos[b], 0), T_alloc - 1) : (int)(n % Tn);
         int kvsel = c / d, h = (c % d) / hd, x = c % hd;
         Mg[kvsel * plane + (((long long)b * H + h) * T_alloc + p) * hd + x] = from_f<T>(kv[i]);
     }
 }
 
 __global__ void k_state_init(const float* __restrict__ s_star, int B, int d, float* __restrict__ s,
-                             StateHeader* sh, uint64_t version) {
+                             StateHeader* sh, uint64_t version, int32_t* __restrict__ pos, int row) {
     pdl_wait();
     pdl_trigger();
-    long long n = (long long)B * d;
+    // every row, or only row `row` (>= 0) of a batch state
+    const long long n = row >= 0 ? d : (long long)B * d;
+    float* s0 = row >= 0 ? s + (long long)row * d : s;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
          i += (long long)gridDim.x * blockDim.x)
-        s[i] = s_star[i % d];
+        s0[i] = s_star[i % d];
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < (row >= 0 ? 1 : B);
+         i += (long long)gridDim.x * blockDim.x)
+        pos[row >= 0 ? row : i] = 0;
+    if (row >= 0) return;
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         sh->magic = STATE_MAGIC;
         sh->t = 0;
@@ -336,36 +354,36 @@ cudaError_t launch_embed(Launch L, const int32_t* tok, int N, const T* embed, in
 
 template <typename T>
 cudaError_t launch_rmsnorm(Launch L, const float* x, int N, int d, const float* gain, float eps, T* out,
-                           int out_ld, int rows_per_seq, int out_rows_per_seq, T* out2) {
+                           int out_ld, int rows_per_seq, int out_rows_per_seq, T* out2, const int32_t* row_pos) {
     return launch_k(L, k_rmsnorm<T>, cdiv(N, 8), 256, 0, x, N, d, gain, eps, out, out_ld, rows_per_seq,
-                    out_rows_per_seq, out2);
+                    out_rows_per_seq, out2, row_pos);
 }
 
 template <typename T>
-cudaError_t launch_merge_prep(Launch L, const T* e, int T_alloc, int t, const float* s, T* A, int B,
+cudaError_t launch_merge_prep(Launch L, const T* e, int T_alloc, const int32_t* pos, const float* s, T* A, int B,
                               int d, const StateHeader* sh, uint64_t version, DevHeader* hdr) {
-    return launch_k(L, k_merge_prep<T>, B, 256, 0, e, T_alloc, t, s, A, B, d, sh, version, hdr);
+    return launch_k(L, k_merge_prep<T>, B, 256, 0, e, T_alloc, pos, s, A, B, d, sh, version, hdr);
 }
 
 template <typename T>
 cudaError_t launch_final_norm(Launch L, const float* x, int B, int d, const float* gain, float eps,
-                              float* s, T* hs, StateHeader* sh, int t) {
-    return launch_k(L, k_final_norm<T>, cdiv(B, 8), 256, 0, x, B, d, gain, eps, s, hs, sh, t);
+                              float* s, T* hs, StateHeader* sh, int t, int32_t* pos) {
+    return launch_k(L, k_final_norm<T>, cdiv(B, 8), 256, 0, x, B, d, gain, eps, s, hs, sh, t, pos);
 }
 
 cudaError_t launch_lse_gather(Launch L, const float* logits, int B, int V, float tau, const int32_t* tok,
                               int tok_stride, float* logp_tok, int lp_stride, float* lse,
-                              float* logp_full, float* score, const int32_t* prompt_len, int t,
+                              float* logp_full, float* score, const int32_t* prompt_len, const int32_t* pos,
                               DevHeader* hdr) {
     return launch_k(L, k_lse_gather, B, 512, 0, logits, B, V, tau, tok, tok_stride, logp_tok, lp_stride, lse,
-                    logp_full, score, prompt_len, t, hdr);
+                    logp_full, score, prompt_len, pos, hdr);
 }
 
 cudaError_t launch_lse_combine(Launch L, const float2* part, int n_tiles, const float* z_tok, int B, int V,
                                const int32_t* tok, int tok_stride, float* logp_tok, int lp_stride, float* lse,
-                               float* score, const int32_t* prompt_len, int t, DevHeader* hdr) {
+                               float* score, const int32_t* prompt_len, const int32_t* pos, DevHeader* hdr) {
     return launch_k(L, k_lse_combine, cdiv(B, 8), 256, 0, part, n_tiles, z_tok, B, V, tok, tok_stride, logp_tok,
-                    lp_stride, lse, score, prompt_len, t, hdr);
+                    lp_stride, lse, score, prompt_len, pos, hdr);
 }
 
 template <typename T>
@@ -376,21 +394,23 @@ cudaError_t launch_enc_qkv_layout(Launch L, const float* qkv, int B, int Tn, int
 }
 
 template <typename T>
-cudaError_t launch_mem_layout(Launch L, const float* kv, int B, int Tn, int T_alloc, int H, int hd, T* Mg) {
+cudaError_t launch_mem_layout(Launch L, const float* kv, int B, int Tn, int T_alloc, int H, int hd, T* Mg,
+                              const int32_t* row_pos) {
     return launch_k(L, k_mem_layout<T>, grid_for((long long)B * Tn * 2 * H * hd, 256), 256, 0, kv, B, Tn, T_alloc,
-                    H, hd, Mg);
+                    H, hd, Mg, row_pos);
 }
 
 template <typename T>
 cudaError_t launch_enc_cache_write(Launch L, const float* qkv, int B, int Tn, int H, int hd, const float2* rope,
-                                   int pos0, T* cache_l, int T_max, float* q_out) {
+                                   int pos0, const int32_t* row_pos, T* cache_l, int T_max, float* q_out) {
     return launch_k(L, k_enc_cache_write<T>, grid_for((long long)B * Tn * H * (hd / 2), 256), 256, 0, qkv, B, Tn, H,
-                    hd, rope, pos0, cache_l, T_max, q_out);
+                    hd, rope, pos0, row_pos, cache_l, T_max, q_out);
 }
 
 cudaError_t launch_state_init(Launch L, const float* s_star, int B, int d, float* s, StateHeader* sh,
-                              uint64_t version) {
-    return launch_k(L, k_state_init, grid_for((long long)B * d, 256), 256, 0, s_star, B, d, s, sh, version);
+                              uint64_t version, int32_t* pos, int row) {
+    return launch_k(L, k_state_init, grid_for((long long)(row >= 0 ? 1 : B) * d, 256), 256, 0, s_star, B, d, s, sh,
+                    version, pos, row);
 }
 
 #define RLT_INST(T)                                                                                   \
@@ -398,16 +418,17 @@ cudaError_t launch_state_init(Launch L, const float* s_star, int B, int d, float
     template cudaError_t launch_embed<T>(Launch, const int32_t*, int, const T*, int, int, float*,     \
                                          DevHeader*, int);                                            \
     template cudaError_t launch_rmsnorm<T>(Launch, const float*, int, int, const float*, float, T*,   \
-                                           int, int, int, T*);                                        \
-    template cudaError_t launch_merge_prep<T>(Launch, const T*, int, int, const float*, T*, int, int, \
-                                              const StateHeader*, uint64_t, DevHeader*);              \
+                                           int, int, int, T*, const int32_t*);                        \
+    template cudaError_t launch_merge_prep<T>(Launch, const T*, int, const int32_t*, const float*, T*, \
+                                              int, int, const StateHeader*, uint64_t, DevHeader*);    \
     template cudaError_t launch_final_norm<T>(Launch, const float*, int, int, const float*, float,    \
-                                              float*, T*, StateHeader*, int);                         \
+                                              float*, T*, StateHeader*, int, int32_t*);               \
     template cudaError_t launch_enc_qkv_layout<T>(Launch, const float*, int, int, int, int,           \
                                                   const float2*, T*, bool);                           \
-    template cudaError_t launch_mem_layout<T>(Launch, const float*, int, int, int, int, int, T*);       \
+    template cudaError_t launch_mem_layout<T>(Launch, const float*, int, int, int, int, int, T*,      \
+                                              const int32_t*);                                        \
     template cudaError_t launch_enc_cache_write<T>(Launch, const float*, int, int, int, int, const float2*, int, \
-                                                   T*, int, float*);
+                                                   const int32_t*, T*, int, float*);
 RLT_INST(float)
 RLT_INST(bf16)
 #undef RLT_INST

@@ -67,47 +67,56 @@ cudaError_t launch_embed(Launch L, const int32_t* tok, int N, const T* embed, in
 // out[row_map(n), out_col_off + :] = T(RMSNorm(x[n, :]) * gain).  row_map(n) =
 // (n / rows_per_seq) * out_rows_per_seq + n % rows_per_seq; out2 (optional) is a second
 // contiguous T copy with leading dimension d.
+// With row_pos (device, one entry per row; rows_per_seq must be 1) row n lands at
+// n * out_rows_per_seq + row_pos[n] instead.
 template <typename T>
 cudaError_t launch_rmsnorm(Launch L, const float* x, int N, int d, const float* gain, float eps,
-                           T* out, int out_ld, int rows_per_seq, int out_rows_per_seq, T* out2);
-// A[b, :] = [e[b, t-1, :] | T(s[b, :])]; also checks the state header
+                           T* out, int out_ld, int rows_per_seq, int out_rows_per_seq, T* out2,
+                           const int32_t* row_pos = nullptr);
+// A[b, :] = [e[b, pos[b], :] | T(s[b, :])] (the step of sequence b consumes its token at
+// 0-based position pos[b]); also checks the state header and the position's range
 template <typename T>
-cudaError_t launch_merge_prep(Launch L, const T* e, int T_alloc, int t, const float* s, T* A, int B,
+cudaError_t launch_merge_prep(Launch L, const T* e, int T_alloc, const int32_t* pos, const float* s, T* A, int B,
                               int d, const StateHeader* sh, uint64_t version, DevHeader* hdr);
-// s[b, :] = RMSNorm(x[b, :]) * gain (float32) and hs = T(s); sets the state header's t
+// s[b, :] = RMSNorm(x[b, :]) * gain (float32) and hs = T(s); pos[b] += 1; sets the state
+// header's t (the batch's largest position) when sh is given
 template <typename T>
 cudaError_t launch_final_norm(Launch L, const float* x, int B, int d, const float* gain, float eps,
-                              float* s, T* hs, StateHeader* sh, int t);
+                              float* s, T* hs, StateHeader* sh, int t, int32_t* pos);
 // Per row b: z = logits[b, :] / tau, lse = logsumexp(z), gather z[tok] - lse, optional full
-// row, optional score accumulation when t >= P[b].
+// row, optional score accumulation when the step t = pos[b] (positions after the step's
+// advance) is at least P[b].
 cudaError_t launch_lse_gather(Launch L, const float* logits, int B, int V, float tau,
                               const int32_t* tok, int tok_stride, float* logp_tok, int lp_stride,
                               float* lse, float* logp_full, float* score, const int32_t* prompt_len,
-                              int t, DevHeader* hdr);
+                              const int32_t* pos, DevHeader* hdr);
 // Per row b: LSE = log sum_j part.y exp(part.x - max) + max over the n_tiles column-tile
 // partials of the fused head; the gathered log-prob z_tok[b] - LSE, the LSE itself and the
 // score accumulation as in launch_lse_gather (bad token ids latch ERR_BAD_TOKEN).
 cudaError_t launch_lse_combine(Launch L, const float2* part, int n_tiles, const float* z_tok, int B, int V,
                                const int32_t* tok, int tok_stride, float* logp_tok, int lp_stride, float* lse,
-                               float* score, const int32_t* prompt_len, int t, DevHeader* hdr);
+                               float* score, const int32_t* prompt_len, const int32_t* pos, DevHeader* hdr);
 // Encoder q/k/v: qkv float32 [B*T, 3d] -> planes T [3][B][H][T][hd], RoPE on q and k; the v
 // plane is skipped when write_v is false (the tensor-core path writes V transposed instead).
 template <typename T>
 cudaError_t launch_enc_qkv_layout(Launch L, const float* qkv, int B, int Tn, int H, int hd,
                                   const float2* rope, T* planes, bool write_v = true);
-// Memory projection output float32 [B*T, 2d] -> M_g T [2][B][H][T_alloc][hd]
+// Memory projection output float32 [B*T, 2d] -> M_g T [2][B][H][T_alloc][hd]; with row_pos
+// (Tn = 1) sequence b's row lands at position row_pos[b]
 template <typename T>
 cudaError_t launch_mem_layout(Launch L, const float* kv, int B, int Tn, int T_alloc, int H, int hd,
-                              T* Mg);
+                              T* Mg, const int32_t* row_pos = nullptr);
 // Encoder key/value cache of one layer [2][B][H][T_max][hd]: rotated keys and values of the Tn
 // tokens of qkv float32 [B*Tn, 3d] at positions pos0 .. pos0+Tn-1, in the storage type; with
 // q_out (Tn = 1) also the rotated, storage-rounded query as float32 [B, d].
+// With row_pos (device, Tn = 1) sequence b's token is at position row_pos[b] instead.
 template <typename T>
 cudaError_t launch_enc_cache_write(Launch L, const float* qkv, int B, int Tn, int H, int hd, const float2* rope,
-                                   int pos0, T* cache_l, int T_max, float* q_out);
-// H_0: s[b, :] = s_star, header (t=0, version, B)
+                                   int pos0, const int32_t* row_pos, T* cache_l, int T_max, float* q_out);
+// H_0: s[b, :] = s_star, pos[b] = 0, header (t=0, version, B); with row >= 0 only that row's s
+// and position (the header is left alone)
 cudaError_t launch_state_init(Launch L, const float* s_star, int B, int d, float* s, StateHeader* sh,
-                              uint64_t version);
+                              uint64_t version, int32_t* pos, int row = -1);
 
 // ------------------------------------------------------------------ gemm_simt.cu
 // C[M, N] = A[M, K] (leading dim lda) x W[N, K]^T, float32 accumulation, then an epilogue.
@@ -196,18 +205,21 @@ cudaError_t launch_gemm_swap(Launch L, Epi epi, const bf16* A, int lda, const bf
                              const EpiArgs& ea, DevHeader* hdr, int split = 0);
 
 // ------------------------------------------------------------------ attention.cu
-// Decoder sliding-window self-attention for one layer at step t (1-based): RoPE at
-// position t-1 on q/k from qkv [B, 3d]; attends over the min(t-1, W-1) cached entries plus
-// the current token; then stores k_t, v_t into ring slot (t-1) mod (W-1).
+// Decoder sliding-window self-attention for one layer: sequence b is at step t = pos[b] + 1
+// (clamped to 1 .. max_t): RoPE at position t-1 (rows of the rotary table `rope`) on q/k from
+// qkv [B, 3d]; attends over the min(t-1, W-1) cached entries plus the current token; then
+// stores k_t, v_t into ring slot (t-1) mod (W-1).
 template <typename T>
-cudaError_t launch_swa_decode(Launch L, const float* qkv, const float2* rope_row, T* ring, T* o,
-                              int B, int H, int hd, int W, int t);
+cudaError_t launch_swa_decode(Launch L, const float* qkv, const float2* rope, T* ring, T* o,
+                              int B, int H, int hd, int W, const int32_t* pos, int max_t);
 // Decoder cross-attention over M_{<=t} (positions 0..t-1) of one memory group: keys of
-// (b, h) at Mg + (b*H + h)*T_alloc*hd, values `plane` elements further.  Splits the keys of
-// each (b, h) into n_splits chunks when n_splits > 1 (partials in `part`).
+// (b, h) at Mg + (b*H + h)*T_alloc*hd, values `plane` elements further.  With pos (device,
+// [B]) sequence b reads only positions 0..pos[b] (at most t).  Splits the keys of each (b, h)
+// into n_splits chunks of ceil(t / n_splits) when n_splits > 1 (partials in `part`).
 template <typename T>
 cudaError_t launch_xattn_decode(Launch L, const float* qc, const T* Mg, long long plane, int T_alloc, int t,
-                                T* o, int B, int H, int hd, int n_splits, float* part);
+                                T* o, int B, int H, int hd, int n_splits, float* part,
+                                const int32_t* pos = nullptr);
 // Encoder causal self-attention: planes T [3][B][H][T][hd] -> o T [B*T, d]
 template <typename T>
 cudaError_t launch_enc_attention(Launch L, const T* planes, T* o, int B, int Tn, int H, int hd);

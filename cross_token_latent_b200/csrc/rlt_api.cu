@@ -81,10 +81,25 @@ Layout make_layout(const rlt_config& c) {
     return L;
 }
 
+// Host mirror of a registered state: the batch, the model version it was built under and the
+// position (tokens consumed) of every row.  The device copy of the positions lives in the state
+// buffer and is advanced by the step's kernels in the same way.
 struct StateInfo {
-    int B;
-    int64_t t;
-    uint64_t version;
+    int B = 0;
+    uint64_t version = 0;
+    std::vector<int64_t> pos;
+    int64_t t_max() const {
+        int64_t t = 0;
+        for (int64_t p : pos) t = p > t ? p : t;
+        return t;
+    }
+    static StateInfo uniform(int B, int64_t t, uint64_t version) {
+        StateInfo s;
+        s.B = B;
+        s.version = version;
+        s.pos.assign((size_t)B, t);
+        return s;
+    }
 };
 
 // How one canonical weight maps into the arena.
@@ -250,6 +265,12 @@ size_t state_ring_off(const rlt_config& c, int B) { return align_up(ALIGN + (siz
 size_t ring_layer_elems(const rlt_config& c, int B) {
     return (size_t)B * 2 * c.n_heads * (size_t)(c.W - 1) * c.head_dim;
 }
+size_t state_pos_off(const rlt_config& c, int B) {
+    return align_up(state_ring_off(c, B) + (size_t)c.L_D * ring_layer_elems(c, B) * (c.dtype == RLT_BF16 ? 2 : 4));
+}
+int32_t* state_pos(const rlt_config& c, uint8_t* state, int B) {
+    return reinterpret_cast<int32_t*>(state + state_pos_off(c, B));
+}
 
 struct EncWS {
     size_t h, a, act, qkv, planes, att, ews, total;
@@ -338,7 +359,7 @@ rlt_status encode_impl(rlt_model* m, const int32_t* tokens, int B, int Tn, int T
         ea.out_f32 = qkv; ea.ld_out = 3 * d;
         CK(launch_gemm<T>(L, Epi::StoreF32, a, d, m->at<T>(m->lay.wqkv[l]), N, 3 * d, d, ea));
         if (cache)
-            CK(launch_enc_cache_write<T>(L, qkv, B, Tn, H, hd, rope, 0,
+            CK(launch_enc_cache_write<T>(L, qkv, B, Tn, H, hd, rope, 0, nullptr,
                                          cache + (size_t)l * enc_cache_layer_elems(c, B, T_max), T_max, nullptr));
         if (use_tc_attn) {
             bf16* pl = reinterpret_cast<bf16*>(planes);
@@ -396,8 +417,9 @@ AppWS app_ws(const rlt_config& c, int B) {
 // causal attention reads the cached keys/values of positions 0..pos (the new ones written
 // first), and the new encoder output and memory rows go to e[:, pos] and M[..., pos, :].
 template <typename T>
-rlt_status encode_append_impl(rlt_model* m, const int32_t* tok, int tok_stride, int B, int pos, T* cache, int T_max,
-                              T* e, T* M, int T_alloc, uint8_t* ws, cudaStream_t st) {
+rlt_status encode_append_impl(rlt_model* m, const int32_t* tok, int tok_stride, int B, int pos,
+                              const int32_t* positions, T* cache, int T_max, T* e, T* M, int T_alloc, uint8_t* ws,
+                              cudaStream_t st) {
     const rlt_config& c = m->cfg;
     Launch L{st, &m->launches};
     AppWS w = app_ws(c, B);
@@ -421,8 +443,8 @@ rlt_status encode_append_impl(rlt_model* m, const int32_t* tok, int tok_stride, 
         CK(launch_rmsnorm<T>(L, h, B, d, m->at<float>(m->lay.attn_norm[l]), c.rms_eps, a, d, B, B, nullptr));
         ea.out_f32 = qkv; ea.ld_out = 3 * d;
         CK(launch_gemm<T>(L, Epi::StoreF32, a, d, m->at<T>(m->lay.wqkv[l]), B, 3 * d, d, ea));
-        CK(launch_enc_cache_write<T>(L, qkv, B, 1, H, hd, rope, pos, cache_l, T_max, q));
-        CK(launch_xattn_decode<T>(L, q, cache_l, cplane, T_max, pos + 1, att, B, H, hd, splits, part));
+        CK(launch_enc_cache_write<T>(L, qkv, B, 1, H, hd, rope, pos, positions, cache_l, T_max, q));
+        CK(launch_xattn_decode<T>(L, q, cache_l, cplane, T_max, pos + 1, att, B, H, hd, splits, part, positions));
         ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = h; ea.ld_out = d;
         CK(launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.wo[l]), B, d, d, ea));
         CK(launch_rmsnorm<T>(L, h, B, d, m->at<float>(m->lay.ffn_norm[l]), c.rms_eps, a, d, B, B, nullptr));
@@ -431,15 +453,22 @@ rlt_status encode_append_impl(rlt_model* m, const int32_t* tok, int tok_stride, 
         ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = h; ea.ld_out = d;
         CK(launch_gemm<T>(L, Epi::ResidAdd, act, F, m->at<T>(m->lay.wdown[l]), B, d, F, ea));
     }
-    // e[:, pos] = RMSNorm(h) (row b lands at b * T_alloc + pos), plus a contiguous copy for M
-    CK(launch_rmsnorm<T>(L, h, B, d, m->at<float>(m->lay.enc_norm), c.rms_eps, e + (size_t)pos * d, d, 1, T_alloc,
-                         ews));
+    // e[:, pos] = RMSNorm(h) (row b lands at b * T_alloc + pos, or + positions[b]), plus a
+    // contiguous copy for M
+    if (positions)
+        CK(launch_rmsnorm<T>(L, h, B, d, m->at<float>(m->lay.enc_norm), c.rms_eps, e, d, 1, T_alloc, ews, positions));
+    else
+        CK(launch_rmsnorm<T>(L, h, B, d, m->at<float>(m->lay.enc_norm), c.rms_eps, e + (size_t)pos * d, d, 1, T_alloc,
+                             ews));
     const size_t group_elems = (size_t)2 * B * H * (size_t)T_alloc * hd;
     for (int g = 0; g < c.G; ++g) {
         EpiArgs ea; ea.hdr = m->hdr();
         ea.out_f32 = qkv; ea.ld_out = 2 * d;
         CK(launch_gemm<T>(L, Epi::StoreF32, ews, d, m->at<T>(m->lay.mem) + (size_t)g * 2 * d * d, B, 2 * d, d, ea));
-        CK(launch_mem_layout<T>(L, qkv, B, 1, T_alloc, H, hd, M + g * group_elems + (size_t)pos * hd));
+        if (positions)
+            CK(launch_mem_layout<T>(L, qkv, B, 1, T_alloc, H, hd, M + g * group_elems, positions));
+        else
+            CK(launch_mem_layout<T>(L, qkv, B, 1, T_alloc, H, hd, M + g * group_elems + (size_t)pos * hd));
     }
     m->prof.end(p, st);
     return RLT_OK;
@@ -461,7 +490,9 @@ struct StepIO {
 
 // Rows [b0, b0 + Bg) of a step over a batch of B sequences: every row-indexed buffer is offset
 // by b0; `part` is this row group's key-split buffer; `first` says whether this group checks
-// and advances the state header.
+// and advances the state header.  Sequence b takes its own step pos[b] + 1 (the positions
+// live in the state); t is the largest of those steps (it sizes the key splits and bounds
+// every position).
 template <typename T>
 rlt_status step_rows(rlt_model* m, uint8_t* state, int B, int b0, int Bg, const T* e, const T* M, int T_alloc,
                      int t, const StepIO& io, uint8_t* ws, float* part, bool first, Launch L) {
@@ -472,6 +503,7 @@ rlt_status step_rows(rlt_model* m, uint8_t* state, int B, int b0, int Bg, const 
     StateHeader* sh = first ? reinterpret_cast<StateHeader*>(state) : nullptr;
     float* s = reinterpret_cast<float*>(state + state_s_off()) + rb * d;
     T* ring = reinterpret_cast<T*>(state + state_ring_off(c, B)) + rb * 2 * H * (size_t)(c.W - 1) * hd;
+    int32_t* pos = state_pos(c, state, B) + rb;
     float* x = reinterpret_cast<float*>(ws + w.x) + rb * d;
     T* A = reinterpret_cast<T*>(ws + w.A) + rb * 2 * d;
     float* qkv = reinterpret_cast<float*>(ws + w.qkv) + rb * 3 * d;
@@ -479,7 +511,7 @@ rlt_status step_rows(rlt_model* m, uint8_t* state, int B, int b0, int Bg, const 
     float* qc = reinterpret_cast<float*>(ws + w.qc) + rb * d;
     T* act = reinterpret_cast<T*>(ws + w.act) + rb * F;
     float* logits = reinterpret_cast<float*>(ws + w.logits) + rb * c.V;
-    const float2* rope_row = m->at<float2>(m->lay.rope) + (size_t)(t - 1) * (hd / 2);
+    const float2* rope = m->at<float2>(m->lay.rope);
     const size_t group_elems = (size_t)2 * B * H * (size_t)T_alloc * hd;
     const long long plane = (long long)B * H * T_alloc * hd;        // keys -> values of one memory group
     const T* eg = e + rb * T_alloc * d;
@@ -512,7 +544,7 @@ rlt_status step_rows(rlt_model* m, uint8_t* state, int B, int b0, int Bg, const 
     const T* hin = fuse ? xn : A;
 
     // gated merge: x = e_t + sigmoid(W_ge e_t + W_gs s + b_g) * (W_fb s)
-    CKP(RLT_K_MERGE, launch_merge_prep<T>(L, eg, T_alloc, t, s, A, Bg, d, sh, m->version, m->hdr()));
+    CKP(RLT_K_MERGE, launch_merge_prep<T>(L, eg, T_alloc, pos, s, A, Bg, d, sh, m->version, m->hdr()));
     {
         EpiArgs ea; ea.hdr = m->hdr();
         ea.out_f32 = x; ea.ld_out = d; ea.merge_e = A; ea.ld_e = 2 * d; ea.bias = m->at<float>(m->lay.merge_b);
@@ -526,8 +558,8 @@ rlt_status step_rows(rlt_model* m, uint8_t* state, int B, int b0, int Bg, const 
         ea.out_f32 = qkv; ea.ld_out = 3 * d;
         norm_in(ea);
         CKP(RLT_K_QKV, launch_gemm<T>(L, Epi::StoreF32, hin, d, m->at<T>(m->lay.wqkv[l]), Bg, 3 * d, d, ea));
-        CKP(RLT_K_SWA, launch_swa_decode<T>(L, qkv, rope_row, ring + (size_t)l * ring_layer_elems(c, B), att, Bg, H,
-                                            hd, c.W, t));
+        CKP(RLT_K_SWA, launch_swa_decode<T>(L, qkv, rope, ring + (size_t)l * ring_layer_elems(c, B), att, Bg, H,
+                                            hd, c.W, pos, t));
         ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = x; ea.ld_out = d;
         norm_out(ea, m->at<float>(m->lay.xattn_norm[l]));
         CKP(RLT_K_O, launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.wo[l]), Bg, d, d, ea));
@@ -537,7 +569,7 @@ rlt_status step_rows(rlt_model* m, uint8_t* state, int B, int b0, int Bg, const 
         norm_in(ea);
         CKP(RLT_K_QC, launch_gemm<T>(L, Epi::StoreF32, hin, d, m->at<T>(m->lay.wqc[l]), Bg, d, d, ea));
         const T* Mg = Mrows + (c.G == 1 ? 0 : (size_t)l * group_elems);
-        CKP(RLT_K_XATTN, launch_xattn_decode<T>(L, qc, Mg, plane, T_alloc, t, att, Bg, H, hd, splits, part));
+        CKP(RLT_K_XATTN, launch_xattn_decode<T>(L, qc, Mg, plane, T_alloc, t, att, Bg, H, hd, splits, part, pos));
         ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = x; ea.ld_out = d;
         norm_out(ea, m->at<float>(m->lay.ffn_norm[l]));
         CKP(RLT_K_OC, launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.woc[l]), Bg, d, d, ea));
@@ -551,7 +583,7 @@ rlt_status step_rows(rlt_model* m, uint8_t* state, int B, int b0, int Bg, const 
         CKP(RLT_K_FFN_DOWN, launch_gemm<T>(L, Epi::ResidAdd, act, F, m->at<T>(m->lay.wdown[l]), Bg, d, F, ea));
     }
     // split: s_t = RMSNorm(x) becomes the state; the same s_t feeds the head
-    CKP(RLT_K_FINAL, launch_final_norm<T>(L, x, Bg, d, m->at<float>(m->lay.dec_norm), c.rms_eps, s, A, sh, t));
+    CKP(RLT_K_FINAL, launch_final_norm<T>(L, x, Bg, d, m->at<float>(m->lay.dec_norm), c.rms_eps, s, A, sh, t, pos));
     const int32_t* tok = io.tok ? io.tok + rb * io.tok_stride : nullptr;
     float* lp_tok = io.logp_tok ? io.logp_tok + rb * io.lp_stride : nullptr;
     float* lse = io.lse ? io.lse + rb : nullptr;
@@ -570,13 +602,13 @@ rlt_status step_rows(rlt_model* m, uint8_t* state, int B, int b0, int Bg, const 
                                            reinterpret_cast<const bf16*>(m->at<T>(m->lay.unembed)), Bg, c.V, d, ea,
                                            m->hdr(), &n_tiles));
         CKP(RLT_K_LSE, launch_lse_combine(L, ea.lse_part, n_tiles, ea.z_tok, Bg, c.V, tok, io.tok_stride, lp_tok,
-                                          io.lp_stride, lse, score, plen, t, m->hdr()));
+                                          io.lp_stride, lse, score, plen, pos, m->hdr()));
     } else if (io.head) {
         EpiArgs ea; ea.hdr = m->hdr();
         ea.out_f32 = logits; ea.ld_out = c.V;
         CKP(RLT_K_HEAD, launch_gemm<T>(L, Epi::StoreF32, A, d, m->at<T>(m->lay.unembed), Bg, c.V, d, ea));
         CKP(RLT_K_LSE, launch_lse_gather(L, logits, Bg, c.V, io.tau, tok, io.tok_stride, lp_tok, io.lp_stride, lse,
-                                         io.logp_full ? io.logp_full + rb * c.V : nullptr, score, plen, t,
+                                         io.logp_full ? io.logp_full + rb * c.V : nullptr, score, plen, pos,
                                          m->hdr()));
     }
     return RLT_OK;
@@ -623,7 +655,7 @@ rlt_status state_init_impl(rlt_model* m, uint8_t* state, int B, cudaStream_t st)
     Launch L{st, &m->launches};
     CK(launch_state_init(L, m->at<float>(m->lay.s_star), B, m->cfg.d,
                          reinterpret_cast<float*>(state + state_s_off()),
-                         reinterpret_cast<StateHeader*>(state), m->version));
+                         reinterpret_cast<StateHeader*>(state), m->version, state_pos(m->cfg, state, B)));
     return RLT_OK;
 }
 
@@ -756,7 +788,7 @@ rlt_status rlt_encode(rlt_model* m, const int32_t* tokens, int B, int T, int T_a
 size_t rlt_state_bytes(const rlt_model* m, int B) {
     if (!m || B < 1) return 0;
     const rlt_config& c = m->cfg;
-    return align_up(state_ring_off(c, B) + (size_t)c.L_D * ring_layer_elems(c, B) * m->lay.esz);
+    return state_pos_off(c, B) + align_up((size_t)B * 4);
 }
 
 rlt_status rlt_state_init(rlt_model* m, void* state, int B, void* stream) {
@@ -766,7 +798,7 @@ rlt_status rlt_state_init(rlt_model* m, void* state, int B, void* stream) {
         ? state_init_impl<bf16>(m, (uint8_t*)state, B, (cudaStream_t)stream)
         : state_init_impl<float>(m, (uint8_t*)state, B, (cudaStream_t)stream);
     if (s != RLT_OK) return s;
-    m->states[state] = StateInfo{B, 0, m->version};
+    m->states[state] = StateInfo::uniform(B, 0, m->version);
     return RLT_OK;
 }
 
@@ -785,13 +817,176 @@ rlt_status rlt_state_position(const rlt_model* m, const void* state, int64_t* t)
     if (!m || !state || !t) return RLT_EINVAL;
     auto it = m->states.find(state);
     if (it == m->states.end()) return RLT_ESTATE;
-    *t = it->second.t;
+    *t = it->second.t_max();
     return RLT_OK;
 }
 
 rlt_status rlt_state_release(rlt_model* m, const void* state) {
     if (!m || !state) return RLT_EINVAL;
     return m->states.erase(state) ? RLT_OK : RLT_ESTATE;
+}
+
+rlt_status rlt_state_positions(const rlt_model* m, const void* state, int64_t* positions) {
+    if (!m || !state || !positions) return RLT_EINVAL;
+    auto it = m->states.find(state);
+    if (it == m->states.end()) return RLT_ESTATE;
+    for (size_t b = 0; b < it->second.pos.size(); ++b) positions[b] = it->second.pos[b];
+    return RLT_OK;
+}
+
+size_t rlt_state_positions_offset(const rlt_model* m, int B) {
+    if (!m || B < 1) return 0;
+    return state_pos_off(m->cfg, B);
+}
+
+rlt_status rlt_state_reset_row(rlt_model* m, void* state, int row, void* stream) {
+    if (!m || !state) return RLT_EINVAL;
+    auto it = m->states.find(state);
+    if (it == m->states.end()) return RLT_ESTATE;
+    if (it->second.version != m->version) return RLT_ESTALE;
+    const int B = it->second.B;
+    if (row < 0 || row >= B) return RLT_EINVAL;
+    Launch L = m->launch(stream);
+    uint8_t* st = reinterpret_cast<uint8_t*>(state);
+    CK(launch_state_init(L, m->at<float>(m->lay.s_star), B, m->cfg.d, reinterpret_cast<float*>(st + state_s_off()),
+                         reinterpret_cast<StateHeader*>(st), m->version, state_pos(m->cfg, st, B), row));
+    it->second.pos[(size_t)row] = 0;
+    return RLT_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- sequence snapshots
+namespace {
+
+constexpr uint64_t SNAP_MAGIC = 0x31504e53544c52ull;   // "RLTSNP1"
+
+struct SnapHeader {            // first 256 bytes of a sequence snapshot
+    uint64_t magic;
+    uint64_t version;          // model version the sequence was built under
+    int64_t t;                 // tokens consumed
+    int32_t d, n_heads, head_dim, L_E, L_D, W, G, V, dtype, has_enc;
+    uint8_t pad[256 - 24 - 40];
+};
+static_assert(sizeof(SnapHeader) == 256, "snapshot header size");
+
+struct SnapLayout {
+    size_t s, ring, mem, enc, total;
+};
+SnapLayout snap_layout(const rlt_config& c, int64_t t) {
+    const size_t e = c.dtype == RLT_BF16 ? 2 : 4, H = c.n_heads, hd = c.head_dim;
+    SnapLayout L;
+    size_t off = ALIGN;
+    auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes); return o; };
+    L.s = take((size_t)c.d * 4);
+    L.ring = take((size_t)c.L_D * 2 * H * (size_t)(c.W - 1) * hd * e);
+    L.mem = take((size_t)c.G * 2 * H * (size_t)t * hd * e);
+    L.enc = take((size_t)c.L_E * 2 * H * (size_t)t * hd * e);
+    L.total = off;
+    return L;
+}
+
+// Copy sequence `row`'s blocks between a batch buffer laid out [n_outer][B][H][cap][hd] and a
+// snapshot laid out [n_outer][H][t][hd] (to_snap: batch -> snapshot).
+cudaError_t copy_rows(uint8_t* snap, uint8_t* batch, int n_outer, int B, int row, int H, int cap, int64_t t, int hd,
+                      size_t esz, bool to_snap, cudaStream_t st) {
+    if (t <= 0) return cudaSuccess;
+    const size_t width = (size_t)t * hd * esz, bpitch = (size_t)cap * hd * esz;
+    for (int o = 0; o < n_outer; ++o) {
+        uint8_t* sp = snap + (size_t)o * H * width;
+        uint8_t* bp = batch + (((size_t)o * B + row) * H) * bpitch;
+        cudaError_t e = to_snap ? cudaMemcpy2DAsync(sp, width, bp, bpitch, width, H, cudaMemcpyDeviceToDevice, st)
+                                : cudaMemcpy2DAsync(bp, bpitch, sp, width, width, H, cudaMemcpyDeviceToDevice, st);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t rlt_snapshot_bytes(const rlt_model* m, int T) {
+    if (!m || T < 0) return 0;
+    return snap_layout(m->cfg, T).total;
+}
+
+rlt_status rlt_snapshot_save(rlt_model* m, const void* state, int row, const void* enc_cache, int T_max,
+                             const void* M, int T_alloc, void* dst, size_t dst_bytes, void* stream) {
+    if (!m || !state || !M || !dst || !aligned(dst)) return RLT_EINVAL;
+    auto it = m->states.find(state);
+    if (it == m->states.end()) return RLT_ESTATE;
+    const StateInfo& info = it->second;
+    if (info.version != m->version) return RLT_ESTALE;
+    const int B = info.B;
+    if (row < 0 || row >= B) return RLT_EINVAL;
+    const rlt_config& c = m->cfg;
+    const int64_t t = info.pos[(size_t)row];
+    if (t > T_alloc || (enc_cache && t > T_max)) return RLT_EINVAL;
+    const SnapLayout S = snap_layout(c, t);
+    if (dst_bytes < S.total) return RLT_EINVAL;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* out = reinterpret_cast<uint8_t*>(dst);
+    const uint8_t* sb = reinterpret_cast<const uint8_t*>(state);
+    const size_t esz = m->lay.esz, H = c.n_heads, hd = c.head_dim;
+    SnapHeader h;
+    std::memset(&h, 0, sizeof(h));
+    h.magic = SNAP_MAGIC; h.version = m->version; h.t = t;
+    h.d = c.d; h.n_heads = c.n_heads; h.head_dim = c.head_dim; h.L_E = c.L_E; h.L_D = c.L_D; h.W = c.W; h.G = c.G;
+    h.V = c.V; h.dtype = c.dtype; h.has_enc = enc_cache ? 1 : 0;
+    CK(cudaMemcpyAsync(out, &h, sizeof(h), cudaMemcpyHostToDevice, st));
+    CK(cudaMemcpyAsync(out + S.s, sb + state_s_off() + (size_t)row * c.d * 4, (size_t)c.d * 4,
+                       cudaMemcpyDeviceToDevice, st));
+    const size_t ring_row = 2 * H * (size_t)(c.W - 1) * hd * esz;
+    if (ring_row > 0)
+        CK(cudaMemcpy2DAsync(out + S.ring, ring_row, sb + state_ring_off(c, B) + (size_t)row * ring_row, B * ring_row,
+                             ring_row, c.L_D, cudaMemcpyDeviceToDevice, st));
+    CK(copy_rows(out + S.mem, (uint8_t*)M, 2 * c.G, B, row, c.n_heads, T_alloc, t, hd, esz, true, st));
+    if (enc_cache)
+        CK(copy_rows(out + S.enc, (uint8_t*)enc_cache, 2 * c.L_E, B, row, c.n_heads, T_max, t, hd, esz, true, st));
+    return RLT_OK;
+}
+
+rlt_status rlt_snapshot_load(rlt_model* m, const void* src, void* state, int row, void* enc_cache, int T_max,
+                             void* M, int T_alloc, void* stream) {
+    if (!m || !src || !state || !M || !aligned(src)) return RLT_EINVAL;
+    auto it = m->states.find(state);
+    if (it == m->states.end()) return RLT_ESTATE;
+    StateInfo& info = it->second;
+    if (info.version != m->version) return RLT_ESTALE;
+    const int B = info.B;
+    if (row < 0 || row >= B) return RLT_EINVAL;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    SnapHeader h;
+    CK(cudaMemcpyAsync(&h, src, sizeof(h), cudaMemcpyDeviceToHost, st));
+    CK(cudaStreamSynchronize(st));
+    const rlt_config& c = m->cfg;
+    if (h.magic != SNAP_MAGIC || h.d != c.d || h.n_heads != c.n_heads || h.head_dim != c.head_dim ||
+        h.L_E != c.L_E || h.L_D != c.L_D || h.W != c.W || h.G != c.G || h.V != c.V || h.dtype != c.dtype)
+        return RLT_EINVAL;
+    if (h.version != m->version) return RLT_ESTALE;      // built under weights since replaced
+    const int64_t t = h.t;
+    if (t < 0 || t >= T_alloc || T_alloc > c.max_pos || (enc_cache && (!h.has_enc || t >= T_max))) return RLT_EINVAL;
+    const SnapLayout S = snap_layout(c, t);
+    const uint8_t* in = reinterpret_cast<const uint8_t*>(src);
+    uint8_t* sb = reinterpret_cast<uint8_t*>(state);
+    const size_t esz = m->lay.esz, H = c.n_heads, hd = c.head_dim;
+    CK(cudaMemcpyAsync(sb + state_s_off() + (size_t)row * c.d * 4, in + S.s, (size_t)c.d * 4,
+                       cudaMemcpyDeviceToDevice, st));
+    const size_t ring_row = 2 * H * (size_t)(c.W - 1) * hd * esz;
+    if (ring_row > 0)
+        CK(cudaMemcpy2DAsync(sb + state_ring_off(c, B) + (size_t)row * ring_row, B * ring_row, in + S.ring, ring_row,
+                             ring_row, c.L_D, cudaMemcpyDeviceToDevice, st));
+    CK(copy_rows(const_cast<uint8_t*>(in) + S.mem, (uint8_t*)M, 2 * c.G, B, row, c.n_heads, T_alloc, t, hd, esz,
+                 false, st));
+    if (enc_cache)
+        CK(copy_rows(const_cast<uint8_t*>(in) + S.enc, (uint8_t*)enc_cache, 2 * c.L_E, B, row, c.n_heads, T_max, t, hd,
+                     esz, false, st));
+    const int32_t p32 = (int32_t)t;
+    CK(cudaMemcpyAsync(state_pos(c, sb, B) + row, &p32, 4, cudaMemcpyHostToDevice, st));
+    CK(cudaStreamSynchronize(st));                         // p32 is a host local
+    info.pos[(size_t)row] = t;
+    return RLT_OK;
 }
 
 size_t rlt_decode_workspace_bytes(const rlt_model* m, int B) {
@@ -806,7 +1001,7 @@ rlt_status rlt_decode_step(rlt_model* m, void* state, int B, const void* e, cons
     auto it = m->states.find(state);
     if (it == m->states.end() || it->second.B != B) return RLT_ESTATE;
     if (it->second.version != m->version) return RLT_ESTALE;
-    int64_t t = it->second.t + 1;
+    int64_t t = it->second.t_max() + 1;           // the furthest sequence's step
     if (t > T_alloc || T_alloc > m->cfg.max_pos) return RLT_EINVAL;
     if (!aligned(e) || !aligned(M) || !aligned(ws)) return RLT_EINVAL;
     if (ws_bytes < dec_ws(m->cfg, B).total) return RLT_EINVAL;
@@ -823,7 +1018,8 @@ rlt_status rlt_decode_step(rlt_model* m, void* state, int B, const void* e, cons
                           (uint8_t*)ws, st)
         : step_impl<float>(m, (uint8_t*)state, B, (const float*)e, (const float*)M, T_alloc, (int)t, io,
                            (uint8_t*)ws, st);
-    if (s == RLT_OK) it->second.t = t;
+    if (s == RLT_OK)
+        for (int64_t& p : it->second.pos) p += 1;
     return s;
 }
 
@@ -855,20 +1051,22 @@ size_t rlt_encode_append_workspace_bytes(const rlt_model* m, int B) {
     return app_ws(m->cfg, B).total;
 }
 
-rlt_status rlt_encode_append(rlt_model* m, const int32_t* tokens, int tok_stride, int B, int pos, void* enc_cache,
-                             int T_max, void* e, void* M, int T_alloc, void* ws, size_t ws_bytes, void* stream) {
+rlt_status rlt_encode_append(rlt_model* m, const int32_t* tokens, int tok_stride, int B, int pos,
+                             const int32_t* positions, void* enc_cache, int T_max, void* e, void* M, int T_alloc,
+                             void* ws, size_t ws_bytes, void* stream) {
     if (!m || !tokens || !enc_cache || !e || !M || !ws || B < 1 || tok_stride < 1 || pos < 0) return RLT_EINVAL;
     if (pos >= T_max || pos >= T_alloc || T_max > m->cfg.max_pos || T_alloc > m->cfg.max_pos) return RLT_EINVAL;
     if (m->version == 0) return RLT_EINVAL;
     if (!aligned(e) || !aligned(M) || !aligned(ws) || !aligned(enc_cache) || !aligned(tokens, 4)) return RLT_EINVAL;
+    if (positions && !aligned(positions, 4)) return RLT_EINVAL;
     if (ws_bytes < app_ws(m->cfg, B).total) return RLT_EINVAL;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* w = reinterpret_cast<uint8_t*>(ws);
     return m->cfg.dtype == RLT_BF16
-        ? encode_append_impl<bf16>(m, tokens, tok_stride, B, pos, (bf16*)enc_cache, T_max, (bf16*)e, (bf16*)M,
-                                   T_alloc, w, st)
-        : encode_append_impl<float>(m, tokens, tok_stride, B, pos, (float*)enc_cache, T_max, (float*)e, (float*)M,
-                                    T_alloc, w, st);
+        ? encode_append_impl<bf16>(m, tokens, tok_stride, B, pos, positions, (bf16*)enc_cache, T_max, (bf16*)e,
+                                   (bf16*)M, T_alloc, w, st)
+        : encode_append_impl<float>(m, tokens, tok_stride, B, pos, positions, (float*)enc_cache, T_max, (float*)e,
+                                    (float*)M, T_alloc, w, st);
 }
 
 rlt_status rlt_sample(rlt_model* m, const float* logp, int B, const float* u, int top_k, float top_p,
@@ -983,7 +1181,7 @@ rlt_status rlt_replay(rlt_model* m, const int32_t* tokens, int B, int T, const i
                : step_impl<float>(m, state, B, (const float*)e, (const float*)M, T, t, io, scratch, st);
         if (s != RLT_OK) return s;
     }
-    if (final_state) m->states[final_state] = StateInfo{B, T, m->version};
+    if (final_state) m->states[final_state] = StateInfo::uniform(B, T, m->version);
     return RLT_OK;
 }
 

@@ -54,11 +54,22 @@ _EXPORTS = {
                                           ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "rlt_encode_append_workspace_bytes": (ctypes.c_size_t, [ctypes.c_void_p, ctypes.c_int]),
     "rlt_encode_append": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                         ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
-                                         ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
+                                         ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t,
+                                         ctypes.c_void_p]),
     "rlt_sample": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int,
                                   ctypes.c_float, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]),
     "rlt_state_bytes": (ctypes.c_size_t, [ctypes.c_void_p, ctypes.c_int]),
+    "rlt_state_positions_offset": (ctypes.c_size_t, [ctypes.c_void_p, ctypes.c_int]),
+    "rlt_state_positions": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(ctypes.c_int64)]),
+    "rlt_state_reset_row": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]),
+    "rlt_snapshot_bytes": (ctypes.c_size_t, [ctypes.c_void_p, ctypes.c_int]),
+    "rlt_snapshot_save": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int,
+                                         ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t,
+                                         ctypes.c_void_p]),
+    "rlt_snapshot_load": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                         ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int,
+                                         ctypes.c_void_p]),
     "rlt_state_init": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]),
     "rlt_state_copy": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "rlt_state_position": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(ctypes.c_int64)]),
@@ -154,6 +165,20 @@ class RLTState:
         """View of s_t [B, d] float32 inside the state buffer."""
         d = self.model.cfg.d
         return self.buf[256:256 + self.B * d * 4].view(torch.float32).view(self.B, d)
+
+    def positions(self) -> list[int]:
+        """Tokens consumed by every sequence (host registry)."""
+        out = (ctypes.c_int64 * self.B)()
+        _check(lib().rlt_state_positions(self.model.handle, _ptr(self.buf), out), "rlt_state_positions")
+        return list(out)
+
+    def positions_device(self) -> torch.Tensor:
+        """View of the state's int32 [B] device positions (what rlt_encode_append takes)."""
+        off = lib().rlt_state_positions_offset(self.model.handle, self.B)
+        return self.buf[off:off + 4 * self.B].view(torch.int32)
+
+    def reset_row(self, row: int) -> None:
+        _check(lib().rlt_state_reset_row(self.model.handle, _ptr(self.buf), int(row), _stream()), "rlt_state_reset_row")
 
     def copy(self) -> "RLTState":
         other = torch.empty_like(self.buf)
@@ -273,15 +298,33 @@ class RLTModel:
         return e, M, cache
 
     def encode_append(self, tokens: torch.Tensor, pos: int, cache: torch.Tensor, T_max: int, e: torch.Tensor,
-                      M: torch.Tensor) -> None:
+                      M: torch.Tensor, positions: torch.Tensor | None = None) -> None:
         """rlt_encode_append: tokens is an int32 device vector [B] or a column view of a [B, T]
-        matrix (its stride is passed through); the token at position pos is encoded."""
+        matrix (its stride is passed through); the token at position pos is encoded, or with
+        `positions` (int32 device [B], e.g. RLTState.positions_device()) sequence b's token at
+        positions[b] <= pos."""
         B = tokens.shape[0]
         stride = tokens.stride(0)
         nb = lib().rlt_encode_append_workspace_bytes(self.handle, B)
         ws = self._workspace(("app", B), nb)
-        _check(lib().rlt_encode_append(self.handle, _ptr(tokens), stride, B, int(pos), _ptr(cache), int(T_max), _ptr(e),
-                                       _ptr(M), e.shape[1], _ptr(ws), ws.numel(), _stream()), "rlt_encode_append")
+        _check(lib().rlt_encode_append(self.handle, _ptr(tokens), stride, B, int(pos), _ptr(positions), _ptr(cache),
+                                       int(T_max), _ptr(e), _ptr(M), e.shape[1], _ptr(ws), ws.numel(), _stream()),
+               "rlt_encode_append")
+
+    # ---------------------------------------------------------------- sequence snapshots
+    def snapshot_save(self, state: "RLTState", row: int, M: torch.Tensor, cache: torch.Tensor | None = None,
+                      T_max: int = 0) -> torch.Tensor:
+        """rlt_snapshot_save of sequence `row` into a new device buffer."""
+        t = state.positions()[row]
+        buf = torch.empty(lib().rlt_snapshot_bytes(self.handle, t), dtype=torch.uint8, device=self.device)
+        _check(lib().rlt_snapshot_save(self.handle, _ptr(state.buf), int(row), _ptr(cache), int(T_max), _ptr(M),
+                                       M.shape[4], _ptr(buf), buf.numel(), _stream()), "rlt_snapshot_save")
+        return buf
+
+    def snapshot_load(self, snap: torch.Tensor, state: "RLTState", row: int, M: torch.Tensor,
+                      cache: torch.Tensor | None = None, T_max: int = 0) -> None:
+        _check(lib().rlt_snapshot_load(self.handle, _ptr(snap), _ptr(state.buf), int(row), _ptr(cache), int(T_max),
+                                       _ptr(M), M.shape[4], _stream()), "rlt_snapshot_load")
 
     def sample(self, logp: torch.Tensor, u: torch.Tensor, top_k: int = 0, top_p: float = 1.0,
                out: torch.Tensor | None = None, behaviour_logp: torch.Tensor | None = None) -> torch.Tensor:

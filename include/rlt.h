@@ -155,11 +155,16 @@ size_t rlt_encode_append_workspace_bytes(const rlt_model* m, int B);
  * token-parallel encoding of the whole prefix (up to summation order).
  *   tokens      device int32, token of sequence b at tokens[b * tok_stride] (a column of a
  *               [B, T] token matrix has tok_stride T)
+ *   positions   device int32 [B] or NULL: sequence b's token is at position positions[b]
+ *               (each at most pos, which then only bounds them); a decoder state's own
+ *               position array (rlt_state_positions_offset) gives every sequence the position
+ *               its next decoder step reads
  *   enc_cache   the cache of capacity T_max; e, M with row capacity T_alloc, as rlt_encode
  * Requires pos < T_max <= max_pos and pos < T_alloc <= max_pos.  Out-of-range ids latch
  * RLT_EDEVICE.  Errors: RLT_EINVAL, RLT_ECUDA. */
-rlt_status rlt_encode_append(rlt_model* m, const int32_t* tokens, int tok_stride, int B, int pos, void* enc_cache,
-                             int T_max, void* e, void* M, int T_alloc, void* ws, size_t ws_bytes, void* stream);
+rlt_status rlt_encode_append(rlt_model* m, const int32_t* tokens, int tok_stride, int B, int pos,
+                             const int32_t* positions, void* enc_cache, int T_max, void* e, void* M, int T_alloc,
+                             void* ws, size_t ws_bytes, void* stream);
 
 /* Draw the next token of each sequence (news summary, model-RL co-design principle: the
  * behaviour log-probability is taken under the distribution actually sampled from).
@@ -183,9 +188,13 @@ rlt_status rlt_sample(rlt_model* m, const float* logp, int B, const float* u, in
 
 /* ---------------------------------------------------------------- decoder state */
 
-/* Bytes of one decoder state H for B sequences: a 256-byte header, s [B, d] float32 and
- * the SWA ring cache [L_D, B, 2, n_heads, W-1, head_dim] (model dtype). */
+/* Bytes of one decoder state H for B sequences: a 256-byte header, s [B, d] float32, the SWA
+ * ring cache [L_D, B, 2, n_heads, W-1, head_dim] (model dtype) and the positions int32 [B]
+ * (tokens each sequence has consumed), each part 256-byte aligned. */
 size_t rlt_state_bytes(const rlt_model* m, int B);
+
+/* Byte offset of the positions int32 [B] inside a state buffer of B sequences. */
+size_t rlt_state_positions_offset(const rlt_model* m, int B);
 
 /* H_0 = (s*, empty cache) at position t = 0 for B sequences (news summary,
  * decoder-state paragraph: initialisation runs once before BOS with the learned start
@@ -197,11 +206,49 @@ rlt_status rlt_state_init(rlt_model* m, void* state, int B, void* stream);
  * and register the copy at the same position and version. */
 rlt_status rlt_state_copy(rlt_model* m, void* dst, const void* src, void* stream);
 
-/* Position t (tokens consumed) of a registered state, from the host-side registry. */
+/* Position t (tokens consumed) of a registered state, from the host-side registry: the
+ * largest over its sequences. */
 rlt_status rlt_state_position(const rlt_model* m, const void* state, int64_t* t);
+
+/* Position of every sequence of a registered state (host int64 [B]).  Sequences advance
+ * together, one token per rlt_decode_step, but need not stand at the same position: rows are
+ * reset (rlt_state_reset_row) or loaded from snapshots (rlt_snapshot_load) one at a time. */
+rlt_status rlt_state_positions(const rlt_model* m, const void* state, int64_t* positions);
+
+/* Start row `row` of a registered batch state afresh: H_0 = (s*, empty cache) at position 0;
+ * the other rows are untouched.  Errors: RLT_EINVAL, RLT_ESTATE, RLT_ESTALE, RLT_ECUDA. */
+rlt_status rlt_state_reset_row(rlt_model* m, void* state, int row, void* stream);
 
 /* Forget a state (it may then be freed by the caller). */
 rlt_status rlt_state_release(rlt_model* m, const void* state);
+
+/* ---------------------------------------------------------------- sequence snapshots */
+
+/* Prefix snapshot of one sequence for multi-turn serving (news summary, multi-turn paragraph:
+ * a conversation continues from its recurrent state, its encoder memory and its position, and
+ * a weight update invalidates it).  A snapshot of a sequence at position t holds a 256-byte
+ * header (position, window, model shape and version), s_t, its SWA ring of every layer,
+ * M_{<=t} of every memory group and, when saved with one, its encoder key/value cache of
+ * positions 0..t-1.  Bytes of a snapshot of a sequence at position T: */
+size_t rlt_snapshot_bytes(const rlt_model* m, int T);
+
+/* Save row `row` of a registered state (at the row's position t <= T_alloc, and t <= T_max
+ * with an encoder cache) into the caller's device buffer dst (at least rlt_snapshot_bytes(m, t)
+ * bytes, 256-byte aligned).  M (row capacity T_alloc) and enc_cache (capacity T_max, or NULL)
+ * are the batch buffers the state's sequences use.  Errors: RLT_EINVAL, RLT_ESTATE,
+ * RLT_ESTALE, RLT_ECUDA. */
+rlt_status rlt_snapshot_save(rlt_model* m, const void* state, int row, const void* enc_cache, int T_max,
+                             const void* M, int T_alloc, void* dst, size_t dst_bytes, void* stream);
+
+/* Load a snapshot into row `row` of a registered batch state (and of M / enc_cache): the row
+ * then stands at the snapshot's position t, the other rows are untouched.  Reads the snapshot
+ * header on the host, so it synchronises `stream`.  Before the row's next decoder step, encode
+ * its next token at position t (rlt_encode_append with the state's positions).  Requires
+ * t < T_alloc, t < T_max with an encoder cache (which the snapshot must hold), and the model's
+ * shape.  Errors: RLT_ESTALE (the snapshot was taken under weights since replaced), RLT_EINVAL,
+ * RLT_ESTATE, RLT_ECUDA. */
+rlt_status rlt_snapshot_load(rlt_model* m, const void* src, void* state, int row, void* enc_cache, int T_max,
+                             void* M, int T_alloc, void* stream);
 
 /* ---------------------------------------------------------------- one decoder step */
 
@@ -220,8 +267,9 @@ size_t rlt_decode_workspace_bytes(const rlt_model* m, int B);
  *   lse        device float [B] or NULL: log-sum-exp of W_U s_t / tau
  *   logp_full  device float [B, V] or NULL: the full log-probability row
  *   ws         workspace of at least rlt_decode_workspace_bytes(m, B) bytes
- * The step reads its position from the registry; t = position + 1 must satisfy
- * t <= T_alloc <= max_pos.  Errors: RLT_ESTATE (unknown state or B mismatch),
+ * Every sequence b takes its own step t_b = (its position) + 1, reading e at position t_b - 1
+ * and M at positions 0..t_b-1; the largest t_b must satisfy t_b <= T_alloc <= max_pos.
+ * Errors: RLT_ESTATE (unknown state or B mismatch),
  * RLT_ESTALE (state older than the current weights), RLT_EINVAL, RLT_ECUDA. */
 rlt_status rlt_decode_step(rlt_model* m, void* state, int B, const void* e, const void* M,
                            int T_alloc, const int32_t* next_tok, float tau, float* logp_tok,

@@ -128,28 +128,24 @@ def sample_token(logp: np.ndarray, u: float, top_k: int = 0, top_p: float = 1.0)
     lp = np.asarray(logp, np.float64)
     p = np.exp(lp)
     V = p.shape[0]
+    # tokens in decreasing probability; for every token, how many and how much probability
+    # mass lie strictly above it (a sort as a library step, then prefix sums)
+    desc = np.sort(p)[::-1]
+    n_above = np.searchsorted(-desc, -p, side="left")          # count of values > p_i
     keep = np.ones(V, bool)
     if top_k > 0:
-        for i in range(V):
-            keep[i] = np.count_nonzero(p > p[i]) < top_k
+        keep = n_above < top_k
     if top_p < 1.0:
         z1 = p[keep].sum()
-        keep_p = np.zeros(V, bool)
-        for i in range(V):
-            if keep[i]:
-                keep_p[i] = p[keep & (p > p[i])].sum() < top_p * z1
-        keep = keep_p
+        mass_above = np.concatenate([[0.0], np.cumsum(desc)])[n_above]   # sum of the values > p_i
+        keep = keep & (mass_above < top_p * z1)
     z = p[keep].sum()
-    target = u * z
-    acc = 0.0
-    last = -1
-    for i in range(V):
-        if keep[i]:
-            acc += p[i]
-            last = i
-            if acc > target:
-                return i, float(lp[i] - np.log(z))
-    return last, float(lp[last] - np.log(z))
+    # inverse CDF over the kept tokens in increasing id order
+    cdf = np.cumsum(np.where(keep, p, 0.0))
+    i = int(np.searchsorted(cdf, u * z, side="right"))
+    if i >= V:
+        i = int(np.nonzero(keep)[0][-1])
+    return i, float(lp[i] - np.log(z))
 
 
 # ----------------------------------------------------------------------------------

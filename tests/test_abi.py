@@ -81,7 +81,12 @@ def test_null_handles_are_rejected():
     assert L.rlt_encoder_cache_bytes(None, 4, 16) == 0
     assert L.rlt_encode_append_workspace_bytes(None, 4) == 0
     assert L.rlt_encode_prefill(None, None, 1, 1, 1, None, None, None, 1, None, 0, None) == 1
-    assert L.rlt_encode_append(None, None, 1, 1, 0, None, 1, None, None, 1, None, 0, None) == 1
+    assert L.rlt_encode_append(None, None, 1, 1, 0, None, None, 1, None, None, 1, None, 0, None) == 1
+    assert L.rlt_state_positions_offset(None, 4) == 0
+    assert L.rlt_snapshot_bytes(None, 4) == 0
+    assert L.rlt_state_reset_row(None, None, 0, None) == 1
+    assert L.rlt_snapshot_save(None, None, 0, None, 1, None, 1, None, 0, None) == 1
+    assert L.rlt_snapshot_load(None, None, None, 0, None, 1, None, 1, None) == 1
     assert L.rlt_sample(None, None, 1, None, 0, 1.0, None, 1, None, None) == 1
     assert L.rlt_set_option(None, b"row_groups", 1) == 1
     assert L.rlt_selftest_wait_timeout(None, None, None, None, 1, 1, 8, 2, 1000000, None) == 1

@@ -400,6 +400,43 @@ def test_sampler_frequencies_match_the_truncated_distribution():
     assert np.all(np.abs(counts - want) <= 1.0 + 1e-9)
 
 
+def _sample_by_definition(logp, u, top_k=0, top_p=1.0):
+    """Reading R12 written out token by token (quadratic; tiny vocabularies only)."""
+    p = np.exp(np.asarray(logp, np.float64))
+    V = len(p)
+    keep = [top_k <= 0 or sum(1 for j in range(V) if p[j] > p[i]) < top_k for i in range(V)]
+    if top_p < 1.0:
+        z1 = sum(p[i] for i in range(V) if keep[i])
+        keep = [keep[i] and sum(p[j] for j in range(V) if keep[j] and p[j] > p[i]) < top_p * z1 for i in range(V)]
+    z = sum(p[i] for i in range(V) if keep[i])
+    acc, last = 0.0, -1
+    for i in range(V):
+        if keep[i]:
+            acc += p[i]
+            last = i
+            if acc > u * z:
+                return i, math.log(p[i] / z)
+    return last, math.log(p[last] / z)
+
+
+def test_sampler_equals_its_definition_by_brute_force():
+    """400 random small rows (a third with exact ties), random top-k / top-p / uniform."""
+    rng = np.random.default_rng(22)
+    for trial in range(400):
+        V = int(rng.integers(2, 40))
+        z = rng.standard_normal(V) * rng.uniform(0.3, 3)
+        if trial % 3 == 0:
+            z = np.round(z * 2) / 2
+        lp = z - scipy.special.logsumexp(z)
+        u = float(rng.random())
+        k = int(rng.integers(0, V + 2)) if trial % 2 else 0
+        tp = float(rng.uniform(0.05, 1.0)) if trial % 4 < 2 else 1.0
+        tok, blp = sample_token(lp, u, k, tp)
+        want_tok, want_blp = _sample_by_definition(lp, u, k, tp)
+        assert tok == want_tok, (trial, tok, want_tok)
+        assert blp == pytest.approx(want_blp, abs=1e-12)
+
+
 # ---------------------------------------------------------------- replay contract
 
 @pytest.fixture(scope="module")
