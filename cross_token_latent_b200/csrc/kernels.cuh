@@ -18,6 +18,9 @@ struct Launch {
     // Cap on the resident CTAs per SM of the attention kernels (0: none).  With two row groups
     // the attention of one group leaves room on every SM for the other group's projections.
     int attn_ctas_per_sm = 0;
+    // Projections with at most this many rows of A run on the weight-streaming CUDA-core kernel
+    // (gemv.cu) when its shape rules hold (0: never).
+    int gemv_max_rows = 0;
 };
 
 // Number of SMs of the current device (queried once per process).
@@ -203,6 +206,15 @@ bool gemm_swap_preferred(int M, int N, int K);
 int gemm_swap_auto_split(int M, int N, int K);
 cudaError_t launch_gemm_swap(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                              const EpiArgs& ea, DevHeader* hdr, int split = 0);
+
+// ------------------------------------------------------------------ gemv.cu
+// Weight-streaming projection for 1..4 rows on CUDA cores, bulk-copied weight rows (requested
+// before the programmatic-launch wait), the same fused epilogues.  Shape rules: N a multiple of
+// 32, K a multiple of 8 and at most 6144, 16-byte aligned operands.
+bool gemv_shape_supported(int M, int N, int K, int lda);
+bool gemv_supported(int M, int N, int K, int lda, const void* A, const void* W);
+cudaError_t launch_gemv(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
+                        const EpiArgs& ea, DevHeader* hdr);
 
 // ------------------------------------------------------------------ attention.cu
 // Decoder sliding-window self-attention for one layer: sequence b is at step t = pos[b] + 1

@@ -171,6 +171,7 @@ struct rlt_model {
     int opt_row_groups = 1;             // 1 one group, 2 two groups when B >= GROUP_MIN_ROWS
     int opt_attn_cap = 0;               // resident attention CTAs per SM (0: no cap)
     int opt_group_pdl = 0;              // programmatic dependent launch inside a group's chain
+    int opt_gemv_rows = 4;              // projections of at most this many rows stream on CUDA cores
     // two row groups: library-owned streams, forked from and joined back to the caller's stream
     cudaStream_t gs[2] = {nullptr, nullptr};
     cudaEvent_t fork_ev = nullptr, join_ev[2] = {nullptr, nullptr};
@@ -197,7 +198,11 @@ struct rlt_model {
 
     DevHeader* hdr() const { return reinterpret_cast<DevHeader*>(arena); }
     template <typename T> T* at(size_t off) const { return reinterpret_cast<T*>(arena + off); }
-    Launch launch(void* stream) { return Launch{reinterpret_cast<cudaStream_t>(stream), &launches}; }
+    Launch launch(void* stream) {
+        Launch L{reinterpret_cast<cudaStream_t>(stream), &launches};
+        L.gemv_max_rows = opt_gemv_rows;
+        return L;
+    }
 
     Dest dest(const std::string& name) const {
         const rlt_config& c = cfg;
@@ -340,7 +345,7 @@ template <typename T>
 rlt_status encode_impl(rlt_model* m, const int32_t* tokens, int B, int Tn, int T_alloc, T* e, T* M,
                        uint8_t* ws, cudaStream_t st, T* cache = nullptr, int T_max = 0) {
     const rlt_config& c = m->cfg;
-    Launch L{st, &m->launches};
+    Launch L = m->launch(st);
     EncWS w = enc_ws(c, B, Tn);
     int N = B * Tn, d = c.d, F = c.F, H = c.n_heads, hd = c.head_dim;
     float* h = reinterpret_cast<float*>(ws + w.h);
@@ -421,7 +426,7 @@ rlt_status encode_append_impl(rlt_model* m, const int32_t* tok, int tok_stride, 
                               const int32_t* positions, T* cache, int T_max, T* e, T* M, int T_alloc, uint8_t* ws,
                               cudaStream_t st) {
     const rlt_config& c = m->cfg;
-    Launch L{st, &m->launches};
+    Launch L = m->launch(st);
     AppWS w = app_ws(c, B);
     const int d = c.d, F = c.F, H = c.n_heads, hd = c.head_dim;
     float* h = reinterpret_cast<float*>(ws + w.h);
@@ -625,7 +630,7 @@ rlt_status step_impl(rlt_model* m, uint8_t* state, int B, const T* e, const T* M
     DecWS w = dec_ws(m->cfg, B);
     float* part = reinterpret_cast<float*>(ws + w.part);
     if (m->row_groups(B) == 1 || !m->group_streams()) {
-        Launch L{st, &m->launches};
+        Launch L = m->launch(st);
         L.attn_ctas_per_sm = m->opt_attn_cap;
         return step_rows<T>(m, state, B, 0, B, e, M, T_alloc, t, io, ws, part, true, L);
     }
@@ -635,7 +640,7 @@ rlt_status step_impl(rlt_model* m, uint8_t* state, int B, const T* e, const T* M
     rlt_status r = RLT_OK;
     for (int g = 0; g < 2 && r == RLT_OK; ++g) {
         CK(cudaStreamWaitEvent(m->gs[g], m->fork_ev, 0));
-        Launch L{m->gs[g], &m->launches};
+        Launch L = m->launch(m->gs[g]);
         L.pdl = m->opt_group_pdl != 0;
         L.attn_ctas_per_sm = m->opt_attn_cap;
         r = g == 0 ? step_rows<T>(m, state, B, 0, B0, e, M, T_alloc, t, io, ws, part, true, L)
@@ -652,7 +657,7 @@ rlt_status step_impl(rlt_model* m, uint8_t* state, int B, const T* e, const T* M
 
 template <typename T>
 rlt_status state_init_impl(rlt_model* m, uint8_t* state, int B, cudaStream_t st) {
-    Launch L{st, &m->launches};
+    Launch L = m->launch(st);
     CK(launch_state_init(L, m->at<float>(m->lay.s_star), B, m->cfg.d,
                          reinterpret_cast<float*>(state + state_s_off()),
                          reinterpret_cast<StateHeader*>(state), m->version, state_pos(m->cfg, state, B)));
@@ -1211,6 +1216,9 @@ rlt_status rlt_set_option(rlt_model* m, const char* name, int64_t value) {
     } else if (n == "attn_ctas_per_sm") {
         if (value < 0 || value > 32) return RLT_EINVAL;
         m->opt_attn_cap = (int)value;
+    } else if (n == "gemv_rows") {
+        if (value < 0 || value > 4) return RLT_EINVAL;
+        m->opt_gemv_rows = (int)value;
     } else if (n == "group_pdl") {
         if (value < 0 || value > 1) return RLT_EINVAL;
         m->opt_group_pdl = (int)value;
@@ -1222,6 +1230,7 @@ rlt_status rlt_set_option(rlt_model* m, const char* name, int64_t value) {
 
 int rlt_gemm_plan(int M, int N, int K) {
     if (M < 1 || N < 1 || K < 1) return -1;
+    if (gemv_shape_supported(M, N, K, K)) return 16;
     if (gemm_swap_preferred(M, N, K)) {
         const int s = gemm_swap_auto_split(M, N, K);
         return 11 + (s == 1 ? 1 : (s == 2 ? 2 : (s == 4 ? 3 : 4)));
@@ -1232,8 +1241,9 @@ int rlt_gemm_plan(int M, int N, int K) {
 rlt_status rlt_gemm_bf16(rlt_model* m, const void* A, const void* W, float* C, int M, int N, int K, int kernel,
                          void* stream) {
     const int n_tc = gemm_tc_variants();
-    if (!m || !A || !W || !C || M < 1 || N < 1 || K < 1 || kernel < 0 || kernel > 1 + n_tc + 5) return RLT_EINVAL;
-    if (kernel > 1 + n_tc && !gemm_swap_supported(M)) return RLT_EINVAL;
+    if (!m || !A || !W || !C || M < 1 || N < 1 || K < 1 || kernel < 0 || kernel > 2 + n_tc + 5) return RLT_EINVAL;
+    if (kernel > 1 + n_tc && kernel <= 1 + n_tc + 5 && !gemm_swap_supported(M)) return RLT_EINVAL;
+    if (kernel == 2 + n_tc + 5 && !gemv_supported(M, N, K, K, A, W)) return RLT_EINVAL;
     if (!aligned(A, 16) || !aligned(W, 16) || !aligned(C, 16) || K % 8 || N % 4) return RLT_EINVAL;
     Launch L = m->launch(stream);
     EpiArgs ea;
@@ -1248,9 +1258,11 @@ rlt_status rlt_gemm_bf16(rlt_model* m, const void* A, const void* W, float* C, i
         CK(launch_gemm_simt<bf16>(L, Epi::StoreF32, a, K, w, M, N, K, ea));
     } else if (kernel <= 1 + n_tc) {
         CK(launch_gemm_tc(L, Epi::StoreF32, a, K, w, M, N, K, ea, m->hdr(), kernel - 2));
-    } else {
+    } else if (kernel <= 1 + n_tc + 5) {
         static const int splits[5] = {0, 1, 2, 4, 8};
         CK(launch_gemm_swap(L, Epi::StoreF32, a, K, w, M, N, K, ea, m->hdr(), splits[kernel - 2 - n_tc]));
+    } else {
+        CK(launch_gemv(L, Epi::StoreF32, a, K, w, M, N, K, ea, m->hdr()));
     }
     return RLT_OK;
 }

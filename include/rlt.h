@@ -340,6 +340,10 @@ uint64_t rlt_launch_count(const rlt_model* m);
  *                        (0, the default: none), leaving room on every SM for projection CTAs
  *                        that start early (programmatic launch) or run on the other group's
  *                        stream.
+ *   "gemv_rows"          projections of at most this many rows (0..4, default 4) run on the
+ *                        weight-streaming CUDA-core kernel (bulk-copied weight rows requested
+ *                        before the programmatic-launch wait) when its shape rules hold; 0 keeps
+ *                        them on the few-row tensor-core kernel.
  *   "group_pdl"          1: programmatic dependent launch inside each row group's chain
  *                        (default 0: an early-launched kernel would hold SM resources the
  *                        other group needs).
@@ -357,14 +361,16 @@ rlt_status rlt_set_option(rlt_model* m, const char* name, int64_t value);
  * CTAs with a shared-memory reduction: 5: 128x128 split 2; 6: 128x128 split 4; 7: 128x64
  * split 2; 8: 128x64 split 4), kernel 11 + s (M <= 64 only) = the few-row kernel with the
  * weights on the MMA's M side and K split over a cluster of (s = 0: chosen, 1: 1, 2: 2, 3: 4,
- * 4: 8) CTAs.  A, W, C 16-byte aligned, K a multiple of 8, N a multiple of 4.
+ * 4: 8) CTAs, kernel 16 (M <= 4, N a multiple of 32, K <= 6144) = the weight-streaming
+ * CUDA-core kernel.  A, W, C 16-byte aligned, K a multiple of 8, N a multiple of 4.
  * Errors: RLT_EINVAL, RLT_ECUDA; a tensor-core wait that times out latches
  * RLT_ETIMEOUT (rlt_last_error). */
 rlt_status rlt_gemm_bf16(rlt_model* m, const void* A, const void* W, float* C, int M, int N, int K,
                          int kernel, void* stream);
 
 /* The kernel id (numbered as for rlt_gemm_bf16: 2 + v for row-tile variant v, 11 + s for the
- * few-row kernel with split s = 1: 1, 2: 2, 3: 4) that the library's own projections use for an
+ * few-row kernel with split s = 1: 1, 2: 2, 3: 4, 16 for the weight-streaming kernel, which the
+ * "gemv_rows" option can turn off) that the library's own projections use for an
  * M x N x K bf16 product whose operands TMA can address, before any epilogue-specific
  * adjustment.  Pure host logic: no device, model or stream is touched.  Returns -1 for
  * non-positive sizes. */

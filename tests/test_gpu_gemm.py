@@ -22,6 +22,9 @@ SHAPES = [
     (300, 200, 136),      # ragged M, N and K (K not a multiple of the 64-wide k-block)
     (4096, 1536, 1024),   # encoder-like
     (129, 40, 64),
+    (2, 6144, 2048),      # weight-streaming kernel: two rows
+    (4, 11264, 5632),     # four rows, the widest K it takes
+    (1, 32000, 1024),     # LM head of the 300M-class model at B=1
 ]
 
 
@@ -30,11 +33,13 @@ def model():
     return build_model(TINY.model, max_pos=8)
 
 
-@pytest.mark.parametrize("kernel", [0, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13, 14, 15])
+@pytest.mark.parametrize("kernel", [0, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13, 14, 15, 16])
 @pytest.mark.parametrize("M,N,K", SHAPES)
 def test_tcgen05_gemm_matches_float64(model, M, N, K, kernel):
     if kernel >= 11 and M > 64:
         pytest.skip("the few-row kernel takes M <= 64")
+    if kernel == 16 and (M > 4 or N % 32 or K > 6144):
+        pytest.skip("the weight-streaming kernel takes M <= 4, N a multiple of 32, K <= 6144")
     g = torch.Generator().manual_seed(M * 7919 + N * 31 + K)
     A = torch.randn(M, K, generator=g).to(torch.bfloat16)
     W = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16)

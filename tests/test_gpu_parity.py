@@ -199,6 +199,27 @@ def test_large_ragged_batch_matches_the_oracle(B):
     np.testing.assert_array_equal(to_np(lp_tok), lp_step)
 
 
+@pytest.mark.parametrize("options", [{"row_groups": 2}, {"row_groups": 2, "group_pdl": 1, "attn_ctas_per_sm": 5},
+                                     {"attn_ctas_per_sm": 3}])
+def test_scheduling_options_keep_parity(options):
+    """The scheduling options (two row groups on library streams, a cap on the attention CTAs
+    per SM) change only summation order: sampled sequences of a 259-row batch match the oracle
+    and the per-token log-probs stay within the bf16 tolerance of the default schedule."""
+    cfg = replace(TINY.model, dtype="bf16", W=5, G=2)
+    w = make_weights(cfg, seed=3)
+    B, T = 259, 20
+    tok = np.random.default_rng([5, B]).integers(0, cfg.V, size=(B, T)).astype(np.int32)
+    model = build_model(cfg, max_pos=T, weights=w)
+    _, _, _, _, lp_default, _ = gpu_run(model, tok, full=False)
+    for k, v in options.items():
+        model.set_option(k, v)
+    _, _, s, lp, lp_tok, _ = gpu_run(model, tok, tau=1.0)
+    assert np.abs(lp_tok - lp_default).max() <= BF16_LP_TOL
+    sample = [0, 127, 128, 255, 256, 258]
+    _, _, s_r, lp_r = RLTOracle(cfg, w).run(tok[sample])
+    check(cfg, s[sample], lp[sample], s_r, lp_r)
+
+
 @pytest.mark.parametrize("B", [40, 7])
 def test_few_row_batch_matches_the_oracle_and_replays_bit_for_bit(B):
     """Batches of at most 64 rows take the swapped few-row projections (K split over clusters,
