@@ -143,40 +143,39 @@ def test_generation_loop_tiny_f32_matches_the_oracle():
 
 
 def test_generation_loop_small_bf16():
-    """bf16 model: (1) the GPU's loop is self-consistent: re-running the decoder over the final
-    tokens (token-parallel encoding) with full log-prob rows and sampling those rows with the same
-    uniforms reproduces the tokens; the loop's own rows came from incremental encoding, which may
-    differ by bf16 rounding, so a draw may differ where log-probs within the 5e-2 tolerance move a
-    CDF boundary across u: such a draw must be the replayed row's draw at a uniform within
-    exp(5e-2) - 1 (about 5 %) of u, and at most 2 % of the draws may differ; (2) on sampled
-    sequences the oracle, teacher-forced on the GPU's tokens, gives the same prompt and
-    behaviour log-probs within the bf16 tolerance."""
+    """bf16 model: (1) the loop's wiring: re-running the same calls teacher-forced on the
+    generated tokens (prefill, decoder steps, resample each full log-prob row with the same
+    uniform, append the token) reproduces every token bit for bit, so each draw came from the
+    step's own row and uniform; (2) on sampled sequences the oracle, teacher-forced on the GPU's
+    tokens, gives the same prompt and behaviour log-probs within the bf16 tolerance."""
     cfg = SMALL.model
     w = make_weights(cfg)
     model = build_model(cfg, max_pos=192, weights=w)
     B, P, n_new, tau, top_k, top_p = 64, 128, 64, 0.8, 0, 0.9
+    T = P + n_new
     prompt = torch.from_numpy(make_tokens(SMALL)[:B, :P]).cuda()
     u = torch.from_numpy(np.random.default_rng(42).random((n_new, B)).astype(np.float32)).cuda()
     toks, blp, lp_prompt, st = model.generate(prompt, n_new, u, tau, top_k, top_p)
     torch.cuda.synchronize()
     assert model.last_error() == 0
     toks_np = toks.cpu().numpy()
-    # (1) replay the decoder over the final tokens and resample
-    _, _, _, lp_full, _, _ = gpu_run(model, toks_np, tau=tau)
+    assert np.array_equal(toks_np[:, :P], prompt.cpu().numpy())
+    # (1) the same calls, teacher-forced
+    tt = torch.from_numpy(np.ascontiguousarray(toks_np.T)).cuda()          # row t = x_{t+1}
+    e, M, cache = model.encode_prefill(prompt.contiguous(), T_alloc=T, T_max=T)
+    st2 = model.new_state(B)
+    row = torch.empty((B, cfg.V), device="cuda")
     redraw = torch.empty(B, dtype=torch.int32, device="cuda")
-    mismatch = 0
-    for j in range(n_new):
-        t = P + j
-        rows = torch.from_numpy(np.ascontiguousarray(lp_full[:, t - 1])).cuda()
-        model.sample(rows, u[j], top_k, top_p, out=redraw)
-        got = redraw.cpu().numpy()
-        for b in np.nonzero(got != toks_np[:, t])[0]:
-            uj = float(u[j, b])
-            reach = {sample_token(lp_full[b, t - 1], min(max(uj + k * 0.0052, 0.0), 1 - 1e-12), top_k, top_p)[0]
-                     for k in range(-10, 11)}
-            assert int(toks_np[b, t]) in reach, (b, t)
-            mismatch += 1
-    assert mismatch <= 0.02 * n_new * B
+    blp2 = torch.empty(B, device="cuda")
+    for t in range(1, T):
+        if t < P:
+            model.decode_step(st2, e, M, next_tok=tt[t], tau=tau)
+            continue
+        model.decode_step(st2, e, M, tau=tau, logp_full=row)
+        model.sample(row, u[t - P], top_k, top_p, out=redraw, behaviour_logp=blp2)
+        assert torch.equal(redraw, tt[t]), t
+        assert torch.equal(blp2, blp[:, t - P]), t
+        model.encode_append(tt[t], t, cache, T, e, M)
     # (2) oracle, teacher-forced, on four sequences
     seqs = [0, 1, 17, 63]
     _, _, _, lp_o = RLTOracle(cfg, w).run(toks_np[seqs], tau=tau)
