@@ -124,12 +124,15 @@ __device__ __forceinline__ void merge_groups(float& m, float& l, float* acc) {
     }
 }
 
-// One CTA of SWA_WARPS warps per (sequence, head).  Every warp computes q and the current
-// k/v (RoPE at position t-1); warp w streams a contiguous share of the n = min(t-1, W-1)
-// cached entries; the warps' partial softmax states are merged through shared memory, then
-// warp 0 writes the output and stores k_t, v_t into ring slot (t-1) mod (W-1) (after every
-// warp has read the ring, so the slot's old entry -- token t-W+1, still in the window -- is
-// used first).
+// One CTA of SWA_WARPS warps per (sequence, head) and key split.  Every warp computes q (RoPE
+// at position t-1); the n = min(t-1, W-1) cached entries are cut into n_splits contiguous
+// ranges of ring slots, one per CTA, and warp w of a CTA streams a contiguous share of its
+// range; the warps' partial softmax states are merged through shared memory.  Split 0 also
+// attends to the current token (k_t, v_t rounded to the storage type).  The CTA whose range
+// holds ring slot (t-1) mod (W-1) (split 0 while the ring is not yet full) stores k_t, v_t
+// there after its warps have read the slot's old entry -- token t-W+1, still in the window.
+// With one split the CTA writes the normalised output; with several, each writes its
+// unnormalised partial (acc, max, sum) and k_attn_combine merges them.
 constexpr int SWA_WARPS = 4;
 
 template <typename T, int HD>
@@ -137,7 +140,8 @@ __global__ void __launch_bounds__(SWA_WARPS * 32, 6) k_swa_decode(const float* _
                                                                   const float2* __restrict__ rope,
                                                                   T* __restrict__ ring, T* __restrict__ o,
                                                                   int B, int H, int W, const int32_t* __restrict__ pos,
-                                                                  int max_t, float qscale) {
+                                                                  int max_t, int n_splits, float* __restrict__ part,
+                                                                  float qscale) {
     using G = Geom<T, HD>;
     constexpr int EPL = G::EPL, LPK = G::LPK;
     __shared__ float sm_m[SWA_WARPS], sm_l[SWA_WARPS];
@@ -147,27 +151,36 @@ __global__ void __launch_bounds__(SWA_WARPS * 32, 6) k_swa_decode(const float* _
     pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane / LPK, li = lane % LPK;
     const int d = H * HD, half = HD / 2;
-    // one (sequence, head) item per iteration; the grid is at most one item per CTA and may be
-    // capped below that (then each CTA takes items blockIdx.x, blockIdx.x + gridDim.x, ...)
-    for (int item = blockIdx.x; item < B * H; item += gridDim.x) {
+    // one (sequence, head, split) work item per iteration; the grid is at most one item per CTA
+    // and may be capped below that (then each CTA takes items blockIdx.x, blockIdx.x +
+    // gridDim.x, ...)
+    for (int wi = blockIdx.x; wi < B * H * n_splits; wi += gridDim.x) {
+        const int item = wi / n_splits, sp = wi % n_splits;
         const int b = item / H, h = item % H;
         // this sequence's step t: it has consumed pos[b] tokens (clamped to the bound the host
         // checked, so that a corrupt state cannot address outside the rotary table)
         const int t = min(max(pos[b] + 1, 1), max_t);
         const float2* rope_row = rope + (long long)(t - 1) * half;
         const float* row = qkv + (long long)b * 3 * d + h * HD;
-        // this warp's share of the ring; its first round of loads is issued before q is formed,
-        // so the ring's memory latency overlaps the q / RoPE loads instead of following them
+        // this split's range of ring slots, and this warp's share of it; the warp's first round
+        // of loads is issued before q is formed, so the ring's memory latency overlaps the q /
+        // RoPE loads instead of following them
         T* Kr = nullptr;
         T* Vr = nullptr;
-        int j0 = 0, nj = 0;
+        int j0 = 0, nj = 0, s0 = 0, s1 = 0, slot = 0;
+        bool writer = false;
         if (W > 1) {
             Kr = ring + (((long long)b * 2 + 0) * H + h) * (long long)(W - 1) * HD;
             Vr = ring + (((long long)b * 2 + 1) * H + h) * (long long)(W - 1) * HD;
-            int n = min(t - 1, W - 1);
-            int per = (n + SWA_WARPS - 1) / SWA_WARPS;
-            j0 = min(n, warp * per);
-            nj = min(n, j0 + per) - j0;
+            const int n = min(t - 1, W - 1);
+            const int per_split = (n + n_splits - 1) / n_splits;
+            s0 = min(n, sp * per_split);
+            s1 = min(n, s0 + per_split);
+            const int per = (s1 - s0 + SWA_WARPS - 1) / SWA_WARPS;
+            j0 = min(s1, s0 + warp * per);
+            nj = min(s1, j0 + per) - j0;
+            slot = (t - 1) % (W - 1);
+            writer = slot < n ? (slot >= s0 && slot < s1) : sp == 0;
         }
         constexpr int SWA_U = 4;
         uint4 kr0[SWA_U], vr0[SWA_U];
@@ -184,7 +197,7 @@ __global__ void __launch_bounds__(SWA_WARPS * 32, 6) k_swa_decode(const float* _
         float m = NEG_BIG, l = 0.f, acc[EPL];
 #pragma unroll
         for (int i = 0; i < EPL; ++i) acc[i] = 0.f;
-        if (warp == 0) {
+        if (warp == 0 && (sp == 0 || writer)) {
             // the current token: k_t (rotated) and v_t rounded to the storage type, as cached
             float k[EPL], v[EPL];
 #pragma unroll
@@ -196,14 +209,18 @@ __global__ void __launch_bounds__(SWA_WARPS * 32, 6) k_swa_decode(const float* _
                 k[i] = round_to<T>(c < half ? ka * cs.x - kp * cs.y : kp * cs.y + ka * cs.x);
                 v[i] = round_to<T>(row[2 * d + c]);
             }
-            float sc = 0.f;
+            if (sp == 0) {
+                float sc = 0.f;
 #pragma unroll
-            for (int i = 0; i < EPL; ++i) sc = fmaf(q[i], k[i], sc);
-            sc = group_sum<LPK>(sc);
+                for (int i = 0; i < EPL; ++i) sc = fmaf(q[i], k[i], sc);
+                sc = group_sum<LPK>(sc);
+                if (g == 0) {
+                    m = sc; l = 1.f;
+#pragma unroll
+                    for (int i = 0; i < EPL; ++i) acc[i] = v[i];
+                }
+            }
             if (g == 0) {
-                m = sc; l = 1.f;
-#pragma unroll
-                for (int i = 0; i < EPL; ++i) acc[i] = v[i];
                 sm_kv[0][li] = Vec16<T>::pack(k);
                 sm_kv[1][li] = Vec16<T>::pack(v);
             }
@@ -234,12 +251,18 @@ __global__ void __launch_bounds__(SWA_WARPS * 32, 6) k_swa_decode(const float* _
 #pragma unroll
                 for (int i = 0; i < EPL; ++i) out[i] += sm_acc[w][li * EPL + i] * c;
             }
-            float inv = 1.0f / L;
+            if (n_splits == 1) {
+                float inv = 1.0f / L;
 #pragma unroll
-            for (int i = 0; i < EPL; ++i) out[i] *= inv;
-            st16(o + (long long)b * d + h * HD + li * EPL, Vec16<T>::pack(out));
-            if (W > 1) {
-                int slot = (t - 1) % (W - 1);
+                for (int i = 0; i < EPL; ++i) out[i] *= inv;
+                st16(o + (long long)b * d + h * HD + li * EPL, Vec16<T>::pack(out));
+            } else {
+                float* pp = part + (long long)wi * (HD + 2);
+#pragma unroll
+                for (int i = 0; i < EPL; ++i) pp[li * EPL + i] = out[i];
+                if (li == 0) { pp[HD] = mx; pp[HD + 1] = L; }
+            }
+            if (W > 1 && writer) {
                 st16(Kr + (long long)slot * HD + li * EPL, sm_kv[0][li]);
                 st16(Vr + (long long)slot * HD + li * EPL, sm_kv[1][li]);
             }
@@ -372,10 +395,19 @@ inline unsigned capped(const Launch& L, unsigned blocks) {
     }
 
 template <typename T>
+static cudaError_t swa_main(Launch L, const float* qkv, const float2* rope, T* ring, T* o, int B, int H, int hd,
+                           int W, const int32_t* pos, int max_t, int n_splits, float* part) {
+    RLT_HD_DISPATCH(hd, launch_k(L, k_swa_decode<T, HD>, capped(L, (unsigned)(B * H * n_splits)), SWA_WARPS * 32, 0,
+                                 qkv, rope, ring, o, B, H, W, pos, max_t, n_splits, part, qscale_for(hd)));
+}
+
+template <typename T>
 cudaError_t launch_swa_decode(Launch L, const float* qkv, const float2* rope, T* ring, T* o, int B,
-                              int H, int hd, int W, const int32_t* pos, int max_t) {
-    RLT_HD_DISPATCH(hd, launch_k(L, k_swa_decode<T, HD>, capped(L, (unsigned)(B * H)), SWA_WARPS * 32, 0, qkv, rope,
-                                 ring, o, B, H, W, pos, max_t, qscale_for(hd)));
+                              int H, int hd, int W, const int32_t* pos, int max_t, int n_splits, float* part) {
+    if (n_splits < 1 || !part) n_splits = 1;
+    cudaError_t e = swa_main<T>(L, qkv, rope, ring, o, B, H, hd, W, pos, max_t, n_splits, part);
+    if (e != cudaSuccess || n_splits == 1) return e;
+    return launch_k(L, k_attn_combine<T>, (unsigned)(B * H), (unsigned)hd, 0, (const float*)part, n_splits, hd, H, o);
 }
 
 template <typename T>
@@ -403,7 +435,7 @@ cudaError_t launch_enc_attention(Launch L, const T* planes, T* o, int B, int Tn,
 
 #define RLT_INST(T)                                                                                    \
     template cudaError_t launch_swa_decode<T>(Launch, const float*, const float2*, T*, T*, int, int,   \
-                                              int, int, const int32_t*, int);                          \
+                                              int, int, const int32_t*, int, int, float*);             \
     template cudaError_t launch_xattn_decode<T>(Launch, const float*, const T*, long long, int, int, T*, int, \
                                                 int, int, int, float*, const int32_t*);                \
     template cudaError_t launch_enc_attention<T>(Launch, const T*, T*, int, int, int, int);

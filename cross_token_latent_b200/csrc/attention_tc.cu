@@ -3,15 +3,20 @@
 // One CTA computes 128 queries of one (sequence, head) against the causal key range in tiles
 // of 128 keys, flash-attention style, with every operand K-major in the 128-byte swizzle
 // layout that TMA writes:
-//   warp 4, lane 0  TMA producer: the Q tile once, then K and V^T tiles into two stages;
-//   warp 5, lane 0  MMA issuer: S = Q K^T into TMEM columns [0, 128), then O += P V into TMEM
-//                   columns [128, 128 + head_dim) once the softmax warps have written P;
-//   warp 5          allocates / frees the 256 TMEM columns;
-//   warps 0-3       softmax: thread r owns query row r (TMEM lane r): causal mask on the
-//                   diagonal tile, running max, exp2, P rounded to bf16 into shared memory (the
-//                   row sum is taken over the rounded values, so P V / sum stays a convex
-//                   combination), rescale of O in TMEM when the max grows, and the epilogue
-//                   O / sum -> bf16.
+//   warp 8, lane 0  TMA producer: the Q tile once, then K and V^T tiles into two stages;
+//   warp 9          allocates / frees the 512 TMEM columns; lane 0 issues the MMAs: S_j = Q K_j^T
+//                   into one of two S buffers (TMEM columns [0, 128) and [128, 256)) as soon as
+//                   K_j has landed and the buffer's previous tile has been read, so the next
+//                   tile's scores are ready while the softmax of this one runs; then O += P_j V_j
+//                   into TMEM columns [256, 256 + head_dim) once P_j is written;
+//   warps 0-7       softmax, two warps per TMEM lane quadrant: warp w owns query row
+//                   32 (w % 4) + lane and key columns [64 h, 64 h + 64) of each tile, h = w / 4.
+//                   The two halves of a row post their partial maxima to shared memory (an
+//                   mbarrier per quadrant, bounded waits) and both continue with the row's
+//                   maximum: causal mask on the diagonal tile, exp2, P rounded to bf16 into
+//                   shared memory (the row sum is taken over the rounded values, so P V / sum
+//                   stays a convex combination), rescale of their half of O in TMEM when the
+//                   maximum grows, and the epilogue O / sum -> bf16 over their half of head_dim.
 // V is stored transposed per (sequence, head) ([head_dim][T_pad], keys contiguous) so that it
 // is a K-major B operand like the others.  Every mbarrier wait is bounded.
 #include <cudaTypedefs.h>
@@ -37,14 +42,18 @@ struct FaShape {
     static constexpr int OFF_K = OFF_Q + Q_BYTES;         // 2 stages
     static constexpr int OFF_V = OFF_K + 2 * K_BYTES;     // 2 stages
     static constexpr int OFF_P = OFF_V + 2 * V_BYTES;
-    static constexpr int OFF_BAR = OFF_P + P_BYTES;
+    static constexpr int OFF_RED = OFF_P + P_BYTES;       // row-max exchange [2][2 halves][128 rows]
+    static constexpr int OFF_BAR = OFF_RED + 2 * 2 * QT * 4;
     static constexpr int SMEM = OFF_BAR + 256 + 1024;
-    static constexpr int TMEM_COLS = 256;
-    static constexpr uint32_t S_COL = 0, O_COL = 128;
+    static constexpr int TMEM_COLS = 512;
+    static constexpr uint32_t S_COL = 0, O_COL = 256;     // S double-buffered at 0 and 128
 };
 
+constexpr int FA_SOFTMAX_WARPS = 8;                        // two per TMEM lane quadrant
+constexpr int FA_THREADS = (FA_SOFTMAX_WARPS + 2) * 32;    // + TMA producer + MMA issuer
+
 template <int HD>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(FA_THREADS, 1)
 k_enc_fa_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
             const __grid_constant__ CUtensorMap tmV, bf16* __restrict__ o, int B, int Tn, int H, float qscale,
             DevHeader* hdr) {
@@ -54,10 +63,13 @@ k_enc_fa_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
     uint64_t* kv_full = q_full + 1;       // [2]
     uint64_t* kv_empty = kv_full + 2;     // [2]
-    uint64_t* s_full = kv_empty + 2;
-    uint64_t* p_full = s_full + 1;
-    uint64_t* o_done = p_full + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
+    uint64_t* s_full = kv_empty + 2;      // [2] S buffer b holds S_j for j % 2 == b
+    uint64_t* s_free = s_full + 2;        // [2] the softmax warps have read S buffer b
+    uint64_t* p_full = s_free + 2;        // P_j written and O rescaled
+    uint64_t* o_done = p_full + 1;        // O += P_j V_j complete
+    uint64_t* red_ready = o_done + 1;     // [2][4] both halves of a quadrant posted their row max
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_ready + 8);
+    float* red = reinterpret_cast<float*>(smem + S::OFF_RED);
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -66,6 +78,7 @@ k_enc_fa_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     const int bh = blockIdx.y;
     const int q0 = qt * QT;
     const int nt = qt + 1;                                 // key tiles 0..qt
+    const int PRODUCER = FA_SOFTMAX_WARPS, ISSUER = FA_SOFTMAX_WARPS + 1;
     pdl_trigger();
 
     if (threadIdx.x == 0) {
@@ -73,14 +86,16 @@ k_enc_fa_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         for (int s = 0; s < 2; ++s) {
             mbar_init(&kv_full[s], 1);
             mbar_init(&kv_empty[s], 1);
+            mbar_init(&s_full[s], 1);
+            mbar_init(&s_free[s], FA_SOFTMAX_WARPS);
         }
-        mbar_init(s_full, 1);
-        mbar_init(p_full, 128);
+        mbar_init(p_full, FA_SOFTMAX_WARPS);
         mbar_init(o_done, 1);
+        for (int i = 0; i < 8; ++i) mbar_init(&red_ready[i], 64);
         abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 5) {
+    if (warp == ISSUER) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(S::TMEM_COLS));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -90,7 +105,7 @@ k_enc_fa_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
+    if (warp == PRODUCER) {
         if (lane == 0) {
             asm volatile("prefetch.tensormap [%0];" ::"l"(&tmQ) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(&tmK) : "memory");
@@ -112,24 +127,33 @@ k_enc_fa_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 for (int a = 0; a < 2; ++a) tma_load_3d(vb + a * HD * 128, &tmV, &kv_full[s], j * KT + 64 * a, 0, bh);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == ISSUER) {
         if (lane == 0) {
             constexpr uint32_t id_s = idesc_bf16(QT, KT), id_o = idesc_bf16(QT, HD);
-            const uint32_t tS = tmem + S::S_COL, tO = tmem + S::O_COL;
-            bool ok = mbar_wait(q_full, 0, &abort_flag) && mbar_wait(&kv_full[0], 0, &abort_flag);
-            if (ok) {
+            const uint32_t tO = tmem + S::O_COL;
+            // S_j = Q K_j^T into S buffer j % 2, once K_j has landed and the softmax warps have
+            // read that buffer's previous tile j - 2
+            auto issue_s = [&](int j) -> bool {
+                const int s = j & 1;
+                if (!mbar_wait(&kv_full[s], (j >> 1) & 1, &abort_flag)) return false;
+                if (j >= 2 && !mbar_wait(&s_free[s], ((j - 2) >> 1) & 1, &abort_flag)) return false;
                 tc_fence_after();
+                const uint32_t tS = tmem + S::S_COL + s * KT;
 #pragma unroll
                 for (int a = 0; a < S::ATOMS; ++a) {
                     uint64_t dq = sdesc_sw128(smem + S::OFF_Q + a * QT * 128);
-                    uint64_t dk = sdesc_sw128(smem + S::OFF_K + a * KT * 128);
+                    uint64_t dk = sdesc_sw128(smem + S::OFF_K + s * S::K_BYTES + a * KT * 128);
 #pragma unroll
                     for (int k = 0; k < 4; ++k) umma(tS, dq + 2 * k, dk + 2 * k, id_s, (a | k) != 0);
                 }
-                umma_commit(s_full);
-            }
+                umma_commit(&s_full[s]);
+                return true;
+            };
+            bool ok = mbar_wait(q_full, 0, &abort_flag) && issue_s(0);
             for (int j = 0; ok && j < nt; ++j) {
-                int s = j & 1;
+                const int s = j & 1;
+                // the next tile's scores first, so the softmax warps never wait for them
+                if (j + 1 < nt && !issue_s(j + 1)) { ok = false; break; }
                 if (!mbar_wait(p_full, j & 1, &abort_flag)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
@@ -141,52 +165,55 @@ k_enc_fa_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 }
                 umma_commit(&kv_empty[s]);
                 umma_commit(o_done);
-                if (j + 1 < nt) {
-                    int s1 = (j + 1) & 1;
-                    if (!mbar_wait(&kv_full[s1], ((j + 1) >> 1) & 1, &abort_flag)) { ok = false; break; }
-                    tc_fence_after();
-#pragma unroll
-                    for (int a = 0; a < S::ATOMS; ++a) {
-                        uint64_t dq = sdesc_sw128(smem + S::OFF_Q + a * QT * 128);
-                        uint64_t dk = sdesc_sw128(smem + S::OFF_K + s1 * S::K_BYTES + a * KT * 128);
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) umma(tS, dq + 2 * k, dk + 2 * k, id_s, (a | k) != 0);
-                    }
-                    umma_commit(s_full);
-                }
             }
             if (!ok) abort_flag = 1;
         }
     } else {
-        // softmax warps: thread r owns query row r of the tile
-        const int r = threadIdx.x;                        // 0..127
+        // softmax warps: warp w owns query row r = 32 (w % 4) + lane (TMEM lane quadrant w % 4)
+        // and key columns [64 h, 64 h + 64) of every tile, h = w / 4; the two halves of a row
+        // exchange their partial maxima through shared memory on an mbarrier.
+        const int qd = warp & 3, hf = warp >> 2;
+        const int r = qd * 32 + lane;
         const int q = q0 + r;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        const uint32_t tS = tmem + S::S_COL + lane_off, tO = tmem + S::O_COL + lane_off;
-        uint8_t* P = smem + S::OFF_P;
+        const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+        const uint32_t tO = tmem + S::O_COL + lane_off + hf * (HD / 2);
+        uint8_t* P = smem + S::OFF_P + hf * QT * 128;       // this half's 64-key swizzle atom
         float m = -1e30f, l = 0.f;
         bool ok = true;
         for (int j = 0; j < nt; ++j) {
-            ok = ok && mbar_wait(s_full, j & 1, &abort_flag);
+            const int sb = j & 1;
+            ok = ok && mbar_wait(&s_full[sb], (j >> 1) & 1, &abort_flag);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-            float sv[KT];
-#pragma unroll
-            for (int c = 0; c < KT; c += 32) tmem_ld32(tS + c, sv + c);
+            float sv[64];
+            const uint32_t tS = tmem + S::S_COL + sb * KT + lane_off + hf * 64;
+            tmem_ld32(tS, sv);
+            tmem_ld32(tS + 32, sv + 32);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_free[sb]);
             const bool diag = (j == nt - 1);
             float mx = m;
 #pragma unroll
-            for (int c = 0; c < KT; ++c) {
+            for (int c = 0; c < 64; ++c) {
                 float v = sv[c] * qscale;
-                if (diag && j * KT + c > q) v = -1e30f;
+                if (diag && j * KT + hf * 64 + c > q) v = -1e30f;
                 sv[c] = v;
                 mx = fmaxf(mx, v);
             }
+            // the row's maximum over both halves
+            float* rb = red + (size_t)sb * 2 * QT;
+            rb[hf * QT + r] = mx;
+            mbar_arrive(&red_ready[sb * 4 + qd]);
+            ok = mbar_wait(&red_ready[sb * 4 + qd], (j >> 1) & 1, &abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            mx = fmaxf(mx, rb[(1 - hf) * QT + r]);
             const float alpha = exp2f(m - mx);
             float rowsum = 0.f;
-            // P_j overwrites P_{j-1}: wait until P_{j-1} V_{j-1} has completed (it also makes O final
-            // for the rescale below)
+            // P_j overwrites P_{j-1}: wait until P_{j-1} V_{j-1} has completed (it also makes O
+            // final for the rescale below)
             if (j > 0) {
                 ok = mbar_wait(o_done, (j - 1) & 1, &abort_flag);
                 ok = __all_sync(0xffffffffu, ok);
@@ -194,24 +221,21 @@ k_enc_fa_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 tc_fence_after();
             }
 #pragma unroll
-            for (int a = 0; a < 2; ++a) {
+            for (int ch = 0; ch < 8; ++ch) {
+                float p8[8];
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    float p8[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        float p = round_to<bf16>(exp2f(sv[a * 64 + ch * 8 + i] - mx));
-                        p8[i] = p;
-                        rowsum += p;
-                    }
-                    uint8_t* dst = P + a * QT * 128 + r * 128 + ((ch ^ (r & 7)) << 4);
-                    *reinterpret_cast<uint4*>(dst) = Vec16<bf16>::pack(p8);
+                for (int i = 0; i < 8; ++i) {
+                    float p = round_to<bf16>(exp2f(sv[ch * 8 + i] - mx));
+                    p8[i] = p;
+                    rowsum += p;
                 }
+                uint8_t* dst = P + r * 128 + ((ch ^ (r & 7)) << 4);
+                *reinterpret_cast<uint4*>(dst) = Vec16<bf16>::pack(p8);
             }
             l = l * alpha + rowsum;
             if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {     // warp-collective TMEM access
 #pragma unroll 1
-                for (int c = 0; c < HD; c += 32) {
+                for (int c = 0; c < HD / 2; c += 32) {
                     float ov[32];
                     tmem_ld32(tO + c, ov);
 #pragma unroll
@@ -222,7 +246,8 @@ k_enc_fa_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             m = mx;
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(p_full);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);
         }
         pdl_wait();
         if (ok) {
@@ -230,12 +255,22 @@ k_enc_fa_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             ok = __all_sync(0xffffffffu, ok);
         }
         if (ok) {
+            // the row sum over both halves (the same exchange, on the buffer of tile nt)
+            const int sb = nt & 1;
+            float* rb = red + (size_t)sb * 2 * QT;
+            rb[hf * QT + r] = l;
+            mbar_arrive(&red_ready[sb * 4 + qd]);
+            ok = mbar_wait(&red_ready[sb * 4 + qd], (nt >> 1) & 1, &abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) l += rb[(1 - hf) * QT + r];
+        }
+        if (ok) {
             tc_fence_after();
             const float inv = 1.0f / l;
             const int b = bh / H, h = bh % H;
-            bf16* orow = o + ((long long)b * Tn + q) * H * HD + h * HD;
+            bf16* orow = o + ((long long)b * Tn + q) * H * HD + h * HD + hf * (HD / 2);
 #pragma unroll 1
-            for (int c = 0; c < HD; c += 32) {
+            for (int c = 0; c < HD / 2; c += 32) {
                 float ov[32];
                 tmem_ld32(tO + c, ov);
 #pragma unroll
@@ -252,7 +287,7 @@ k_enc_fa_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == ISSUER) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(S::TMEM_COLS));
     }
@@ -305,7 +340,7 @@ cudaError_t run_fa(Launch L, const bf16* q, const bf16* k, const bf16* vt, bf16*
         return cudaErrorInvalidValue;
     dim3 grid((Tn + QT - 1) / QT, (unsigned)BH);
     const float qscale = 1.4426950408889634f / sqrtf((float)HD);
-    return launch_k(L, k_enc_fa_tc<HD>, grid, 192, S::SMEM, tq, tk, tv, o, B, Tn, H, qscale, hdr);
+    return launch_k(L, k_enc_fa_tc<HD>, grid, FA_THREADS, S::SMEM, tq, tk, tv, o, B, Tn, H, qscale, hdr);
 }
 
 }  // namespace

@@ -107,7 +107,7 @@ cudaError_t launch_gemm<float>(Launch L, Epi epi, const float* A, int lda, const
 template <>
 cudaError_t launch_gemm<bf16>(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                               const EpiArgs& ea) {
-    if (M <= L.gemv_max_rows && gemv_supported(M, N, K, lda, A, W))
+    if (M <= L.gemv_max_rows && gemv_preferred(M, N, K) && gemv_supported(M, N, K, lda, A, W))
         return launch_gemv(L, epi, A, lda, W, M, N, K, ea, ea.hdr);
     if (gemm_tc_supported(A, lda, W, K)) {
         if (gemm_swap_preferred(M, N, K)) return launch_gemm_swap(L, epi, A, lda, W, M, N, K, ea, ea.hdr);

@@ -160,6 +160,44 @@ struct RowNorm {
     }
 };
 
+// Fused head (Epi::LsePart) for one row m over the BN accumulator columns at lane_base: the
+// row's (max, sum of exp) of z = acc * scale over the tile's columns n0 .. n0+BN-1 (those
+// below N) goes to lse_part[m * lse_ld + tn], and the tile that holds the row's target column
+// writes its z to z_tok[m].  Nothing is stored per logit.  Warp-collective (TMEM loads).
+template <int BN>
+__device__ __forceinline__ void lse_row(const EpiArgs& ea, uint32_t lane_base, int m, int M, int n0, int N, int tn) {
+    int tk = -1;
+    if (m < M && ea.lse_tok) {
+        tk = ea.lse_tok[(long long)m * ea.tok_stride];
+        if (tk < 0 || tk >= N) tk = 0;
+    }
+    float mx = -INFINITY, sm = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+        float v[16];
+        tmem_ld16(lane_base + c, v);
+        const int n = n0 + c;
+        if (m < M && n < N) {
+            const int cnt = min(16, N - n);
+            float cm = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                v[j] *= ea.scale;
+                if (j < cnt) cm = fmaxf(cm, v[j]);
+                if (n + j == tk) ea.z_tok[m] = v[j];
+            }
+            if (cm > mx) {
+                sm *= expf(mx - cm);
+                mx = cm;
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                if (j < cnt) sm += expf(v[j] - mx);
+        }
+    }
+    if (m < M) ea.lse_part[(long long)m * ea.lse_ld + tn] = make_float2(mx, sm);
+}
+
 template <int BN, int STAGES, int SPLIT>
 struct TcShape {
     static constexpr int B_BYTES = BN * BK * 2;
@@ -282,40 +320,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     if constexpr (SPLIT == 1) {
         if (ok && epi == Epi::LsePart) {
-            // fused head: this row's (max, sum of exp) over the tile's columns of z = acc * scale,
-            // and the gathered z of its target token when the tile holds it; nothing is stored
-            // per logit
-            const int m = m0 + warp * 32 + lane;
-            int tk = -1;
-            if (m < M && ea.lse_tok) {
-                tk = ea.lse_tok[(long long)m * ea.tok_stride];
-                if (tk < 0 || tk >= N) tk = 0;
-            }
-            float mx = -INFINITY, sm = 0.f;
-#pragma unroll 1
-            for (int c = 0; c < BN; c += 16) {
-                float v[16];
-                tmem_ld16(lane_base + c, v);
-                const int n = n0 + c;
-                if (m < M && n < N) {
-                    const int cnt = min(16, N - n);
-                    float cm = -INFINITY;
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        v[j] *= ea.scale;
-                        if (j < cnt) cm = fmaxf(cm, v[j]);
-                        if (n + j == tk) ea.z_tok[m] = v[j];
-                    }
-                    if (cm > mx) {
-                        sm *= expf(mx - cm);
-                        mx = cm;
-                    }
-#pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        if (j < cnt) sm += expf(v[j] - mx);
-                }
-            }
-            if (m < M) ea.lse_part[(long long)m * ea.lse_ld + blockIdx.x] = make_float2(mx, sm);
+            lse_row<BN>(ea, lane_base, m0 + warp * 32 + lane, M, n0, N, blockIdx.x);
         } else if (ok) {
             const int m = m0 + warp * 32 + lane;
 #pragma unroll 1
@@ -387,6 +392,169 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     if (warp == 2) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(S::TMEM_COLS));
+    }
+}
+
+// Persistent row-tile GEMM for grids of many waves (the encoder's projections, the LM head at
+// large batch): one CTA per SM walks the 128 x BN output tiles (tile = blockIdx.x, then every
+// gridDim.x-th; tiles ordered column-fastest, so that the CTAs in flight share the activation
+// row tile in L2), with two TMEM accumulators so that the epilogue of one tile overlaps the
+// MMAs of the next.  6 warps:
+//   warp 0, lane 0   TMA producer over all k-blocks of all the CTA's tiles (one ring);
+//   warp 1           allocates the 2 * BN TMEM columns; lane 0 issues the MMAs of tile i into
+//                    accumulator i % 2 once the epilogue has drained it (acc_empty), then
+//                    commits acc_full;
+//   warps 2-5        epilogue: warp w reads TMEM lanes 32 * (w % 4) .. +31, i.e. output rows
+//                    of that quadrant, with the fused epilogues of k_gemm_tc, then arrives on
+//                    acc_empty.
+// Every wait is bounded; after a timeout every role stops, the MMA issuer still commits what it
+// issued, the CTA waits (bounded) for its loads in flight, latches ERR_TIMEOUT and stores
+// nothing more.
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(192, 1)
+k_gemm_tc_pers(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW, int M, int N, int K,
+               Epi epi, EpiArgs ea, DevHeader* hdr) {
+    using S = TcShape<BN, STAGES, 1>;
+    constexpr int ACC_COLS = 2 * BN;                 // two accumulators
+    static_assert(ACC_COLS <= 512, "two accumulators must fit in TMEM");
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES);
+    uint64_t* empty = full + STAGES;
+    uint64_t* acc_full = empty + STAGES;             // [2]
+    uint64_t* acc_empty = acc_full + 2;              // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+    __shared__ int abort_flag;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int mt = (M + BM - 1) / BM, nt = (N + BN - 1) / BN;
+    const int tiles = mt * nt;
+    const int nkb = (K + BK - 1) / BK;
+    const uint64_t lim = ea.wait_ns;
+    pdl_trigger();
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&acc_full[a], 1);
+            mbar_init(&acc_empty[a], 4);             // one arrival per epilogue warp
+        }
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(ACC_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    int armed = 0;                                   // producer: k-blocks whose loads were issued
+
+    if (warp == 0) {
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(&tmW) : "memory");
+            pdl_wait();
+            int it = 0;
+            for (int tile = blockIdx.x; tile < tiles && !ea.no_loads; tile += gridDim.x) {
+                const int m0 = (tile / nt) * BM, n0 = (tile % nt) * BN;
+                bool ok = true;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    if (it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, &abort_flag, lim)) {
+                        abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* a = smem + s * S::STAGE_BYTES;
+                    mbar_expect_tx(&full[s], S::STAGE_BYTES);
+                    tma_load_2d(a, &tmA, &full[s], kb * BK, m0);
+                    tma_load_2d(a + A_BYTES, &tmW, &full[s], kb * BK, n0);
+                    armed = it + 1;
+                }
+                if (!ok) break;
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16(BM, BN);
+            int it = 0, count = 0;
+            for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++count) {
+                const int a = count & 1, use = count >> 1;
+                // accumulator a is free once the epilogue has drained its previous tile
+                if (use > 0 && !mbar_wait(&acc_empty[a], (use - 1) & 1, &abort_flag, lim)) { abort_flag = 1; break; }
+                tc_fence_after();
+                bool ok = true;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    if (!mbar_wait(&full[s], (it / STAGES) & 1, &abort_flag, lim)) { abort_flag = 1; ok = false; break; }
+                    tc_fence_after();
+                    uint8_t* st = smem + s * S::STAGE_BYTES;
+                    const uint64_t da = sdesc_sw128(st), dw = sdesc_sw128(st + A_BYTES);
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        umma(tmem + a * BN, da + 2 * k, dw + 2 * k, idesc, (kb | k) != 0);
+                    umma_commit(&empty[s]);
+                }
+                umma_commit(&acc_full[a]);           // also after a timeout: tracks what was issued
+                if (!ok) break;
+            }
+        }
+    } else {
+        // epilogue warps: TMEM lane quadrant q = warp % 4 holds output rows 32q .. 32q+31
+        pdl_wait();
+        const int q = warp & 3;
+        int count = 0;
+        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++count) {
+            const int a = count & 1, use = count >> 1;
+            const int tm = tile / nt, tn = tile % nt;
+            const int m0 = tm * BM, n0 = tn * BN;
+            const int m = m0 + q * 32 + lane;
+            RowNorm rn;
+            if (ea.ss_in && m < M) rn.rinv = deferred_rinv(ea, m);
+            bool ok = mbar_wait(&acc_full[a], use & 1, &abort_flag, lim);
+            ok = __all_sync(0xffffffffu, ok) && abort_flag == 0;
+            if (!ok) { abort_flag = 1; break; }
+            tc_fence_after();
+            const uint32_t lane_base = tmem + a * BN + ((uint32_t)(q * 32) << 16);
+            if (epi == Epi::LsePart) {
+                lse_row<BN>(ea, lane_base, m, M, n0, N, tn);
+            } else {
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 16) {
+                    float v[16];
+                    tmem_ld16(lane_base + c, v);
+                    const int n = n0 + c;
+                    if (m < M && n < N) {
+                        rn.scale(ea, v);
+                        rn.add(epi, ea, m, n, N, epilogue16(epi, ea, m, n, min(16, N - n), v));
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[a]);
+        }
+    }
+    __syncwarp();
+    // a role that gave up raised abort_flag before this barrier
+    const bool ok = __syncthreads_and(1) && abort_flag == 0;
+    if (!ok && threadIdx.x == 0) {
+        raise_flag(hdr, ERR_TIMEOUT);
+        for (int it = armed > STAGES ? armed - STAGES : 0; it < armed; ++it)
+            mbar_wait(&full[it % STAGES], (it / STAGES) & 1, nullptr, lim);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ACC_COLS));
     }
 }
 
@@ -540,6 +708,26 @@ cudaError_t run_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int
     }
 }
 
+// The persistent kernel for grids of more than one wave: one CTA per SM.
+template <int BN, int STAGES>
+cudaError_t run_tc_pers(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
+                        const EpiArgs& ea, DevHeader* hdr) {
+    using S = TcShape<BN, STAGES, 1>;
+    constexpr int SMEM = STAGES * S::STAGE_BYTES + 1024 + 256;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(k_gemm_tc_pers<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             SMEM);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    CUtensorMap ta, tw;
+    if (!cached_map(&ta, A, M, K, lda, BM) || !cached_map(&tw, W, N, K, K, BN)) return cudaErrorInvalidValue;
+    const long long tiles = (long long)((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const unsigned grid = (unsigned)(tiles < sm_count() ? tiles : sm_count());
+    return launch_k(L, k_gemm_tc_pers<BN, STAGES>, grid, 192, SMEM, ta, tw, M, N, K, epi, ea, hdr);
+}
+
 // Tile variants: (BN, stages, k-split over a cluster) and how many CTAs fit on one SM.
 struct TcVariant {
     int bn, stages, per_sm, split;
@@ -624,20 +812,30 @@ bool gemm_tc_supported(const void* A, int lda, const void* W, int K) {
            (lda % 8 == 0) && (K % 8 == 0) && encode_fn() != nullptr;
 }
 
+// Whether a 128 x 256 grid of this shape takes more than one wave (the persistent kernel's case).
+bool multi_wave_256(int M, int N) {
+    return (long long)((M + BM - 1) / BM) * ((N + 255) / 256) > sm_count();
+}
+
 cudaError_t launch_gemm_tc_lse(Launch L, const bf16* A, int lda, const bf16* W, int M, int N, int K, EpiArgs ea,
                                DevHeader* hdr, int* n_tiles) {
     int v = pick_variant(M, N, K);
     if (VARIANTS[v].split > 1) v = 4;                 // the fused head needs whole rows per CTA
     ea.lse_ld = (N + VARIANTS[v].bn - 1) / VARIANTS[v].bn;
     *n_tiles = ea.lse_ld;
+    if (v == 4 && multi_wave_256(M, N)) return run_tc_pers<256, 4>(L, Epi::LsePart, A, lda, W, M, N, K, ea, hdr);
     return run_variant(v, L, Epi::LsePart, A, lda, W, M, N, K, ea, hdr);
 }
 
 cudaError_t launch_gemm_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                            const EpiArgs& ea, DevHeader* hdr, int variant) {
+    if (variant == PERSISTENT_VARIANT) return run_tc_pers<256, 4>(L, epi, A, lda, W, M, N, K, ea, hdr);
     int v = (variant >= 0 && variant < N_VARIANTS) ? variant : pick_variant(M, N, K);
     // a merge's deferred-norm group spans 32 GEMM columns and must stay in one column band
     if (epi == Epi::Merge && ea.norm_y && VARIANTS[v].split > 1 && VARIANTS[v].bn / VARIANTS[v].split < 32) v = 7;
+    // grids of several waves of the widest tile run persistently (epilogue overlapped)
+    if (variant < 0 && v == 4 && L.persistent && multi_wave_256(M, N))
+        return run_tc_pers<256, 4>(L, epi, A, lda, W, M, N, K, ea, hdr);
     return run_variant(v, L, epi, A, lda, W, M, N, K, ea, hdr);
 }
 

@@ -216,6 +216,15 @@ bool gemv_shape_supported(int M, int N, int K, int lda) {
     return gv_rows_per_cta(N) <= GV_MAX_ROWS;
 }
 
+// Measured on B200 against the few-row tensor-core kernel (single launches, weights from HBM):
+// faster where the weight matrix gives every SM at least one 32-row block and rows are short
+// (1 x 32768 x 2048: 37 vs 52 us; 1 x 8192 x 1024: 8.9 vs 10.2; 1 x 6144 x 2048: 10.9 vs 11.8),
+// slower where a few dozen CTAs each stream long rows (1 x 2048 x 2048: 9.7 vs 5.4;
+// 1 x 2048 x 5632: 18.5 vs 9.6; 4 x 2048 x 2048: 21.5 vs 5.5).
+bool gemv_preferred(int M, int N, int K) {
+    return gemv_shape_supported(M, N, K, K) && N >= 32 * sm_count() && K <= 2048;
+}
+
 bool gemv_supported(int M, int N, int K, int lda, const void* A, const void* W) {
     return gemv_shape_supported(M, N, K, lda) && reinterpret_cast<uintptr_t>(A) % 16 == 0 &&
            reinterpret_cast<uintptr_t>(W) % 16 == 0;

@@ -21,6 +21,8 @@ struct Launch {
     // Projections with at most this many rows of A run on the weight-streaming CUDA-core kernel
     // (gemv.cu) when its shape rules hold (0: never).
     int gemv_max_rows = 0;
+    // Grids of several waves of 128 x 256 tiles run on the persistent row-tile kernel.
+    bool persistent = true;
 };
 
 // Number of SMs of the current device (queried once per process).
@@ -185,6 +187,8 @@ cudaError_t launch_gemm_simt(Launch L, Epi epi, const T* A, int lda, const T* W,
 // ------------------------------------------------------------------ gemm_tc.cu
 bool gemm_tc_supported(const void* A, int lda, const void* W, int K);
 int gemm_tc_variants();
+// launch_gemm_tc's variant id of the persistent 128 x 256 kernel (two TMEM accumulators)
+constexpr int PERSISTENT_VARIANT = 100;
 // the row-tile variant the library picks for an M x N x K product (host logic only)
 int gemm_tc_pick(int M, int N, int K);
 // variant < 0: pick the tile shape from (M, N); otherwise force tile variant `variant`.
@@ -212,6 +216,8 @@ cudaError_t launch_gemm_swap(Launch L, Epi epi, const bf16* A, int lda, const bf
 // before the programmatic-launch wait), the same fused epilogues.  Shape rules: N a multiple of
 // 32, K a multiple of 8 and at most 6144, 16-byte aligned operands.
 bool gemv_shape_supported(int M, int N, int K, int lda);
+// the shapes where it measured faster than the few-row tensor-core kernel
+bool gemv_preferred(int M, int N, int K);
 bool gemv_supported(int M, int N, int K, int lda, const void* A, const void* W);
 cudaError_t launch_gemv(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                         const EpiArgs& ea, DevHeader* hdr);
@@ -220,10 +226,13 @@ cudaError_t launch_gemv(Launch L, Epi epi, const bf16* A, int lda, const bf16* W
 // Decoder sliding-window self-attention for one layer: sequence b is at step t = pos[b] + 1
 // (clamped to 1 .. max_t): RoPE at position t-1 (rows of the rotary table `rope`) on q/k from
 // qkv [B, 3d]; attends over the min(t-1, W-1) cached entries plus the current token; then
-// stores k_t, v_t into ring slot (t-1) mod (W-1).
+// stores k_t, v_t into ring slot (t-1) mod (W-1).  With n_splits > 1 the cached entries of
+// each (b, h) are cut into n_splits ranges, one CTA each, whose partials (in `part`, as for
+// the cross-attention) a combine kernel merges.
 template <typename T>
 cudaError_t launch_swa_decode(Launch L, const float* qkv, const float2* rope, T* ring, T* o,
-                              int B, int H, int hd, int W, const int32_t* pos, int max_t);
+                              int B, int H, int hd, int W, const int32_t* pos, int max_t,
+                              int n_splits = 1, float* part = nullptr);
 // Decoder cross-attention over M_{<=t} (positions 0..t-1) of one memory group: keys of
 // (b, h) at Mg + (b*H + h)*T_alloc*hd, values `plane` elements further.  With pos (device,
 // [B]) sequence b reads only positions 0..pos[b] (at most t).  Splits the keys of each (b, h)

@@ -1,5 +1,6 @@
 // C ABI of the RLT library (declared in include/rlt.h): model arena layout, weight
 // packing, the decoder-state registry and the encode / decode-step / replay drivers.
+#include <algorithm>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -27,7 +28,7 @@ constexpr int GROUP_MIN_ROWS = 256;
 // Cross-attention key-split partials: capacity in (sequence, head, split) work items.
 constexpr long long XATTN_PART_ITEMS = 32768;
 constexpr int XATTN_MAX_SPLITS = 64;
-constexpr int XATTN_MIN_CHUNK = 64;
+constexpr int XATTN_MIN_CHUNK = 32;
 constexpr long long XATTN_TARGET_WARPS = 148LL * 64 * 2;
 
 struct Layout {
@@ -172,6 +173,7 @@ struct rlt_model {
     int opt_attn_cap = 0;               // resident attention CTAs per SM (0: no cap)
     int opt_group_pdl = 0;              // programmatic dependent launch inside a group's chain
     int opt_gemv_rows = 4;              // projections of at most this many rows stream on CUDA cores
+    int opt_persistent = 1;             // grids of several waves of 128 x 256 tiles run persistently
     // two row groups: library-owned streams, forked from and joined back to the caller's stream
     cudaStream_t gs[2] = {nullptr, nullptr};
     cudaEvent_t fork_ev = nullptr, join_ev[2] = {nullptr, nullptr};
@@ -201,6 +203,7 @@ struct rlt_model {
     Launch launch(void* stream) {
         Launch L{reinterpret_cast<cudaStream_t>(stream), &launches};
         L.gemv_max_rows = opt_gemv_rows;
+        L.persistent = opt_persistent != 0;
         return L;
     }
 
@@ -320,6 +323,18 @@ DecWS dec_ws(const rlt_config& c, int B) {
     w.ss = take((size_t)B * (d / 16) * 4);        // its 16-column sum-of-squares partials
     w.total = off;
     return w;
+}
+
+// Key splits of the decoder's sliding-window attention: one CTA per (sequence, head) fills
+// the GPU at large batches; below ~6 CTAs per SM the window is cut into ranges of at least 32
+// cached entries, one CTA each.
+int swa_splits(const rlt_config& c, int B, int t) {
+    const long long bh = (long long)B * c.n_heads;
+    const int n = std::min(t - 1, c.W - 1);
+    const long long want = (148LL * 6 + bh - 1) / bh;
+    long long s = std::min<long long>(want, (n + 31) / 32);
+    s = std::min<long long>(s, std::min<long long>(16, XATTN_PART_ITEMS / bh));
+    return s < 1 ? 1 : (int)s;
 }
 
 int xattn_splits(const rlt_config& c, int B, int t) {
@@ -564,7 +579,7 @@ rlt_status step_rows(rlt_model* m, uint8_t* state, int B, int b0, int Bg, const 
         norm_in(ea);
         CKP(RLT_K_QKV, launch_gemm<T>(L, Epi::StoreF32, hin, d, m->at<T>(m->lay.wqkv[l]), Bg, 3 * d, d, ea));
         CKP(RLT_K_SWA, launch_swa_decode<T>(L, qkv, rope, ring + (size_t)l * ring_layer_elems(c, B), att, Bg, H,
-                                            hd, c.W, pos, t));
+                                            hd, c.W, pos, t, swa_splits(c, Bg, t), part));
         ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = x; ea.ld_out = d;
         norm_out(ea, m->at<float>(m->lay.xattn_norm[l]));
         CKP(RLT_K_O, launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.wo[l]), Bg, d, d, ea));
@@ -1216,6 +1231,9 @@ rlt_status rlt_set_option(rlt_model* m, const char* name, int64_t value) {
     } else if (n == "attn_ctas_per_sm") {
         if (value < 0 || value > 32) return RLT_EINVAL;
         m->opt_attn_cap = (int)value;
+    } else if (n == "persistent_gemm") {
+        if (value < 0 || value > 1) return RLT_EINVAL;
+        m->opt_persistent = (int)value;
     } else if (n == "gemv_rows") {
         if (value < 0 || value > 4) return RLT_EINVAL;
         m->opt_gemv_rows = (int)value;
@@ -1230,7 +1248,7 @@ rlt_status rlt_set_option(rlt_model* m, const char* name, int64_t value) {
 
 int rlt_gemm_plan(int M, int N, int K) {
     if (M < 1 || N < 1 || K < 1) return -1;
-    if (gemv_shape_supported(M, N, K, K)) return 16;
+    if (gemv_preferred(M, N, K)) return 16;
     if (gemm_swap_preferred(M, N, K)) {
         const int s = gemm_swap_auto_split(M, N, K);
         return 11 + (s == 1 ? 1 : (s == 2 ? 2 : (s == 4 ? 3 : 4)));
@@ -1241,7 +1259,7 @@ int rlt_gemm_plan(int M, int N, int K) {
 rlt_status rlt_gemm_bf16(rlt_model* m, const void* A, const void* W, float* C, int M, int N, int K, int kernel,
                          void* stream) {
     const int n_tc = gemm_tc_variants();
-    if (!m || !A || !W || !C || M < 1 || N < 1 || K < 1 || kernel < 0 || kernel > 2 + n_tc + 5) return RLT_EINVAL;
+    if (!m || !A || !W || !C || M < 1 || N < 1 || K < 1 || kernel < 0 || kernel > 3 + n_tc + 5) return RLT_EINVAL;
     if (kernel > 1 + n_tc && kernel <= 1 + n_tc + 5 && !gemm_swap_supported(M)) return RLT_EINVAL;
     if (kernel == 2 + n_tc + 5 && !gemv_supported(M, N, K, K, A, W)) return RLT_EINVAL;
     if (!aligned(A, 16) || !aligned(W, 16) || !aligned(C, 16) || K % 8 || N % 4) return RLT_EINVAL;
@@ -1261,8 +1279,10 @@ rlt_status rlt_gemm_bf16(rlt_model* m, const void* A, const void* W, float* C, i
     } else if (kernel <= 1 + n_tc + 5) {
         static const int splits[5] = {0, 1, 2, 4, 8};
         CK(launch_gemm_swap(L, Epi::StoreF32, a, K, w, M, N, K, ea, m->hdr(), splits[kernel - 2 - n_tc]));
-    } else {
+    } else if (kernel == 2 + n_tc + 5) {
         CK(launch_gemv(L, Epi::StoreF32, a, K, w, M, N, K, ea, m->hdr()));
+    } else {
+        CK(launch_gemm_tc(L, Epi::StoreF32, a, K, w, M, N, K, ea, m->hdr(), PERSISTENT_VARIANT));
     }
     return RLT_OK;
 }

@@ -340,10 +340,15 @@ uint64_t rlt_launch_count(const rlt_model* m);
  *                        (0, the default: none), leaving room on every SM for projection CTAs
  *                        that start early (programmatic launch) or run on the other group's
  *                        stream.
+ *   "persistent_gemm"    1 (default): projections whose grid of 128 x 256 tiles exceeds one
+ *                        wave run on the persistent kernel (rlt_gemm_bf16 kernel 17); 0: one
+ *                        CTA per tile.
  *   "gemv_rows"          projections of at most this many rows (0..4, default 4) run on the
  *                        weight-streaming CUDA-core kernel (bulk-copied weight rows requested
- *                        before the programmatic-launch wait) when its shape rules hold; 0 keeps
- *                        them on the few-row tensor-core kernel.
+ *                        before the programmatic-launch wait) on the shapes where it measured
+ *                        faster than the few-row tensor-core kernel (at least one 32-row block
+ *                        of weights per SM, K <= 2048); 0 keeps every projection on the few-row
+ *                        kernel.
  *   "group_pdl"          1: programmatic dependent launch inside each row group's chain
  *                        (default 0: an early-launched kernel would hold SM resources the
  *                        other group needs).
@@ -362,7 +367,10 @@ rlt_status rlt_set_option(rlt_model* m, const char* name, int64_t value);
  * split 2; 8: 128x64 split 4), kernel 11 + s (M <= 64 only) = the few-row kernel with the
  * weights on the MMA's M side and K split over a cluster of (s = 0: chosen, 1: 1, 2: 2, 3: 4,
  * 4: 8) CTAs, kernel 16 (M <= 4, N a multiple of 32, K <= 6144) = the weight-streaming
- * CUDA-core kernel.  A, W, C 16-byte aligned, K a multiple of 8, N a multiple of 4.
+ * CUDA-core kernel, kernel 17 = the persistent row-tile kernel (128x256 tiles, one CTA per SM
+ * walking the tiles, two tensor-memory accumulators so that a tile's epilogue overlaps the next
+ * tile's MMAs; the library's choice for grids of more than one wave).  A, W, C 16-byte aligned,
+ * K a multiple of 8, N a multiple of 4.
  * Errors: RLT_EINVAL, RLT_ECUDA; a tensor-core wait that times out latches
  * RLT_ETIMEOUT (rlt_last_error). */
 rlt_status rlt_gemm_bf16(rlt_model* m, const void* A, const void* W, float* C, int M, int N, int K,

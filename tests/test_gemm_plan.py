@@ -27,9 +27,10 @@ PLANS = [
     ((32, 2048, 2048), 14, "<= 32 rows: few-row kernel, split 4"),
     ((32, 6144, 2048), 13, "q/k/v at B=32"),
     ((32, 2048, 5632), 14, "down at B=32"),
-    ((1, 2048, 2048), 16, "B=1: weight-streaming kernel"),
-    ((1, 11264, 2048), 16, "gate/up at B=1"),
-    ((4, 2048, 5632), 16, "down at B=4"),
+    ((1, 2048, 2048), 14, "B=1, narrow output: few-row kernel, split 4 (the weight-streaming kernel measured slower)"),
+    ((1, 11264, 2048), 16, "gate/up at B=1: every SM gets weight rows, weight-streaming kernel"),
+    ((1, 32768, 2048), 16, "LM head at B=1"),
+    ((4, 2048, 5632), 14, "down at B=4: long rows, few-row kernel"),
     ((5, 2048, 2048), 14, "five rows: few-row tensor-core kernel"),
     ((1, 2048, 8192), 14, "K above the weight-streaming kernel's ring: few-row kernel"),
     # small shapes and the encoder

@@ -25,6 +25,7 @@ SHAPES = [
     (2, 6144, 2048),      # weight-streaming kernel: two rows
     (4, 11264, 5632),     # four rows, the widest K it takes
     (1, 32000, 1024),     # LM head of the 300M-class model at B=1
+    (2000, 3000, 520),    # persistent kernel: ragged M, N and K over several waves
 ]
 
 
@@ -33,7 +34,7 @@ def model():
     return build_model(TINY.model, max_pos=8)
 
 
-@pytest.mark.parametrize("kernel", [0, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13, 14, 15, 16])
+@pytest.mark.parametrize("kernel", [0, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13, 14, 15, 16, 17])
 @pytest.mark.parametrize("M,N,K", SHAPES)
 def test_tcgen05_gemm_matches_float64(model, M, N, K, kernel):
     if kernel >= 11 and M > 64:
@@ -55,7 +56,7 @@ def test_tcgen05_gemm_matches_float64(model, M, N, K, kernel):
         assert bool(((c_simt - ref).abs() <= 1e-4 * bound + 1e-6).all())
 
 
-@pytest.mark.parametrize("kernel", [0, 7, 8, 9, 10, 14, 15])
+@pytest.mark.parametrize("kernel", [0, 7, 8, 9, 10, 14, 15, 17])
 def test_tcgen05_gemm_is_deterministic(model, kernel):
     g = torch.Generator().manual_seed(5)
     A = torch.randn(512 if kernel < 11 else 64, 1024, generator=g).to(torch.bfloat16)

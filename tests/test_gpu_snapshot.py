@@ -71,8 +71,8 @@ def test_rows_loaded_from_snapshots_at_different_positions_follow_the_oracle(nam
     # a batch of three rows: row 0 <- sequence 1 (t=5), row 1 <- sequence 0 (t=13), row 2 fresh
     rows = np.stack([seqs[1], seqs[0], seqs[2]])
     bt = Batch(model, rows, P=1)
-    model.snapshot_load(snaps[0], bt.st, 0, bt.M, bt.cache, T)
-    model.snapshot_load(snaps[1], bt.st, 1, bt.M, bt.cache, T)
+    model.snapshot_load(snaps[1], bt.st, 0, bt.M, bt.cache, T)    # sequence 1 at t = 5
+    model.snapshot_load(snaps[0], bt.st, 1, bt.M, bt.cache, T)    # sequence 0 at t = 13
     assert bt.st.positions() == [5, 13, 0]
     got_lp, got_s, got_pos = [], [], []
     for _ in range(20):
