@@ -84,6 +84,9 @@ def kind_cost(kind: str, m, B: int, T: int) -> tuple[str, float]:
         return "hbm", float(T * n * B * d * (4 + bw))
     if kind == "lse":
         return "hbm", float((T - 1) * B * V * 4)
+    if kind == "small_step":
+        # one launch per step: the step's algorithmic bytes (weights, window, memory, e_t)
+        return "hbm", float(sum(step_cost(m, B, int(t))[0] for t in ts))
     return "hbm", 0.0
 
 

@@ -255,6 +255,56 @@ int sample_max_vocab();
 cudaError_t launch_sample(Launch L, const float* logp, int B, int V, const float* u, int top_k, float top_p,
                           int32_t* tok, int tok_stride, float* blp);
 
+// ------------------------------------------------------------------ small_step.cu
+// The whole decoder step of a small model in one launch, one CTA per sequence.
+constexpr int SS_MAX_LAYERS = 8;
+struct DecWeights {             // device pointers into the weight arena (matrices in storage type)
+    const void* merge;          // [2d, 2d], rows 2j / 2j+1 = gate_j / feedback_j
+    const float* merge_b;
+    const float* dec_norm;
+    const void* unembed;        // [V, d]
+    const float* attn_norm[SS_MAX_LAYERS];
+    const float* xattn_norm[SS_MAX_LAYERS];
+    const float* ffn_norm[SS_MAX_LAYERS];
+    const void* wqkv[SS_MAX_LAYERS];
+    const void* wo[SS_MAX_LAYERS];
+    const void* wqc[SS_MAX_LAYERS];
+    const void* woc[SS_MAX_LAYERS];
+    const void* wgu[SS_MAX_LAYERS];     // [2F, d], rows 2j / 2j+1 = gate_j / up_j
+    const void* wdown[SS_MAX_LAYERS];
+};
+struct SmallStepArgs {
+    int B, d, H, F, V, W, G, L;
+    float eps, tau;
+    const void* e;              // [B, T_alloc, d]
+    int T_alloc;
+    const void* M;              // [G][2][B][H][T_alloc][hd]
+    long long plane;            // keys -> values of one memory group
+    size_t group_elems;
+    float* s;                   // state s [B, d]
+    void* ring;                 // state ring [L][B][2][H][W-1][hd]
+    size_t ring_layer;          // elements per layer of the ring
+    int32_t* pos;               // state positions [B]
+    StateHeader* sh;
+    int t_host;                 // the largest step of the batch (the header's t)
+    uint64_t version;
+    DevHeader* hdr;
+    const float2* rope;
+    DecWeights w;
+    bool head;
+    const int32_t* tok;
+    int tok_stride;
+    float* logp_tok;
+    int lp_stride;
+    float* lse;
+    float* logp_full;
+    float* score;
+    const int32_t* prompt_len;
+};
+bool small_step_supported(int d, int F, int V, int hd, int L);
+template <typename T>
+cudaError_t launch_small_step(Launch L, const SmallStepArgs& a, int hd);
+
 // ------------------------------------------------------------------ attention_tc.cu
 // Tensor-core encoder attention (bf16, head_dim 64 or 128): q, k planes [B][H][T][hd] and the
 // transposed values vt [B][H][hd][enc_vt_pitch(T)] -> o [B*T, d].

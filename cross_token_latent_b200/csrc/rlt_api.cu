@@ -174,6 +174,7 @@ struct rlt_model {
     int opt_group_pdl = 0;              // programmatic dependent launch inside a group's chain
     int opt_gemv_rows = 4;              // projections of at most this many rows stream on CUDA cores
     int opt_persistent = 1;             // grids of several waves of 128 x 256 tiles run persistently
+    int opt_small_step = 1;             // small models: the whole step in one launch
     // two row groups: library-owned streams, forked from and joined back to the caller's stream
     cudaStream_t gs[2] = {nullptr, nullptr};
     cudaEvent_t fork_ev = nullptr, join_ev[2] = {nullptr, nullptr};
@@ -639,9 +640,51 @@ rlt_status step_rows(rlt_model* m, uint8_t* state, int B, int b0, int Bg, const 
 // attention streams HBM, the other group's projections run on the tensor cores.  The
 // attention grids of both groups are capped so that every SM keeps room for the other
 // group's GEMM CTAs.
+// A small model's whole step in one launch (small_step.cu): one CTA per sequence.
+template <typename T>
+rlt_status small_step(rlt_model* m, uint8_t* state, int B, const T* e, const T* M, int T_alloc, int t,
+                      const StepIO& io, cudaStream_t st) {
+    const rlt_config& c = m->cfg;
+    const Layout& y = m->lay;
+    SmallStepArgs a = {};
+    a.B = B; a.d = c.d; a.H = c.n_heads; a.F = c.F; a.V = c.V; a.W = c.W; a.G = c.G; a.L = c.L_D;
+    a.eps = c.rms_eps; a.tau = io.tau;
+    a.e = e; a.T_alloc = T_alloc; a.M = M;
+    a.plane = (long long)B * c.n_heads * T_alloc * c.head_dim;
+    a.group_elems = (size_t)2 * B * c.n_heads * (size_t)T_alloc * c.head_dim;
+    a.s = reinterpret_cast<float*>(state + state_s_off());
+    a.ring = state + state_ring_off(c, B);
+    a.ring_layer = ring_layer_elems(c, B);
+    a.pos = state_pos(c, state, B);
+    a.sh = reinterpret_cast<StateHeader*>(state);
+    a.t_host = t;
+    a.version = m->version;
+    a.hdr = m->hdr();
+    a.rope = m->at<float2>(y.rope);
+    a.w.merge = m->at<T>(y.merge_w); a.w.merge_b = m->at<float>(y.merge_b);
+    a.w.dec_norm = m->at<float>(y.dec_norm); a.w.unembed = m->at<T>(y.unembed);
+    for (int l = 0; l < c.L_D; ++l) {
+        a.w.attn_norm[l] = m->at<float>(y.attn_norm[l]);
+        a.w.xattn_norm[l] = m->at<float>(y.xattn_norm[l]);
+        a.w.ffn_norm[l] = m->at<float>(y.ffn_norm[l]);
+        a.w.wqkv[l] = m->at<T>(y.wqkv[l]); a.w.wo[l] = m->at<T>(y.wo[l]);
+        a.w.wqc[l] = m->at<T>(y.wqc[l]); a.w.woc[l] = m->at<T>(y.woc[l]);
+        a.w.wgu[l] = m->at<T>(y.wgu[l]); a.w.wdown[l] = m->at<T>(y.wdown[l]);
+    }
+    a.head = io.head;
+    a.tok = io.tok; a.tok_stride = io.tok_stride; a.logp_tok = io.logp_tok; a.lp_stride = io.lp_stride;
+    a.lse = io.lse; a.logp_full = io.logp_full; a.score = io.score; a.prompt_len = io.prompt_len;
+    Launch L = m->launch(st);
+    CKP(RLT_K_SMALL_STEP, launch_small_step<T>(L, a, c.head_dim));
+    return RLT_OK;
+}
+
 template <typename T>
 rlt_status step_impl(rlt_model* m, uint8_t* state, int B, const T* e, const T* M, int T_alloc, int t,
                      const StepIO& io, uint8_t* ws, cudaStream_t st) {
+    const rlt_config& c = m->cfg;
+    if (m->opt_small_step && small_step_supported(c.d, c.F, c.V, c.head_dim, c.L_D))
+        return small_step<T>(m, state, B, e, M, T_alloc, t, io, st);
     DecWS w = dec_ws(m->cfg, B);
     float* part = reinterpret_cast<float*>(ws + w.part);
     if (m->row_groups(B) == 1 || !m->group_streams()) {
@@ -1231,6 +1274,9 @@ rlt_status rlt_set_option(rlt_model* m, const char* name, int64_t value) {
     } else if (n == "attn_ctas_per_sm") {
         if (value < 0 || value > 32) return RLT_EINVAL;
         m->opt_attn_cap = (int)value;
+    } else if (n == "small_step") {
+        if (value < 0 || value > 1) return RLT_EINVAL;
+        m->opt_small_step = (int)value;
     } else if (n == "persistent_gemm") {
         if (value < 0 || value > 1) return RLT_EINVAL;
         m->opt_persistent = (int)value;

@@ -340,6 +340,10 @@ uint64_t rlt_launch_count(const rlt_model* m);
  *                        (0, the default: none), leaving room on every SM for projection CTAs
  *                        that start early (programmatic launch) or run on the other group's
  *                        stream.
+ *   "small_step"         1 (default): a model with d <= 256, F <= 1024, V <= 8192, head_dim
+ *                        16 or 32 and at most 8 layers runs each decoder step as one launch,
+ *                        one CTA per sequence (its weights stay in L2); 0: the per-sublayer
+ *                        kernels.
  *   "persistent_gemm"    1 (default): projections whose grid of 128 x 256 tiles exceeds one
  *                        wave run on the persistent kernel (rlt_gemm_bf16 kernel 17); 0: one
  *                        CTA per tile.
@@ -414,7 +418,8 @@ enum {
     RLT_K_HEAD = 11,     /* LM-head projection                                           */
     RLT_K_LSE = 12,      /* log-sum-exp + gather + score                                 */
     RLT_K_ENCODER = 13,  /* a whole rlt_encode call                                      */
-    RLT_K_COUNT = 14
+    RLT_K_SMALL_STEP = 14, /* a small model's whole decoder step in one launch           */
+    RLT_K_COUNT = 15
 };
 
 /* Start recording a CUDA event pair on the launch stream around every launch of the kinds
