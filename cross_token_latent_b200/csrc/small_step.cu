@@ -13,8 +13,9 @@
 // attention outputs, SiLU(g) * u and s fed to the merge and the head are rounded likewise;
 // decoder queries, softmax, the residual stream, s_t and log-probabilities stay float32.
 // Projections are warp-per-output-row dot products over rows of W read from L2 (16-byte
-// loads) against the input vector in shared memory.  Attention runs one warp per head, one
-// key per lane, with the head's online softmax merged across lanes (head_dim 16 or 32).
+// loads) against the input vector in shared memory.  Attention gives every head
+// SS_WARPS / n_heads warps, one key per lane, whose online-softmax states are merged through
+// shared memory (head_dim 16 or 32).
 #include "kernels.cuh"
 
 namespace rlt {
@@ -26,23 +27,44 @@ constexpr int SS_WARPS = SS_THREADS / 32;
 constexpr int SS_MAX_D = 256, SS_MAX_F = 1024, SS_MAX_V = 8192;
 
 // y[n] = sum_k W[n, k] x[k] for n < N (W row-major [N, K] in storage type, x float in shared
-// memory); one warp per row, lanes over 16-byte pieces of the row.
+// memory).  A row is split over a group of lpr lanes (lpr = the power of two <= K/8 up to 32,
+// 16-byte pieces each), a warp works on 32/lpr rows per pass and GV_U passes at once, so that
+// several independent row loads are in flight per lane; the group reduces by shuffles.
 template <typename T>
 __device__ __forceinline__ void gemv_rows(const T* __restrict__ W, int N, int K, const float* x, float* y) {
     constexpr int EPL = Vec16<T>::N;
+    constexpr int U = 4;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nv = K / EPL;
-    for (int n = warp; n < N; n += SS_WARPS) {
-        const uint4* wr = reinterpret_cast<const uint4*>(W + (size_t)n * K);
-        float acc = 0.f;
-        for (int v = lane; v < nv; v += 32) {
-            float w[EPL];
-            Vec16<T>::unpack(__ldg(wr + v), w);
+    int lpr = 32;
+    while (lpr > 1 && lpr > nv) lpr >>= 1;
+    const int rpp = 32 / lpr, sub = lane / lpr, li = lane % lpr;
+    for (int base = warp * rpp * U; base < N; base += SS_WARPS * rpp * U) {
+        float acc[U];
 #pragma unroll
-            for (int i = 0; i < EPL; ++i) acc = fmaf(w[i], x[v * EPL + i], acc);
+        for (int u = 0; u < U; ++u) acc[u] = 0.f;
+        for (int v = li; v < nv; v += lpr) {
+            uint4 wv[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int n = base + u * rpp + sub;
+                wv[u] = n < N ? __ldg(reinterpret_cast<const uint4*>(W + (size_t)n * K) + v) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                float w[EPL];
+                Vec16<T>::unpack(wv[u], w);
+#pragma unroll
+                for (int i = 0; i < EPL; ++i) acc[u] = fmaf(w[i], x[v * EPL + i], acc[u]);
+            }
         }
-        acc = warp_sum(acc);
-        if (lane == 0) y[n] = acc;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            float a = acc[u];
+            for (int o = lpr / 2; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+            const int n = base + u * rpp + sub;
+            if (li == 0 && n < N) y[n] = a;
+        }
     }
 }
 
@@ -64,16 +86,18 @@ __device__ __forceinline__ void norm_round(const float* x, int d, const float* _
     __syncthreads();
 }
 
-// One warp's attention of query q (float, HD, already scaled by log2(e)/sqrt(hd)) over n keys
-// K[j*HD ..], V[j*HD ..] (storage type) plus, optionally, one extra key/value in float (the
-// current token): lanes take keys j = lane, lane + 32, ...; returns the output in out[HD] on
-// every lane of the warp.
+// Partial softmax state of one warp over its keys: lanes take keys j = j0 + lane, j0 + lane +
+// stride, ... (< n) of K, V (storage type, row stride HD), q float (already scaled by
+// log2(e)/sqrt(hd)); optionally one extra key/value in float (the current token) folded in by
+// lane 0.  On return every lane holds the warp's (m, l, acc).
 template <typename T, int HD>
-__device__ __forceinline__ void warp_attend(const float* q, const T* __restrict__ K, const T* __restrict__ V, int n,
-                                            const float* kx, const float* vx, float* out) {
+__device__ __forceinline__ void warp_partial(const float* q, const T* __restrict__ K, const T* __restrict__ V, int j0,
+                                             int n, int stride, const float* kx, const float* vx, float& m, float& l,
+                                             float* acc) {
     const int lane = threadIdx.x & 31;
     constexpr int EPL = Vec16<T>::N;
-    float m = -1e30f, l = 0.f, acc[HD];
+    m = -1e30f;
+    l = 0.f;
 #pragma unroll
     for (int i = 0; i < HD; ++i) acc[i] = 0.f;
     auto fold = [&](float s, const float* vrow) {
@@ -84,7 +108,7 @@ __device__ __forceinline__ void warp_attend(const float* q, const T* __restrict_
         for (int i = 0; i < HD; ++i) acc[i] = acc[i] * c + p * vrow[i];
         m = mx;
     };
-    for (int j = lane; j < n; j += 32) {
+    for (int j = j0 + lane; j < n; j += stride) {
         float r[HD];
 #pragma unroll
         for (int v = 0; v < HD / EPL; ++v) Vec16<T>::unpack(ld16(K + (size_t)j * HD + v * EPL), r + v * EPL);
@@ -101,7 +125,6 @@ __device__ __forceinline__ void warp_attend(const float* q, const T* __restrict_
         for (int i = 0; i < HD; ++i) s = fmaf(q[i], kx[i], s);
         fold(s, vx);
     }
-    // merge the lanes' running states
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         const float mo = __shfl_xor_sync(0xffffffffu, m, o), lo = __shfl_xor_sync(0xffffffffu, l, o);
@@ -112,9 +135,30 @@ __device__ __forceinline__ void warp_attend(const float* q, const T* __restrict_
         for (int i = 0; i < HD; ++i) acc[i] = acc[i] * c1 + __shfl_xor_sync(0xffffffffu, acc[i], o) * c2;
         m = mx;
     }
-    const float inv = 1.0f / l;
-#pragma unroll
-    for (int i = 0; i < HD; ++i) out[i] = acc[i] * inv;
+}
+
+// Shared scratch of the per-head attention: each warp's partial state.
+template <int HD>
+struct AttnScratch {
+    float m[SS_WARPS], l[SS_WARPS];
+    float acc[SS_WARPS][HD];
+};
+
+// Merge the partial states of head hh's wph warps (warps hh*wph .. hh*wph+wph-1) and write the
+// normalised output rounded to the storage type into out[hh*HD ..].  Called by the first warp
+// of the head after a __syncthreads.
+template <typename T, int HD>
+__device__ __forceinline__ void merge_head(const AttnScratch<HD>& sc, int hh, int wph, float* out) {
+    const int lane = threadIdx.x & 31;
+    float mx = -1e30f;
+    for (int w = 0; w < wph; ++w) mx = fmaxf(mx, sc.m[hh * wph + w]);
+    float L = 0.f;
+    for (int w = 0; w < wph; ++w) L += sc.l[hh * wph + w] * exp2f(sc.m[hh * wph + w] - mx);
+    for (int i = lane; i < HD; i += 32) {
+        float a = 0.f;
+        for (int w = 0; w < wph; ++w) a += sc.acc[hh * wph + w][i] * exp2f(sc.m[hh * wph + w] - mx);
+        out[hh * HD + i] = round_to<T>(a / L);
+    }
 }
 
 template <typename T, int HD>
@@ -124,12 +168,14 @@ __global__ void __launch_bounds__(SS_THREADS) k_small_step(SmallStepArgs a) {
     __shared__ float y[2 * SS_MAX_F > 3 * SS_MAX_D ? 2 * SS_MAX_F : 3 * SS_MAX_D];
     __shared__ float att[SS_MAX_D];
     __shared__ float red[SS_WARPS];
+    __shared__ AttnScratch<HD> sc;
     extern __shared__ float logits[];                // V floats
     pdl_wait();
     pdl_trigger();
     const int b = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int d = a.d, H = a.H, F = a.F, V = a.V, W = a.W, half = HD / 2;
+    const int wph = SS_WARPS / H;                    // warps per head (H <= 16)
     const float qscale = 1.4426950408889634f / sqrtf((float)HD);
     const DecWeights& w = a.w;
     auto mat = [](const void* p) { return static_cast<const T*>(p); };
@@ -165,31 +211,41 @@ __global__ void __launch_bounds__(SS_THREADS) k_small_step(SmallStepArgs a) {
         gemv_rows<T>(mat(w.wqkv[l]), 3 * d, d, h, y);
         __syncthreads();
         T* ring_l = static_cast<T*>(a.ring) + (size_t)l * a.ring_layer;
-        for (int hh = warp; hh < H; hh += SS_WARPS) {
-            float q[HD], k[HD], v[HD];
-#pragma unroll
-            for (int i = 0; i < HD; ++i) {
-                const int cp = i < half ? i + half : i - half;
-                const float2 cs = rope_row[i % half];
-                const float qa = y[hh * HD + i], qp = y[hh * HD + cp];
-                const float ka = y[d + hh * HD + i], kp = y[d + hh * HD + cp];
-                q[i] = (i < half ? qa * cs.x - qp * cs.y : qp * cs.y + qa * cs.x) * qscale;
-                k[i] = round_to<T>(i < half ? ka * cs.x - kp * cs.y : kp * cs.y + ka * cs.x);
-                v[i] = round_to<T>(y[2 * d + hh * HD + i]);
-            }
-            T* Kr = ring_l + (((size_t)b * 2 + 0) * H + hh) * (size_t)(W - 1) * HD;
-            T* Vr = ring_l + (((size_t)b * 2 + 1) * H + hh) * (size_t)(W - 1) * HD;
-            const int n = W > 1 ? min(t - 1, W - 1) : 0;
-            float o[HD];
-            warp_attend<T, HD>(q, Kr, Vr, n, k, v, o);
-            for (int i = lane; i < HD; i += 32) att[hh * HD + i] = round_to<T>(o[i]);
-            __syncwarp();
-            if (W > 1 && lane == 0) {                       // after the warp has read the slot
-                const int slot = (t - 1) % (W - 1);
+        {
+            // head hh = warp / wph; its wph warps split the cached entries, the first of them
+            // also attends to the current token and later writes it into the ring
+            const int hh = warp / wph, sub = warp % wph;
+            float q[HD], k[HD], v[HD], mm, ll, acc[HD];
+            T* Kr = nullptr;
+            T* Vr = nullptr;
+            if (hh < H) {
 #pragma unroll
                 for (int i = 0; i < HD; ++i) {
-                    Kr[(size_t)slot * HD + i] = from_f<T>(k[i]);
-                    Vr[(size_t)slot * HD + i] = from_f<T>(v[i]);
+                    const int cp = i < half ? i + half : i - half;
+                    const float2 cs = rope_row[i % half];
+                    const float qa = y[hh * HD + i], qp = y[hh * HD + cp];
+                    const float ka = y[d + hh * HD + i], kp = y[d + hh * HD + cp];
+                    q[i] = (i < half ? qa * cs.x - qp * cs.y : qp * cs.y + qa * cs.x) * qscale;
+                    k[i] = round_to<T>(i < half ? ka * cs.x - kp * cs.y : kp * cs.y + ka * cs.x);
+                    v[i] = round_to<T>(y[2 * d + hh * HD + i]);
+                }
+                Kr = ring_l + (((size_t)b * 2 + 0) * H + hh) * (size_t)(W - 1) * HD;
+                Vr = ring_l + (((size_t)b * 2 + 1) * H + hh) * (size_t)(W - 1) * HD;
+                const int n = W > 1 ? min(t - 1, W - 1) : 0;
+                warp_partial<T, HD>(q, Kr, Vr, sub * 32, n, wph * 32, sub == 0 ? k : nullptr, v, mm, ll, acc);
+                if (lane == 0) { sc.m[warp] = mm; sc.l[warp] = ll; }
+                for (int i = lane; i < HD; i += 32) sc.acc[warp][i] = acc[i];
+            }
+            __syncthreads();                            // every warp has read its ring entries
+            if (hh < H && sub == 0) {
+                merge_head<T, HD>(sc, hh, wph, att);
+                if (W > 1 && lane == 0) {
+                    const int slot = (t - 1) % (W - 1);
+#pragma unroll
+                    for (int i = 0; i < HD; ++i) {
+                        Kr[(size_t)slot * HD + i] = from_f<T>(k[i]);
+                        Vr[(size_t)slot * HD + i] = from_f<T>(v[i]);
+                    }
                 }
             }
         }
@@ -203,13 +259,19 @@ __global__ void __launch_bounds__(SS_THREADS) k_small_step(SmallStepArgs a) {
         gemv_rows<T>(mat(w.wqc[l]), d, d, h, y);
         __syncthreads();
         const T* Mg = static_cast<const T*>(a.M) + (a.G == 1 ? 0 : (size_t)l * a.group_elems);
-        for (int hh = warp; hh < H; hh += SS_WARPS) {
-            float q[HD], o[HD];
+        {
+            const int hh = warp / wph, sub = warp % wph;
+            if (hh < H) {
+                float q[HD], mm, ll, acc[HD];
 #pragma unroll
-            for (int i = 0; i < HD; ++i) q[i] = y[hh * HD + i] * qscale;
-            const T* Km = Mg + ((size_t)b * H + hh) * (size_t)a.T_alloc * HD;
-            warp_attend<T, HD>(q, Km, Km + a.plane, t, nullptr, nullptr, o);
-            for (int i = lane; i < HD; i += 32) att[hh * HD + i] = round_to<T>(o[i]);
+                for (int i = 0; i < HD; ++i) q[i] = y[hh * HD + i] * qscale;
+                const T* Km = Mg + ((size_t)b * H + hh) * (size_t)a.T_alloc * HD;
+                warp_partial<T, HD>(q, Km, Km + a.plane, sub * 32, t, wph * 32, nullptr, nullptr, mm, ll, acc);
+                if (lane == 0) { sc.m[warp] = mm; sc.l[warp] = ll; }
+                for (int i = lane; i < HD; i += 32) sc.acc[warp][i] = acc[i];
+            }
+            __syncthreads();
+            if (hh < H && sub == 0) merge_head<T, HD>(sc, hh, wph, att);
         }
         __syncthreads();
         gemv_rows<T>(mat(w.woc[l]), d, d, att, y);
@@ -283,7 +345,7 @@ __global__ void __launch_bounds__(SS_THREADS) k_small_step(SmallStepArgs a) {
 }  // namespace
 
 bool small_step_supported(int d, int F, int V, int hd, int L) {
-    return d <= SS_MAX_D && F <= SS_MAX_F && V <= SS_MAX_V && L <= SS_MAX_LAYERS && d % 8 == 0 &&
+    return d <= SS_MAX_D && F <= SS_MAX_F && V <= SS_MAX_V && L <= SS_MAX_LAYERS && d % 8 == 0 && d / hd <= SS_WARPS &&
            F % 8 == 0 && (hd == 16 || hd == 32);
 }
 
