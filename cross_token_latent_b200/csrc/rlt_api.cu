@@ -28,7 +28,7 @@ constexpr int GROUP_MIN_ROWS = 256;
 // Cross-attention key-split partials: capacity in (sequence, head, split) work items.
 constexpr long long XATTN_PART_ITEMS = 32768;
 constexpr int XATTN_MAX_SPLITS = 64;
-constexpr int XATTN_MIN_CHUNK = 32;
+constexpr int XATTN_MIN_CHUNK = 64;
 constexpr long long XATTN_TARGET_WARPS = 148LL * 64 * 2;
 
 struct Layout {
@@ -172,7 +172,7 @@ struct rlt_model {
     int opt_row_groups = 1;             // 1 one group, 2 two groups when B >= GROUP_MIN_ROWS
     int opt_attn_cap = 0;               // resident attention CTAs per SM (0: no cap)
     int opt_group_pdl = 0;              // programmatic dependent launch inside a group's chain
-    int opt_gemv_rows = 4;              // projections of at most this many rows stream on CUDA cores
+    int opt_gemv_rows = 0;              // projections of at most this many rows stream on CUDA cores
     int opt_persistent = 1;             // grids of several waves of 128 x 256 tiles run persistently
     int opt_small_step = 1;             // small models: the whole step in one launch
     // two row groups: library-owned streams, forked from and joined back to the caller's stream
@@ -341,7 +341,9 @@ int swa_splits(const rlt_config& c, int B, int t) {
 int xattn_splits(const rlt_config& c, int B, int t) {
     long long bh = (long long)B * c.n_heads;
     long long want = (XATTN_TARGET_WARPS + bh - 1) / bh;
-    long long by_len = (t + XATTN_MIN_CHUNK - 1) / XATTN_MIN_CHUNK;
+    // few (sequence, head) pairs: shorter chunks, so that more warps stream the keys
+    const int min_chunk = bh < 592 ? XATTN_MIN_CHUNK / 2 : XATTN_MIN_CHUNK;
+    long long by_len = (t + min_chunk - 1) / min_chunk;
     long long cap = XATTN_PART_ITEMS / bh;
     long long s = want;
     if (s > by_len) s = by_len;
@@ -1294,7 +1296,6 @@ rlt_status rlt_set_option(rlt_model* m, const char* name, int64_t value) {
 
 int rlt_gemm_plan(int M, int N, int K) {
     if (M < 1 || N < 1 || K < 1) return -1;
-    if (gemv_preferred(M, N, K)) return 16;
     if (gemm_swap_preferred(M, N, K)) {
         const int s = gemm_swap_auto_split(M, N, K);
         return 11 + (s == 1 ? 1 : (s == 2 ? 2 : (s == 4 ? 3 : 4)));

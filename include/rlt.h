@@ -347,12 +347,11 @@ uint64_t rlt_launch_count(const rlt_model* m);
  *   "persistent_gemm"    1 (default): projections whose grid of 128 x 256 tiles exceeds one
  *                        wave run on the persistent kernel (rlt_gemm_bf16 kernel 17); 0: one
  *                        CTA per tile.
- *   "gemv_rows"          projections of at most this many rows (0..4, default 4) run on the
- *                        weight-streaming CUDA-core kernel (bulk-copied weight rows requested
- *                        before the programmatic-launch wait) on the shapes where it measured
- *                        faster than the few-row tensor-core kernel (at least one 32-row block
- *                        of weights per SM, K <= 2048); 0 keeps every projection on the few-row
- *                        kernel.
+ *   "gemv_rows"          projections of at most this many rows (0..4; default 0) run on the
+ *                        weight-streaming CUDA-core kernel (rlt_gemm_bf16 kernel 16) on the
+ *                        shapes where it measured faster on its own than the few-row tensor-core
+ *                        kernel (at least one 32-row block of weights per SM, K <= 2048).  Off by
+ *                        default: inside a single-sequence decoder step it measured slower.
  *   "group_pdl"          1: programmatic dependent launch inside each row group's chain
  *                        (default 0: an early-launched kernel would hold SM resources the
  *                        other group needs).
@@ -381,8 +380,7 @@ rlt_status rlt_gemm_bf16(rlt_model* m, const void* A, const void* W, float* C, i
                          int kernel, void* stream);
 
 /* The kernel id (numbered as for rlt_gemm_bf16: 2 + v for row-tile variant v, 11 + s for the
- * few-row kernel with split s = 1: 1, 2: 2, 3: 4, 16 for the weight-streaming kernel, which the
- * "gemv_rows" option can turn off) that the library's own projections use for an
+ * few-row kernel with split s = 1: 1, 2: 2, 3: 4) that the library's own projections use for an
  * M x N x K bf16 product whose operands TMA can address, before any epilogue-specific
  * adjustment.  Pure host logic: no device, model or stream is touched.  Returns -1 for
  * non-positive sizes. */

@@ -4,7 +4,7 @@ workloads' decode and encoder shapes, i.e. the choices the measured timings pick
 Ids as rlt_gemm_bf16 numbers them: 2 + v = row-tile variant v (0: 128x32, 1: 128x64,
 2: 128x128 x3 stages, 3: 128x128 x6, 4: 128x256, 5: 128x128 split 2, 6: 128x128 split 4,
 7: 128x64 split 2, 8: 128x64 split 4); 11 + s = few-row kernel, s = 1, 2, 3 for a K split of
-1, 2, 4; 16 = the weight-streaming CUDA-core kernel (at most four rows).
+1, 2, 4.
 """
 import pytest
 
@@ -27,12 +27,9 @@ PLANS = [
     ((32, 2048, 2048), 14, "<= 32 rows: few-row kernel, split 4"),
     ((32, 6144, 2048), 13, "q/k/v at B=32"),
     ((32, 2048, 5632), 14, "down at B=32"),
-    ((1, 2048, 2048), 14, "B=1, narrow output: few-row kernel, split 4 (the weight-streaming kernel measured slower)"),
-    ((1, 11264, 2048), 16, "gate/up at B=1: every SM gets weight rows, weight-streaming kernel"),
-    ((1, 32768, 2048), 16, "LM head at B=1"),
-    ((4, 2048, 5632), 14, "down at B=4: long rows, few-row kernel"),
-    ((5, 2048, 2048), 14, "five rows: few-row tensor-core kernel"),
-    ((1, 2048, 8192), 14, "K above the weight-streaming kernel's ring: few-row kernel"),
+    ((1, 2048, 2048), 14, "B=1"),
+    ((1, 11264, 2048), 12, "gate/up at B=1"),
+    ((4, 2048, 5632), 14, "down at B=4"),
     # small shapes and the encoder
     ((64, 384, 128), 2, "two k-blocks: narrow row tiles put the most CTAs in flight"),
     ((65536, 3072, 1024), 6, "encoder q/k/v: grids of many waves take the widest tile"),
