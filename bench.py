@@ -462,8 +462,13 @@ def main() -> int:
         enc_ms = max_over_ranks(a.elapsed_time(b), dev)
         ef = encode_flops(m, B, T)
         enc_roof_ms = 1e3 * ef / (peaks["bf16_tflops"] * 1e12)
+        # one more encode with its launches bracketed by kind (brackets cost a few us each)
+        model.profile_start(["enc_gemm", "enc_attn", "enc_other"])
+        model.encode(tok, out=(e, M))
+        enc_kinds = {k: round(v[0], 2) for k, v in model.profile_stop().items()}
         enc = {"ms": enc_ms, "tflop": ef / 1e12, "achieved_tflops": ef / (enc_ms / 1e3) / 1e12,
                "peak_tflops": peaks["bf16_tflops"], "roofline_ms": enc_roof_ms, "frac": enc_roof_ms / enc_ms,
+               "breakdown_ms": enc_kinds,
                "note": "one rlt_encode of the whole batch; FLOPs of the linear maps and the causal attention"}
 
     replay = None

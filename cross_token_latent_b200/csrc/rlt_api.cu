@@ -375,42 +375,42 @@ rlt_status encode_impl(rlt_model* m, const int32_t* tokens, int B, int Tn, int T
     T* ews = reinterpret_cast<T*>(ws + w.ews);
     const float2* rope = m->at<float2>(m->lay.rope);
     const bool use_tc_attn = sizeof(T) == 2 && enc_attention_tc_supported(hd);
-    CK(launch_embed<T>(L, tokens, N, m->at<T>(m->lay.embed), c.V, d, h, m->hdr()));
+    CKP(RLT_K_ENC_OTHER, launch_embed<T>(L, tokens, N, m->at<T>(m->lay.embed), c.V, d, h, m->hdr()));
     for (int l = 0; l < c.L_E; ++l) {
         EpiArgs ea; ea.hdr = m->hdr();
-        CK(launch_rmsnorm<T>(L, h, N, d, m->at<float>(m->lay.attn_norm[l]), c.rms_eps, a, d, N, N, nullptr));
+        CKP(RLT_K_ENC_OTHER, launch_rmsnorm<T>(L, h, N, d, m->at<float>(m->lay.attn_norm[l]), c.rms_eps, a, d, N, N, nullptr));
         ea.out_f32 = qkv; ea.ld_out = 3 * d;
-        CK(launch_gemm<T>(L, Epi::StoreF32, a, d, m->at<T>(m->lay.wqkv[l]), N, 3 * d, d, ea));
+        CKP(RLT_K_ENC_GEMM, launch_gemm<T>(L, Epi::StoreF32, a, d, m->at<T>(m->lay.wqkv[l]), N, 3 * d, d, ea));
         if (cache)
-            CK(launch_enc_cache_write<T>(L, qkv, B, Tn, H, hd, rope, 0, nullptr,
+            CKP(RLT_K_ENC_OTHER, launch_enc_cache_write<T>(L, qkv, B, Tn, H, hd, rope, 0, nullptr,
                                          cache + (size_t)l * enc_cache_layer_elems(c, B, T_max), T_max, nullptr));
         if (use_tc_attn) {
             bf16* pl = reinterpret_cast<bf16*>(planes);
             size_t plane = (size_t)N * d;
-            CK(launch_enc_qkv_layout<T>(L, qkv, B, Tn, H, hd, rope, planes, false));
-            CK(launch_enc_vt(L, qkv, pl + 2 * plane, B, Tn, H, hd));
-            CK(launch_enc_attention_tc(L, pl, pl + plane, pl + 2 * plane, reinterpret_cast<bf16*>(att), B, Tn, H, hd,
+            CKP(RLT_K_ENC_OTHER, launch_enc_qkv_layout<T>(L, qkv, B, Tn, H, hd, rope, planes, false));
+            CKP(RLT_K_ENC_OTHER, launch_enc_vt(L, qkv, pl + 2 * plane, B, Tn, H, hd));
+            CKP(RLT_K_ENC_ATTN, launch_enc_attention_tc(L, pl, pl + plane, pl + 2 * plane, reinterpret_cast<bf16*>(att), B, Tn, H, hd,
                                        m->hdr()));
         } else {
-            CK(launch_enc_qkv_layout<T>(L, qkv, B, Tn, H, hd, rope, planes));
-            CK(launch_enc_attention<T>(L, planes, att, B, Tn, H, hd));
+            CKP(RLT_K_ENC_OTHER, launch_enc_qkv_layout<T>(L, qkv, B, Tn, H, hd, rope, planes));
+            CKP(RLT_K_ENC_ATTN, launch_enc_attention<T>(L, planes, att, B, Tn, H, hd));
         }
         ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = h; ea.ld_out = d;
-        CK(launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.wo[l]), N, d, d, ea));
-        CK(launch_rmsnorm<T>(L, h, N, d, m->at<float>(m->lay.ffn_norm[l]), c.rms_eps, a, d, N, N, nullptr));
+        CKP(RLT_K_ENC_GEMM, launch_gemm<T>(L, Epi::ResidAdd, att, d, m->at<T>(m->lay.wo[l]), N, d, d, ea));
+        CKP(RLT_K_ENC_OTHER, launch_rmsnorm<T>(L, h, N, d, m->at<float>(m->lay.ffn_norm[l]), c.rms_eps, a, d, N, N, nullptr));
         ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_t = act; ea.ld_out = F;
-        CK(launch_gemm<T>(L, Epi::SwiGLU, a, d, m->at<T>(m->lay.wgu[l]), N, 2 * F, d, ea));
+        CKP(RLT_K_ENC_GEMM, launch_gemm<T>(L, Epi::SwiGLU, a, d, m->at<T>(m->lay.wgu[l]), N, 2 * F, d, ea));
         ea = EpiArgs(); ea.hdr = m->hdr(); ea.out_f32 = h; ea.ld_out = d;
-        CK(launch_gemm<T>(L, Epi::ResidAdd, act, F, m->at<T>(m->lay.wdown[l]), N, d, F, ea));
+        CKP(RLT_K_ENC_GEMM, launch_gemm<T>(L, Epi::ResidAdd, act, F, m->at<T>(m->lay.wdown[l]), N, d, F, ea));
     }
     // e = RMSNorm(h) written with row capacity T_alloc, plus a contiguous copy for M
-    CK(launch_rmsnorm<T>(L, h, N, d, m->at<float>(m->lay.enc_norm), c.rms_eps, e, d, Tn, T_alloc, ews));
+    CKP(RLT_K_ENC_OTHER, launch_rmsnorm<T>(L, h, N, d, m->at<float>(m->lay.enc_norm), c.rms_eps, e, d, Tn, T_alloc, ews));
     size_t group_elems = (size_t)2 * B * H * (size_t)T_alloc * hd;
     for (int g = 0; g < c.G; ++g) {
         EpiArgs ea; ea.hdr = m->hdr();
         ea.out_f32 = qkv; ea.ld_out = 2 * d;
-        CK(launch_gemm<T>(L, Epi::StoreF32, ews, d, m->at<T>(m->lay.mem) + (size_t)g * 2 * d * d, N, 2 * d, d, ea));
-        CK(launch_mem_layout<T>(L, qkv, B, Tn, T_alloc, H, hd, M + g * group_elems));
+        CKP(RLT_K_ENC_GEMM, launch_gemm<T>(L, Epi::StoreF32, ews, d, m->at<T>(m->lay.mem) + (size_t)g * 2 * d * d, N, 2 * d, d, ea));
+        CKP(RLT_K_ENC_OTHER, launch_mem_layout<T>(L, qkv, B, Tn, T_alloc, H, hd, M + g * group_elems));
     }
     return RLT_OK;
 }

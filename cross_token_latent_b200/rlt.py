@@ -102,7 +102,7 @@ _EXPORTS = {
 }
 
 KERNEL_KINDS = ["norm", "merge", "qkv", "swa", "o_proj", "qc_proj", "xattn", "oc_proj", "ffn_up", "ffn_down",
-                "final_norm", "head", "lse", "encoder", "small_step"]
+                "final_norm", "head", "lse", "encoder", "small_step", "enc_gemm", "enc_attn", "enc_other"]
 
 
 def lib() -> ctypes.CDLL:

@@ -417,7 +417,10 @@ enum {
     RLT_K_LSE = 12,      /* log-sum-exp + gather + score                                 */
     RLT_K_ENCODER = 13,  /* a whole rlt_encode call                                      */
     RLT_K_SMALL_STEP = 14, /* a small model's whole decoder step in one launch           */
-    RLT_K_COUNT = 15
+    RLT_K_ENC_GEMM = 15,   /* the encoder's projections (inside RLT_K_ENCODER)            */
+    RLT_K_ENC_ATTN = 16,   /* the encoder's causal attention                               */
+    RLT_K_ENC_OTHER = 17,  /* the encoder's embedding, norms and layout kernels            */
+    RLT_K_COUNT = 18
 };
 
 /* Start recording a CUDA event pair on the launch stream around every launch of the kinds
