@@ -33,7 +33,7 @@ constexpr int SS_MAX_D = 256, SS_MAX_F = 1024, SS_MAX_V = 8192;
 template <typename T>
 __device__ __forceinline__ void gemv_rows(const T* __restrict__ W, int N, int K, const float* x, float* y) {
     constexpr int EPL = Vec16<T>::N;
-    constexpr int U = 8;
+    constexpr int U = 4;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nv = K / EPL;
     int lpr = 32;
@@ -109,21 +109,14 @@ __device__ __forceinline__ void warp_partial(const float* q, const T* __restrict
         m = mx;
     };
     for (int j = j0 + lane; j < n; j += stride) {
-        // the key's K and V rows are requested together (one memory round trip per key)
-        uint4 kv[2 * (HD / EPL)];
-#pragma unroll
-        for (int v = 0; v < HD / EPL; ++v) {
-            kv[v] = ld16(K + (size_t)j * HD + v * EPL);
-            kv[HD / EPL + v] = ld16(V + (size_t)j * HD + v * EPL);
-        }
         float r[HD];
 #pragma unroll
-        for (int v = 0; v < HD / EPL; ++v) Vec16<T>::unpack(kv[v], r + v * EPL);
+        for (int v = 0; v < HD / EPL; ++v) Vec16<T>::unpack(ld16(K + (size_t)j * HD + v * EPL), r + v * EPL);
         float s = 0.f;
 #pragma unroll
         for (int i = 0; i < HD; ++i) s = fmaf(q[i], r[i], s);
 #pragma unroll
-        for (int v = 0; v < HD / EPL; ++v) Vec16<T>::unpack(kv[HD / EPL + v], r + v * EPL);
+        for (int v = 0; v < HD / EPL; ++v) Vec16<T>::unpack(ld16(V + (size_t)j * HD + v * EPL), r + v * EPL);
         fold(s, r);
     }
     if (kx && lane == 0) {
