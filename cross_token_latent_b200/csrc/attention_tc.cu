@@ -52,6 +52,13 @@ struct FaShape {
 constexpr int FA_SOFTMAX_WARPS = 8;                        // two per TMEM lane quadrant
 constexpr int FA_THREADS = (FA_SOFTMAX_WARPS + 2) * 32;    // + TMA producer + MMA issuer
 
+// 2^x by the ex2.approx instruction (relative error ~2^-22; flushes denormals to zero).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 template <int HD>
 __global__ void __launch_bounds__(FA_THREADS, 1)
 k_enc_fa_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -193,15 +200,22 @@ k_enc_fa_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_free[sb]);
+            // the maximum is taken over the raw scores (qscale > 0), and exp2 of
+            // qscale * s - max is one fused multiply-add and one ex2.approx per element: the
+            // probabilities are rounded to bf16 right after, far coarser than ex2.approx's error
             const bool diag = (j == nt - 1);
-            float mx = m;
+            float rmx = -1e30f;
+            if (diag) {
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                float v = sv[c] * qscale;
-                if (diag && j * KT + hf * 64 + c > q) v = -1e30f;
-                sv[c] = v;
-                mx = fmaxf(mx, v);
+                for (int c = 0; c < 64; ++c) {
+                    if (j * KT + hf * 64 + c > q) sv[c] = -1e30f;
+                    rmx = fmaxf(rmx, sv[c]);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 64; ++c) rmx = fmaxf(rmx, sv[c]);
             }
+            float mx = fmaxf(m, rmx * qscale);
             // the row's maximum over both halves
             float* rb = red + (size_t)sb * 2 * QT;
             rb[hf * QT + r] = mx;
@@ -210,7 +224,8 @@ k_enc_fa_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             mx = fmaxf(mx, rb[(1 - hf) * QT + r]);
-            const float alpha = exp2f(m - mx);
+            const float alpha = ex2_approx(m - mx);
+            const float nmx = -mx;
             float rowsum = 0.f;
             // P_j overwrites P_{j-1}: wait until P_{j-1} V_{j-1} has completed (it also makes O
             // final for the rescale below)
@@ -224,13 +239,13 @@ k_enc_fa_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             for (int ch = 0; ch < 8; ++ch) {
                 float p8[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    float p = round_to<bf16>(exp2f(sv[ch * 8 + i] - mx));
-                    p8[i] = p;
-                    rowsum += p;
-                }
+                for (int i = 0; i < 8; ++i) p8[i] = ex2_approx(fmaf(sv[ch * 8 + i], qscale, nmx));
+                const uint4 packed = Vec16<bf16>::pack(p8);          // rounded to bf16 once
+                Vec16<bf16>::unpack(packed, p8);                      // the rounded values
+#pragma unroll
+                for (int i = 0; i < 8; ++i) rowsum += p8[i];
                 uint8_t* dst = P + r * 128 + ((ch ^ (r & 7)) << 4);
-                *reinterpret_cast<uint4*>(dst) = Vec16<bf16>::pack(p8);
+                *reinterpret_cast<uint4*>(dst) = packed;
             }
             l = l * alpha + rowsum;
             if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {     // warp-collective TMEM access
