@@ -10,7 +10,7 @@
 //   warp 2          allocates / frees the TMEM columns;
 //   all 4 warps     epilogue: warp w reads TMEM lanes 32w..32w+31 (one output row per
 //                   thread) with tcgen05.ld and applies the fused epilogue.
-// No multicast is used anywhere.  Every mbarrier wait is bounded by %globaltimer; on
+// No load uses multicast.  Every mbarrier wait is bounded by %globaltimer; on
 // expiry the CTA raises ERR_TIMEOUT, stops issuing work, frees its TMEM and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -149,6 +149,12 @@ struct RowNorm {
             for (int j = 0; j < 16; ++j) v[j] *= rinv;
         }
     }
+    __device__ __forceinline__ void scale32(const EpiArgs& ea, float* v) const {
+        if (ea.ss_in) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] *= rinv;
+        }
+    }
     __device__ __forceinline__ void add(Epi epi, const EpiArgs& ea, int m, int n, int N, float part) {
         if (!ea.norm_y) return;
         acc += part;
@@ -196,6 +202,173 @@ __device__ __forceinline__ void lse_row(const EpiArgs& ea, uint32_t lane_base, i
         }
     }
     if (m < M) ea.lse_part[(long long)m * ea.lse_ld + tn] = make_float2(mx, sm);
+}
+
+// ---- Staged epilogue.  A warp owns 32 consecutive output rows (lane = row).  Writing each
+// row's values with its own thread puts the 32 lanes of every store on 32 different rows, i.e.
+// 32 separate memory transactions per instruction; the staged path instead passes 32-column
+// chunks through the warp's 4 KB staging area in shared memory (32 rows x 128 bytes, 16-byte
+// pieces XOR-swizzled by row, so that both the row-wise and the column-wise accesses are free of
+// bank conflicts) and moves whole row segments: every global instruction of the warp then
+// covers 4 rows x 128 bytes (or 8 x 64, 16 x 32).  The arithmetic per element is that of
+// epilogue16, in the same order.
+constexpr int STG_BYTES = 32 * 128;          // one warp's staging area
+
+__device__ __forceinline__ uint4* stg_at(uint8_t* stg, int row, int piece) {
+    return reinterpret_cast<uint4*>(stg + row * 128 + ((piece ^ (row & 7)) << 4));
+}
+// rows row0 .. row0+31 (those below M) of `row_bytes` (32, 64 or 128) bytes each, between the
+// staging area and global memory at g + (row0 + r) * ld_bytes
+template <int ROW_BYTES>
+__device__ __forceinline__ void stg_store_rows(uint8_t* stg, uint8_t* g, long long ld_bytes, int row0, int M) {
+    constexpr int PPR = ROW_BYTES / 16, RPI = 32 / PPR;      // pieces per row, rows per instruction
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int i = 0; i < PPR; ++i) {
+        const int r = i * RPI + lane / PPR, pc = lane % PPR;
+        if (row0 + r < M) st16(g + (row0 + r) * ld_bytes + pc * 16, *stg_at(stg, r, pc));
+    }
+}
+template <int ROW_BYTES>
+__device__ __forceinline__ void stg_load_rows(uint8_t* stg, const uint8_t* g, long long ld_bytes, int row0, int M) {
+    constexpr int PPR = ROW_BYTES / 16, RPI = 32 / PPR;
+    const int lane = threadIdx.x & 31;
+    uint4 t[PPR];
+#pragma unroll
+    for (int i = 0; i < PPR; ++i) {
+        const int r = i * RPI + lane / PPR, pc = lane % PPR;
+        t[i] = row0 + r < M ? ld16(g + (row0 + r) * ld_bytes + pc * 16) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < PPR; ++i) *stg_at(stg, i * RPI + lane / PPR, lane % PPR) = t[i];
+}
+
+// Whether the 32 columns n .. n+31 can take the staged path: the chunk lies inside N and every
+// row segment it moves starts on a 16-byte boundary.
+__device__ __forceinline__ bool staged_ok(Epi epi, const EpiArgs& ea, int n, int N) {
+    if (n + 32 > N) return false;
+    switch (epi) {
+        case Epi::StoreF32:
+            return ((reinterpret_cast<uintptr_t>(ea.out_f32) | ((uintptr_t)ea.ld_out * 4)) & 15) == 0;
+        case Epi::ResidAdd:
+            return ((reinterpret_cast<uintptr_t>(ea.out_f32) | ((uintptr_t)ea.ld_out * 4)) & 15) == 0 &&
+                   (!ea.norm_y || (reinterpret_cast<uintptr_t>(ea.norm_y) & 15) == 0);
+        case Epi::SwiGLU:
+            return ((reinterpret_cast<uintptr_t>(ea.out_t) | ((uintptr_t)ea.ld_out * 2)) & 15) == 0;
+        default:
+            return false;
+    }
+}
+
+// The staged epilogue of columns n .. n+31 for rows row0 .. row0+31 (this lane: row0 + lane),
+// v = this lane's 32 accumulators after the deferred norm's scale.  Warp-collective.
+__device__ __forceinline__ void epilogue32_staged(Epi epi, const EpiArgs& ea, int row0, int M, int n, float* v,
+                                                  uint8_t* stg) {
+    const int lane = threadIdx.x & 31, m = row0 + lane;
+    switch (epi) {
+        case Epi::StoreF32: {
+#pragma unroll
+            for (int p = 0; p < 8; ++p)
+                *stg_at(stg, lane, p) = make_uint4(__float_as_uint(v[4 * p] * ea.scale), __float_as_uint(v[4 * p + 1] * ea.scale),
+                                                   __float_as_uint(v[4 * p + 2] * ea.scale),
+                                                   __float_as_uint(v[4 * p + 3] * ea.scale));
+            __syncwarp();
+            stg_store_rows<128>(stg, reinterpret_cast<uint8_t*>(ea.out_f32 + n), (long long)ea.ld_out * 4, row0, M);
+            __syncwarp();
+            break;
+        }
+        case Epi::ResidAdd: {
+            uint8_t* xg = reinterpret_cast<uint8_t*>(ea.out_f32 + n);
+            const long long xld = (long long)ea.ld_out * 4;
+            stg_load_rows<128>(stg, xg, xld, row0, M);
+            __syncwarp();
+            float x[32];
+#pragma unroll
+            for (int p = 0; p < 8; ++p) {
+                float t[4];
+                Vec16<float>::unpack(*stg_at(stg, lane, p), t);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) x[4 * p + j] = t[j] + v[4 * p + j];
+            }
+            __syncwarp();
+#pragma unroll
+            for (int p = 0; p < 8; ++p) *stg_at(stg, lane, p) = Vec16<float>::pack(x + 4 * p);
+            __syncwarp();
+            stg_store_rows<128>(stg, xg, xld, row0, M);
+            if (ea.norm_y) {
+                float y[32];
+                float ss0 = 0.f, ss1 = 0.f;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    y[j] = x[j] * ea.norm_g[n + j];
+                    ss0 += x[j] * x[j];
+                }
+#pragma unroll
+                for (int j = 16; j < 32; ++j) {
+                    y[j] = x[j] * ea.norm_g[n + j];
+                    ss1 += x[j] * x[j];
+                }
+                __syncwarp();
+#pragma unroll
+                for (int p = 0; p < 4; ++p) *stg_at(stg, lane, p) = Vec16<bf16>::pack(y + 8 * p);
+                __syncwarp();
+                stg_store_rows<64>(stg, reinterpret_cast<uint8_t*>(ea.norm_y + n), (long long)ea.ld_out * 2, row0, M);
+                if (m < M) {
+                    ea.ss_out[(long long)m * ea.ss_ld + n / 16] = ss0;
+                    ea.ss_out[(long long)m * ea.ss_ld + n / 16 + 1] = ss1;
+                }
+            }
+            __syncwarp();
+            break;
+        }
+        case Epi::SwiGLU: {     // columns 2j = gate_j, 2j+1 = up_j -> 16 outputs at n / 2
+            float h[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) h[j] = siluf_(v[2 * j]) * v[2 * j + 1];
+            *stg_at(stg, lane, 0) = Vec16<bf16>::pack(h);
+            *stg_at(stg, lane, 1) = Vec16<bf16>::pack(h + 8);
+            __syncwarp();
+            stg_store_rows<32>(stg, reinterpret_cast<uint8_t*>(reinterpret_cast<bf16*>(ea.out_t) + n / 2),
+                               (long long)ea.ld_out * 2, row0, M);
+            __syncwarp();
+            break;
+        }
+        default:
+            break;
+    }
+}
+
+// The epilogue of one accumulator row m (TMEM lanes at lane_base, columns n0 .. n0+BN-1 of
+// output column tile tn), through the warp's staging area stg where the chunk allows it.
+// Warp-collective (TMEM loads, staging).
+template <int BN>
+__device__ __forceinline__ void epilogue_row(Epi epi, const EpiArgs& ea, uint32_t lane_base, int m, int M, int n0,
+                                             int N, int tn, RowNorm& rn, uint8_t* stg) {
+    if (epi == Epi::LsePart) {
+        lse_row<BN>(ea, lane_base, m, M, n0, N, tn);
+        return;
+    }
+    const int row0 = m - (int)(threadIdx.x & 31);
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+        const int n = n0 + c;
+        if (staged_ok(epi, ea, n, N)) {
+            float v[32];
+            tmem_ld32(lane_base + c, v);
+            rn.scale32(ea, v);
+            epilogue32_staged(epi, ea, row0, M, n, v, stg);
+            continue;
+        }
+#pragma unroll 1
+        for (int h = c; h < c + 32 && h < BN; h += 16) {
+            float v[16];
+            tmem_ld16(lane_base + h, v);
+            if (m < M && n0 + h < N) {
+                rn.scale(ea, v);
+                rn.add(epi, ea, m, n0 + h, N, epilogue16(epi, ea, m, n0 + h, min(16, N - n0 - h), v));
+            }
+        }
+    }
 }
 
 template <int BN, int STAGES, int SPLIT>
@@ -319,21 +492,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     tc_fence_after();
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     if constexpr (SPLIT == 1) {
-        if (ok && epi == Epi::LsePart) {
-            lse_row<BN>(ea, lane_base, m0 + warp * 32 + lane, M, n0, N, blockIdx.x);
-        } else if (ok) {
-            const int m = m0 + warp * 32 + lane;
-#pragma unroll 1
-            for (int c = 0; c < BN; c += 16) {
-                float v[16];
-                tmem_ld16(lane_base + c, v);
-                int n = n0 + c;
-                if (m < M && n < N) {
-                    rn.scale(ea, v);
-                    rn.add(epi, ea, m, n, N, epilogue16(epi, ea, m, n, min(16, N - n), v));
-                }
-            }
-        }
+        // every stage of the ring has been consumed: its first 16 KB are the warps' staging areas
+        if (ok) epilogue_row<BN>(epi, ea, lane_base, m0 + warp * 32 + lane, M, n0, N, blockIdx.x, rn,
+                                 smem + warp * STG_BYTES);
     } else {
         // Column bands: rank r owns output columns [r * BAND, (r + 1) * BAND) of the tile for
         // all 128 rows, so every thread keeps its row.  It sends each band of its partial row
@@ -361,8 +522,24 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         cluster_wait_acquire();                                  // all partials have landed
         if (ok) {
             const int m = m0 + row;
+            uint8_t* stg = smem + warp * STG_BYTES;       // the consumed ring
 #pragma unroll 1
             for (int c = 0; c < S::BAND; c += 16) {
+                const int n = n0 + (int)rank * S::BAND + c;
+                if (S::BAND % 32 == 0 && c % 32 == 0 && staged_ok(epi, ea, n, N)) {
+                    float v[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = 0.f;
+                    for (int src = 0; src < SPLIT; ++src) {
+                        const float* p = recv + ((size_t)src * S::BAND + c) * BM + row;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] += p[j * BM];
+                    }
+                    rn.scale32(ea, v);
+                    epilogue32_staged(epi, ea, m0 + warp * 32, M, n, v, stg);
+                    c += 16;                               // the chunk covered 32 columns
+                    continue;
+                }
                 float v[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) v[j] = 0.f;
@@ -371,7 +548,6 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 #pragma unroll
                     for (int j = 0; j < 16; ++j) v[j] += p[j * BM];
                 }
-                int n = n0 + (int)rank * S::BAND + c;
                 if (m < M && n < N) {
                     rn.scale(ea, v);
                     rn.add(epi, ea, m, n, N, epilogue16(epi, ea, m, n, min(16, N - n), v));
@@ -392,6 +568,163 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     if (warp == 2) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(S::TMEM_COLS));
+    }
+}
+
+// CTA-pair row-tile GEMM: a cluster of two CTAs computes one 256 x BN output tile with
+// tcgen05.mma.cta_group::2 (M = 256).  CTA r of the pair stages rows 128 r .. 128 r + 127 of the
+// A tile and rows (BN / 2) r .. (BN / 2)(r + 1) - 1 of the W tile, so each CTA reads 1/3 fewer
+// bytes per k-block than a 128 x BN tile of the same MMA work, and holds accumulator rows 128 r ..
+// in its own TMEM.  Roles per CTA as in k_gemm_tc, except:
+//   - both producers' loads complete on the leader's (rank 0) full[s] barrier, which the leader
+//     arms for both CTAs' bytes (a load landing first leaves the barrier's transaction count
+//     below zero until the leader arrives, so the phase cannot complete early);
+//   - the leader's lane issues the pair MMAs; its commits arrive on empty[s] and done in both
+//     CTAs, so each producer refills its own stage and each CTA's epilogue starts on its own;
+//     after a timeout the leader commits to its own `drain` barrier instead of done, so the
+//     peer's bounded wait for done runs out and neither CTA stores a partial accumulator;
+//   - TMEM is allocated and freed by warp 2 of both CTAs together (cta_group::2), and a
+//     cluster barrier orders the barrier initialisation and allocation before any load or MMA,
+//     and every TMEM read of both CTAs before the free.
+// Every CTA of the pair reaches both cluster barriers on every path (no early return).
+template <int BN, int STAGES>
+struct PairShape {
+    static constexpr int WB = BN / 2;                       // W rows per CTA
+    static constexpr int B_BYTES = WB * BK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int TMEM_COLS = BN < 32 ? 32 : BN;
+    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
+    static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "pair MMA: N a multiple of 16 per CTA half, at most 256");
+};
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(128, 1)
+k_gemm_tc_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW, int M, int N, int K,
+               Epi epi, EpiArgs ea, DevHeader* hdr) {
+    using S = PairShape<BN, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES);   // used in the leader
+    uint64_t* empty = full + STAGES;
+    uint64_t* done = empty + STAGES;
+    uint64_t* drain = done + 1;               // leader: the MMAs issued before a timeout completed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    __shared__ int abort_flag, fin;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const int m0 = blockIdx.y * 2 * BM + (int)rank * BM;
+    const int n0 = (blockIdx.x >> 1) * BN;
+    const int nkb = (K + BK - 1) / BK;
+    pdl_trigger();
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(done, 1);
+        mbar_init(drain, 1);
+        abort_flag = 0;
+        fin = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 2) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(S::TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_arrive_release();
+    cluster_wait_acquire();                  // both CTAs' barriers initialised, TMEM allocated
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    // the MMA writes the peer's rows at the leader's TMEM address: both allocations must agree
+    if (rank == 0 && threadIdx.x == 0 && dsmem_ld_u32(cluster_addr(tmem_slot, 1)) != tmem) abort_flag = 1;
+    __syncthreads();
+
+    const uint64_t lim = ea.wait_ns;
+    int armed = 0;
+    if (warp == 0 && lane == 0) {
+        // producer of this CTA's halves; weight tiles before the programmatic-launch wait
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&tmW) : "memory");
+        const uint32_t full0 = cluster_addr(full, 0);
+        const int wrow = n0 + (int)rank * S::WB;
+        const int pre = (ea.no_loads || abort_flag) ? 0 : (nkb < STAGES ? nkb : STAGES);
+        for (int kb = 0; kb < pre; ++kb) {
+            uint8_t* a = smem + kb * S::STAGE_BYTES;
+            if (rank == 0) mbar_expect_tx(&full[kb], 2 * S::STAGE_BYTES);
+            tma_load_2d_pair(a + A_BYTES, &tmW, full0 + 8u * kb, kb * BK, wrow);
+        }
+        pdl_wait();
+        for (int kb = 0; kb < pre; ++kb) tma_load_2d_pair(smem + kb * S::STAGE_BYTES, &tmA, full0 + 8u * kb, kb * BK, m0);
+        armed = pre;
+        for (int kb = pre; kb < nkb && pre > 0; ++kb) {
+            const int s = kb % STAGES;
+            const uint32_t ph = (kb / STAGES) & 1;
+            if (!mbar_wait(&empty[s], ph ^ 1, &abort_flag, lim)) { abort_flag = 1; break; }
+            uint8_t* a = smem + s * S::STAGE_BYTES;
+            if (rank == 0) mbar_expect_tx(&full[s], 2 * S::STAGE_BYTES);
+            tma_load_2d_pair(a, &tmA, full0 + 8u * s, kb * BK, m0);
+            tma_load_2d_pair(a + A_BYTES, &tmW, full0 + 8u * s, kb * BK, wrow);
+            armed = kb + 1;
+        }
+    } else if (warp == 1 && lane == 0 && rank == 0) {
+        // MMA issuer of the pair (leader only)
+        constexpr uint32_t idesc = idesc_bf16(2 * BM, BN);
+        for (int kb = 0; kb < nkb && !abort_flag; ++kb) {
+            const int s = kb % STAGES;
+            const uint32_t ph = (kb / STAGES) & 1;
+            if (!mbar_wait(&full[s], ph, &abort_flag, lim)) { abort_flag = 1; break; }
+            tc_fence_after();
+            uint8_t* a = smem + s * S::STAGE_BYTES;
+            const uint64_t da = sdesc_sw128(a), dw = sdesc_sw128(a + A_BYTES);
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k) umma_pair(tmem, da + 2 * k, dw + 2 * k, idesc, (kb | k) != 0);
+            umma_commit_pair(&empty[s]);
+        }
+        // exactly one commit tracks every MMA issued (none in flight when TMEM is read or freed)
+        if (abort_flag) {
+            umma_commit_pair(drain, 1);
+            fin = 2;
+        } else if (nkb > 0) {
+            umma_commit_pair(done, 3);
+            fin = 1;
+        }
+    }
+    __syncwarp();
+    pdl_wait();
+
+    RowNorm rn;
+    const int m = m0 + warp * 32 + lane;
+    if (ea.ss_in && m < M) rn.rinv = deferred_rinv(ea, m);
+    // the leader stops waiting as soon as one of its roles gives up
+    bool ok = nkb == 0 ? true : mbar_wait(done, 0, rank == 0 ? &abort_flag : nullptr, lim);
+    ok = __syncthreads_and(ok) && abort_flag == 0;
+    tc_fence_after();
+    if (ok)
+        epilogue_row<BN>(epi, ea, tmem + ((uint32_t)(warp * 32) << 16), m, M, n0, N, blockIdx.x >> 1, rn,
+                         smem + warp * STG_BYTES);     // the consumed ring stages the epilogue
+    if (!ok && threadIdx.x == 0) {
+        raise_flag(hdr, ERR_TIMEOUT);
+        if (rank == 0) {
+            // the leader waits (bounded) for the MMAs it issued and for the stages it armed (a
+            // peer's loads complete on them too)
+            if (fin == 1) mbar_wait(done, 0, nullptr, lim);
+            if (fin == 2) mbar_wait(drain, 0, nullptr, lim);
+            for (int kb = armed > STAGES ? armed - STAGES : 0; kb < armed; ++kb)
+                mbar_wait(&full[kb % STAGES], (kb / STAGES) & 1, nullptr, lim);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_arrive_release();
+    cluster_wait_acquire();                  // both CTAs have read their accumulators
+    if (warp == 2) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(S::TMEM_COLS));
     }
 }
 
@@ -424,6 +757,8 @@ k_gemm_tc_pers(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     uint64_t* acc_full = empty + STAGES;             // [2]
     uint64_t* acc_empty = acc_full + 2;              // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+    // the epilogue warps' staging areas (the ring keeps loading the next tiles meanwhile)
+    uint8_t* stg_all = smem + STAGES * S::STAGE_BYTES + 256;
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -523,20 +858,7 @@ k_gemm_tc_pers(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             if (!ok) { abort_flag = 1; break; }
             tc_fence_after();
             const uint32_t lane_base = tmem + a * BN + ((uint32_t)(q * 32) << 16);
-            if (epi == Epi::LsePart) {
-                lse_row<BN>(ea, lane_base, m, M, n0, N, tn);
-            } else {
-#pragma unroll 1
-                for (int c = 0; c < BN; c += 16) {
-                    float v[16];
-                    tmem_ld16(lane_base + c, v);
-                    const int n = n0 + c;
-                    if (m < M && n < N) {
-                        rn.scale(ea, v);
-                        rn.add(epi, ea, m, n, N, epilogue16(epi, ea, m, n, min(16, N - n), v));
-                    }
-                }
-            }
+            epilogue_row<BN>(epi, ea, lane_base, m, M, n0, N, tn, rn, stg_all + q * STG_BYTES);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[a]);
@@ -708,12 +1030,44 @@ cudaError_t run_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int
     }
 }
 
+// The CTA-pair kernel: clusters of two CTAs along x, one 256-row band of tiles per grid row.
+template <int BN, int STAGES>
+cudaError_t run_tc_pair(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
+                        const EpiArgs& ea, DevHeader* hdr) {
+    using S = PairShape<BN, STAGES>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(k_gemm_tc_pair<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             S::SMEM);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    CUtensorMap ta, tw;
+    if (!cached_map(&ta, A, M, K, lda, BM) || !cached_map(&tw, W, N, K, K, S::WB)) return cudaErrorInvalidValue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * ((N + BN - 1) / BN), (M + 2 * BM - 1) / (2 * BM), 1);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = S::SMEM;
+    cfg.stream = L.stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = L.pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    *L.count += 1;
+    return cudaLaunchKernelEx(&cfg, k_gemm_tc_pair<BN, STAGES>, ta, tw, M, N, K, epi, ea, hdr);
+}
+
 // The persistent kernel for grids of more than one wave: one CTA per SM.
 template <int BN, int STAGES>
 cudaError_t run_tc_pers(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                         const EpiArgs& ea, DevHeader* hdr) {
     using S = TcShape<BN, STAGES, 1>;
-    constexpr int SMEM = STAGES * S::STAGE_BYTES + 1024 + 256;
+    constexpr int SMEM = STAGES * S::STAGE_BYTES + 1024 + 256 + 4 * STG_BYTES;   // + the epilogue staging
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(k_gemm_tc_pers<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -830,6 +1184,12 @@ cudaError_t launch_gemm_tc_lse(Launch L, const bf16* A, int lda, const bf16* W, 
 cudaError_t launch_gemm_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                            const EpiArgs& ea, DevHeader* hdr, int variant) {
     if (variant == PERSISTENT_VARIANT) return run_tc_pers<256, 4>(L, epi, A, lda, W, M, N, K, ea, hdr);
+    switch (variant) {      // CTA-pair tiles 256 x 64 / 128 / 256 (stages: ~200 KB of ring per CTA)
+        case PAIR_VARIANT + 0: return run_tc_pair<64, 10>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case PAIR_VARIANT + 1: return run_tc_pair<128, 8>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case PAIR_VARIANT + 2: return run_tc_pair<256, 6>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        default: break;
+    }
     int v = (variant >= 0 && variant < N_VARIANTS) ? variant : pick_variant(M, N, K);
     // a merge's deferred-norm group spans 32 GEMM columns and must stay in one column band
     if (epi == Epi::Merge && ea.norm_y && VARIANTS[v].split > 1 && VARIANTS[v].bn / VARIANTS[v].split < 32) v = 7;

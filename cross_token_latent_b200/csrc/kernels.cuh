@@ -189,6 +189,9 @@ bool gemm_tc_supported(const void* A, int lda, const void* W, int K);
 int gemm_tc_variants();
 // launch_gemm_tc's variant id of the persistent 128 x 256 kernel (two TMEM accumulators)
 constexpr int PERSISTENT_VARIANT = 100;
+// launch_gemm_tc's variant ids of the CTA-pair kernel: PAIR_VARIANT + p, tiles 256 x (64 << p)
+constexpr int PAIR_VARIANT = 200;
+constexpr int N_PAIR_VARIANTS = 3;
 // the row-tile variant the library picks for an M x N x K product (host logic only)
 int gemm_tc_pick(int M, int N, int K);
 // variant < 0: pick the tile shape from (M, N); otherwise force tile variant `variant`.

@@ -1306,7 +1306,8 @@ int rlt_gemm_plan(int M, int N, int K) {
 rlt_status rlt_gemm_bf16(rlt_model* m, const void* A, const void* W, float* C, int M, int N, int K, int kernel,
                          void* stream) {
     const int n_tc = gemm_tc_variants();
-    if (!m || !A || !W || !C || M < 1 || N < 1 || K < 1 || kernel < 0 || kernel > 3 + n_tc + 5) return RLT_EINVAL;
+    if (!m || !A || !W || !C || M < 1 || N < 1 || K < 1 || kernel < 0 || kernel > 3 + n_tc + 5 + N_PAIR_VARIANTS)
+        return RLT_EINVAL;
     if (kernel > 1 + n_tc && kernel <= 1 + n_tc + 5 && !gemm_swap_supported(M)) return RLT_EINVAL;
     if (kernel == 2 + n_tc + 5 && !gemv_supported(M, N, K, K, A, W)) return RLT_EINVAL;
     if (!aligned(A, 16) || !aligned(W, 16) || !aligned(C, 16) || K % 8 || N % 4) return RLT_EINVAL;
@@ -1328,8 +1329,10 @@ rlt_status rlt_gemm_bf16(rlt_model* m, const void* A, const void* W, float* C, i
         CK(launch_gemm_swap(L, Epi::StoreF32, a, K, w, M, N, K, ea, m->hdr(), splits[kernel - 2 - n_tc]));
     } else if (kernel == 2 + n_tc + 5) {
         CK(launch_gemv(L, Epi::StoreF32, a, K, w, M, N, K, ea, m->hdr()));
-    } else {
+    } else if (kernel == 3 + n_tc + 5) {
         CK(launch_gemm_tc(L, Epi::StoreF32, a, K, w, M, N, K, ea, m->hdr(), PERSISTENT_VARIANT));
+    } else {
+        CK(launch_gemm_tc(L, Epi::StoreF32, a, K, w, M, N, K, ea, m->hdr(), PAIR_VARIANT + kernel - (4 + n_tc + 5)));
     }
     return RLT_OK;
 }
@@ -1337,8 +1340,11 @@ rlt_status rlt_gemm_bf16(rlt_model* m, const void* A, const void* W, float* C, i
 rlt_status rlt_selftest_wait_timeout(rlt_model* m, const void* A, const void* W, float* C, int M, int N, int K,
                                      int kernel, uint64_t wait_ns, void* stream) {
     const int n_tc = gemm_tc_variants();
-    if (!m || !A || !W || !C || M < 1 || N < 1 || K < 1 || kernel < 2 || kernel > 1 + n_tc + 5) return RLT_EINVAL;
-    if (kernel > 1 + n_tc && !gemm_swap_supported(M)) return RLT_EINVAL;
+    const int pair0 = 4 + n_tc + 5;          // kernel ids of the CTA-pair tiles
+    const bool pair = kernel >= pair0 && kernel < pair0 + N_PAIR_VARIANTS;
+    if (!m || !A || !W || !C || M < 1 || N < 1 || K < 1 || kernel < 2 || (kernel > 1 + n_tc + 5 && !pair))
+        return RLT_EINVAL;
+    if (kernel > 1 + n_tc && !pair && !gemm_swap_supported(M)) return RLT_EINVAL;
     if (!aligned(A, 16) || !aligned(W, 16) || !aligned(C, 16) || K % 8 || N % 4) return RLT_EINVAL;
     if (wait_ns < 1000 || wait_ns > 2000000000ull) return RLT_EINVAL;
     Launch L = m->launch(stream);
@@ -1350,7 +1356,9 @@ rlt_status rlt_selftest_wait_timeout(rlt_model* m, const void* A, const void* W,
     ea.no_loads = 1;
     const bf16* a = reinterpret_cast<const bf16*>(A);
     const bf16* w = reinterpret_cast<const bf16*>(W);
-    if (kernel <= 1 + n_tc) {
+    if (pair) {
+        CK(launch_gemm_tc(L, Epi::StoreF32, a, K, w, M, N, K, ea, m->hdr(), PAIR_VARIANT + kernel - pair0));
+    } else if (kernel <= 1 + n_tc) {
         CK(launch_gemm_tc(L, Epi::StoreF32, a, K, w, M, N, K, ea, m->hdr(), kernel - 2));
     } else {
         static const int splits[5] = {0, 1, 2, 4, 8};

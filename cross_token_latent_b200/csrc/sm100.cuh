@@ -1,6 +1,8 @@
 // sm_100a building blocks shared by the tensor-core kernels: bounded mbarrier waits, TMA
 // tiled loads, tcgen05 (UMMA) descriptors, MMA issue/commit, tensor-memory loads and stores,
-// and cluster barriers / distributed shared memory.  No multicast form is used.
+// cluster barriers / distributed shared memory, and the CTA-pair (cta_group::2) forms.  No load
+// (TMA or other) uses multicast; the one multicast form is the CTA-pair MMA commit, which
+// arrives on the mbarriers of the two CTAs of a pair.
 #pragma once
 
 #include <cuda.h>
@@ -161,6 +163,47 @@ __device__ __forceinline__ void dsmem_store16_strided(const float* local, int st
         asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote + 4u * (uint32_t)(j * stride)), "f"(v[j]) : "memory");
 }
 
+
+// ---- CTA pairs (cta_group::2): a cluster of two CTAs runs one MMA of M = 256.  CTA r of the
+// pair holds rows 128 r .. 128 r + 127 of A and columns (N / 2) r .. of B in its own shared
+// memory at the same offsets, and receives rows 128 r .. of the accumulator in its own TMEM.
+
+// Shared::cluster address of the object at local address p in cluster CTA `rank`.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ uint32_t dsmem_ld_u32(uint32_t cluster_address) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_address) : "memory");
+    return v;
+}
+// 2-D tiled TMA load into this CTA's shared memory whose completion is counted on an mbarrier
+// of either CTA of the pair (bar_cluster: a shared::cluster address).  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
+                                                 int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+        "%4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(bar_cluster), "r"(x), "r"(y)
+        : "memory");
+}
+__device__ __forceinline__ void umma_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+// Arrive on the mbarrier at bar's offset in the CTAs of the pair that cta_mask selects (bit r:
+// cluster CTA r) once every MMA issued so far has completed.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t cta_mask = 3) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+        ::"r"(smem_u32(bar)), "h"(cta_mask)
+        : "memory");
+}
 
 // Host: encode (and cache) a tiled bf16 tensor map with 128-byte swizzle, zero fill out of
 // bounds.  dims/box innermost first; strides_bytes has rank-1 entries.

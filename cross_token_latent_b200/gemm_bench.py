@@ -5,7 +5,8 @@
 
 Kernel ids are those of rlt_gemm_bf16: 0 = the library's own choice for the shape, 1 = CUDA
 cores, 2 + v = row-tile variant v, 11 + s = few-row kernel (s: 0 chosen, 1..4 = split 1/2/4/8),
-16 = the weight-streaming CUDA-core kernel (M <= 4).
+16 = the weight-streaming CUDA-core kernel (M <= 4), 17 = the persistent row-tile kernel,
+18 + p = the CTA-pair tiles 256 x (64 << p).
 The weight matrix cycles through enough copies (> 256 MB) that every launch reads it from
 HBM, as one decoder step does; the activation panel stays L2-resident.  Launches are queued
 behind a device-side sleep so that the host's launch rate does not limit the timing.  With

@@ -416,7 +416,8 @@ class RLTModel:
     def gemm_bf16(self, A: torch.Tensor, W: torch.Tensor, kernel: int = 0,
                   out: torch.Tensor | None = None) -> torch.Tensor:
         """C = A W^T (bf16 in, float32 out) with the kernel id of rlt_gemm_bf16 (0: the library's
-        choice, 1: CUDA cores, 2 + v: row-tile variant v, 11 + s: few-row kernel)."""
+        choice, 1: CUDA cores, 2 + v: row-tile variant v, 11 + s: few-row kernel, 16: weight
+        streaming, 17: persistent, 18 + p: CTA-pair tiles 256 x (64 << p))."""
         A = A.to(self.device, torch.bfloat16).contiguous()
         W = W.to(self.device, torch.bfloat16).contiguous()
         M, K = A.shape

@@ -372,8 +372,10 @@ rlt_status rlt_set_option(rlt_model* m, const char* name, int64_t value);
  * 4: 8) CTAs, kernel 16 (M <= 4, N a multiple of 32, K <= 6144) = the weight-streaming
  * CUDA-core kernel, kernel 17 = the persistent row-tile kernel (128x256 tiles, one CTA per SM
  * walking the tiles, two tensor-memory accumulators so that a tile's epilogue overlaps the next
- * tile's MMAs; the library's choice for grids of more than one wave).  A, W, C 16-byte aligned,
- * K a multiple of 8, N a multiple of 4.
+ * tile's MMAs; the library's choice for grids of more than one wave), kernel 18 + p = the
+ * CTA-pair row-tile kernel (a cluster of two CTAs computes a 256 x (64 << p) tile with one
+ * tcgen05 MMA of M = 256; each CTA stages half of the A rows and half of the W rows).  A, W, C
+ * 16-byte aligned, K a multiple of 8, N a multiple of 4.
  * Errors: RLT_EINVAL, RLT_ECUDA; a tensor-core wait that times out latches
  * RLT_ETIMEOUT (rlt_last_error). */
 rlt_status rlt_gemm_bf16(rlt_model* m, const void* A, const void* W, float* C, int M, int N, int K,

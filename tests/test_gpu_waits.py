@@ -21,9 +21,11 @@ pytestmark = pytest.mark.gpu
 RLT_ETIMEOUT = 4
 WAIT_NS = 1_000_000
 
-# kernel ids as rlt_gemm_bf16 numbers them: 2 + v row-tile variant v, 11 + s few-row kernel
+# kernel ids as rlt_gemm_bf16 numbers them: 2 + v row-tile variant v, 11 + s few-row kernel,
+# 18 + p CTA-pair tiles
 CASES = {
     "row-tile 128x64": (3, 256, 512, 512),
+    "CTA pair 256x128": (19, 512, 512, 1024),
     "row-tile 128x128 K split over 2 CTAs": (7, 256, 512, 1024),
     "few-row K split over 2 CTAs": (13, 16, 512, 1024),
 }
