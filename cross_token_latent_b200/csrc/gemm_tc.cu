@@ -371,10 +371,15 @@ __device__ __forceinline__ void epilogue_row(Epi epi, const EpiArgs& ea, uint32_
     }
 }
 
-template <int BN, int STAGES, int SPLIT>
+// KA: 64-wide k-atoms per pipeline stage.  A stage of narrow tiles is delivered at a roughly
+// fixed rate per stage (measured on B200 at decode sizes: ~0.29 us per 64-wide stage for 32-,
+// 64- and 128-column tiles with 4 to 10 stages in flight, ~0.43 us per 128-wide stage), so
+// two atoms per stage shorten the k-loop of the narrow tiles by about a quarter.  A stage is
+// [KA atoms of A (16 KB each)][KA atoms of W].
+template <int BN, int STAGES, int SPLIT, int KA = 1>
 struct TcShape {
-    static constexpr int B_BYTES = BN * BK * 2;
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int B_BYTES = BN * BK * 2;                // one W atom
+    static constexpr int STAGE_BYTES = KA * (A_BYTES + B_BYTES);
     static constexpr int TMEM_COLS = BN < 32 ? 32 : BN;
     // split-K: the owner CTA of a row band receives every rank's partial rows here
     static constexpr int BAND = BN / SPLIT;          // split-K: output columns each rank owns
@@ -389,11 +394,11 @@ struct TcShape {
 // each column band of its partial tile (BN / SPLIT columns per rank) to the CTA that owns the
 // band through distributed shared memory; the owner adds the SPLIT partials in rank order (the
 // same order for every element and every run) and applies the epilogue with all 128 threads.
-template <int BN, int STAGES, int SPLIT>
+template <int BN, int STAGES, int SPLIT, int KA>
 __global__ void __launch_bounds__(128, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW, int M, int N, int K,
           Epi epi, EpiArgs ea, DevHeader* hdr) {
-    using S = TcShape<BN, STAGES, SPLIT>;
+    using S = TcShape<BN, STAGES, SPLIT, KA>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* recv = reinterpret_cast<float*>(smem + STAGES * S::STAGE_BYTES);
@@ -405,7 +410,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
-    const int nkb_all = (K + BK - 1) / BK;
+    const int nkb_all = (K + BK * KA - 1) / (BK * KA);          // stages of KA atoms
     const uint32_t rank = SPLIT > 1 ? cluster_rank() : 0;
     const int per = (nkb_all + SPLIT - 1) / SPLIT;
     const int kb0 = min(nkb_all, (int)rank * per);
@@ -444,11 +449,15 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         for (int kb = 0; kb < pre; ++kb) {
             uint8_t* a = smem + kb * S::STAGE_BYTES;
             mbar_expect_tx(&full[kb], S::STAGE_BYTES);
-            tma_load_2d(a + A_BYTES, &tmW, &full[kb], (kb0 + kb) * BK, n0);
+#pragma unroll
+            for (int q = 0; q < KA; ++q)
+                tma_load_2d(a + KA * A_BYTES + q * S::B_BYTES, &tmW, &full[kb], ((kb0 + kb) * KA + q) * BK, n0);
         }
         pdl_wait();
         for (int kb = 0; kb < pre; ++kb)
-            tma_load_2d(smem + kb * S::STAGE_BYTES, &tmA, &full[kb], (kb0 + kb) * BK, m0);
+#pragma unroll
+            for (int q = 0; q < KA; ++q)
+                tma_load_2d(smem + kb * S::STAGE_BYTES + q * A_BYTES, &tmA, &full[kb], ((kb0 + kb) * KA + q) * BK, m0);
         armed = pre;
         for (int kb = pre; kb < nkb && !ea.no_loads; ++kb) {
             int s = kb % STAGES;
@@ -456,8 +465,11 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
             if (!mbar_wait(&empty[s], ph ^ 1, &abort_flag, lim)) { abort_flag = 1; break; }
             uint8_t* a = smem + s * S::STAGE_BYTES;
             mbar_expect_tx(&full[s], S::STAGE_BYTES);
-            tma_load_2d(a, &tmA, &full[s], (kb0 + kb) * BK, m0);
-            tma_load_2d(a + A_BYTES, &tmW, &full[s], (kb0 + kb) * BK, n0);
+#pragma unroll
+            for (int q = 0; q < KA; ++q) {
+                tma_load_2d(a + q * A_BYTES, &tmA, &full[s], ((kb0 + kb) * KA + q) * BK, m0);
+                tma_load_2d(a + KA * A_BYTES + q * S::B_BYTES, &tmW, &full[s], ((kb0 + kb) * KA + q) * BK, n0);
+            }
             armed = kb + 1;
         }
     } else if (warp == 1 && lane == 0) {
@@ -470,10 +482,13 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
             if (!mbar_wait(&full[s], ph, &abort_flag, lim)) { abort_flag = 1; break; }
             tc_fence_after();
             uint8_t* a = smem + s * S::STAGE_BYTES;
-            uint64_t da = sdesc_sw128(a), dw = sdesc_sw128(a + A_BYTES);
 #pragma unroll
-            for (int k = 0; k < BK / 16; ++k)      // advance 16 elements = 32 bytes = 2 in (addr >> 4)
-                umma(tmem, da + 2 * k, dw + 2 * k, idesc, (kb | k) != 0);
+            for (int q = 0; q < KA; ++q) {
+                const uint64_t da = sdesc_sw128(a + q * A_BYTES), dw = sdesc_sw128(a + KA * A_BYTES + q * S::B_BYTES);
+#pragma unroll
+                for (int k = 0; k < BK / 16; ++k)  // advance 16 elements = 32 bytes = 2 in (addr >> 4)
+                    umma(tmem, da + 2 * k, dw + 2 * k, idesc, (kb | q | k) != 0);
+            }
             umma_commit(&empty[s]);
         }
         if (nkb > 0) umma_commit(done);
@@ -994,13 +1009,13 @@ bool tma_map_bf16(CUtensorMap* map, const void* ptr, int rank, const uint64_t* d
 
 namespace {
 
-template <int BN, int STAGES, int SPLIT>
+template <int BN, int STAGES, int SPLIT, int KA = 1>
 cudaError_t run_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K, const EpiArgs& ea,
                    DevHeader* hdr) {
-    using S = TcShape<BN, STAGES, SPLIT>;
+    using S = TcShape<BN, STAGES, SPLIT, KA>;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN, STAGES, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN, STAGES, SPLIT, KA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              S::SMEM);
         if (e != cudaSuccess) return e;
         attr_set = true;
@@ -1009,7 +1024,7 @@ cudaError_t run_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int
     if (!cached_map(&ta, A, M, K, lda, BM) || !cached_map(&tw, W, N, K, K, BN)) return cudaErrorInvalidValue;
     dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, SPLIT);
     if constexpr (SPLIT == 1) {
-        return launch_k(L, k_gemm_tc<BN, STAGES, 1>, grid, 128, S::SMEM, ta, tw, M, N, K, epi, ea, hdr);
+        return launch_k(L, k_gemm_tc<BN, STAGES, 1, KA>, grid, 128, S::SMEM, ta, tw, M, N, K, epi, ea, hdr);
     } else {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = grid;
@@ -1026,7 +1041,7 @@ cudaError_t run_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int
         cfg.attrs = attr;
         cfg.numAttrs = 2;
         *L.count += 1;
-        return cudaLaunchKernelEx(&cfg, k_gemm_tc<BN, STAGES, SPLIT>, ta, tw, M, N, K, epi, ea, hdr);
+        return cudaLaunchKernelEx(&cfg, k_gemm_tc<BN, STAGES, SPLIT, KA>, ta, tw, M, N, K, epi, ea, hdr);
     }
 }
 
@@ -1082,37 +1097,39 @@ cudaError_t run_tc_pers(Launch L, Epi epi, const bf16* A, int lda, const bf16* W
     return launch_k(L, k_gemm_tc_pers<BN, STAGES>, grid, 192, SMEM, ta, tw, M, N, K, epi, ea, hdr);
 }
 
-// Tile variants: (BN, stages, k-split over a cluster) and how many CTAs fit on one SM.
+// Tile variants: (BN, stages, CTAs per SM, k-split over a cluster, 64-wide k-atoms per stage).
+// Two atoms per stage where it measured faster at decode sizes (B200, 512 x 1024 x 1024:
+// 128x64 split 2 7.06 -> 6.28 us; 512 x 3072 x 1024: 128x128 9.85 -> 8.51 us; 64 x 2048 x 2048:
+// 128x64 split 4 7.35 -> 6.61 us); the 256-wide tile is bound by its MMAs and keeps one.
 struct TcVariant {
-    int bn, stages, per_sm, split;
+    int bn, stages, per_sm, split, ka;
 };
 constexpr TcVariant VARIANTS[] = {
-    // Decode-size grids run one CTA per SM, and a CTA's k-loop advances one ring of STAGES
-    // tiles per TMA round trip, so the narrow tiles fill ~200 KB of shared memory with stages.
-    {32, 10, 1, 1},    // 200 KB
-    {64, 8, 1, 1},     // 192 KB
-    {128, 3, 2, 1},    //  96 KB (two CTAs per SM for grids of up to two waves)
-    {128, 6, 1, 1},    // 192 KB
-    {256, 4, 1, 1},    // 192 KB
-    {128, 4, 1, 2},    // 128 KB + 64 KB partials
-    {128, 4, 1, 4},
-    {64, 7, 1, 2},     // 168 KB + 32 KB partials
-    {64, 7, 1, 4},
+    // Decode-size grids run one CTA per SM, so the rings fill ~200 KB of shared memory.
+    {32, 5, 1, 1, 2},     // 200 KB
+    {64, 4, 1, 1, 2},     // 192 KB
+    {128, 3, 2, 1, 1},    //  96 KB (two CTAs per SM for grids of up to two waves)
+    {128, 3, 1, 1, 2},    // 192 KB
+    {256, 4, 1, 1, 1},    // 192 KB
+    {128, 4, 1, 2, 1},    // 128 KB + 64 KB partials
+    {128, 2, 1, 4, 2},    // 128 KB + 64 KB
+    {64, 3, 1, 2, 2},     // 144 KB + 32 KB partials
+    {64, 3, 1, 4, 2},     // 144 KB + 32 KB
 };
 constexpr int N_VARIANTS = sizeof(VARIANTS) / sizeof(VARIANTS[0]);
 
 cudaError_t run_variant(int v, Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                         const EpiArgs& ea, DevHeader* hdr) {
     switch (v) {
-        case 0: return run_tc<32, 10, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 1: return run_tc<64, 8, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 2: return run_tc<128, 3, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 3: return run_tc<128, 6, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 4: return run_tc<256, 4, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 5: return run_tc<128, 4, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 6: return run_tc<128, 4, 4>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 7: return run_tc<64, 7, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 8: return run_tc<64, 7, 4>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 0: return run_tc<32, 5, 1, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 1: return run_tc<64, 4, 1, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 2: return run_tc<128, 3, 1, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 3: return run_tc<128, 3, 1, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 4: return run_tc<256, 4, 1, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 5: return run_tc<128, 4, 2, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 6: return run_tc<128, 2, 4, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 7: return run_tc<64, 3, 2, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 8: return run_tc<64, 3, 4, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
     }
     return cudaErrorInvalidValue;
 }
@@ -1142,7 +1159,7 @@ int pick_variant(int M, int N, int K) {
     for (int v = 5; v < N_VARIANTS; ++v) {
         const TcVariant& t = VARIANTS[v];
         long long ctas = mt * ((N + t.bn - 1) / t.bn) * t.split;
-        if (ctas > 148 || t.split > nkb) continue;
+        if (ctas > 148 || t.split * t.ka > nkb) continue;
         if (ctas > best_ctas) { best = v; best_ctas = ctas; }
     }
     if (best >= 0 && best_ctas >= 64) return best;

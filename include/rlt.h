@@ -364,10 +364,10 @@ rlt_status rlt_set_option(rlt_model* m, const char* name, int64_t value);
  * accumulation/output, on the model's stream-ordered error flags.  kernel 0 = the
  * tensor-core (tcgen05 + TMA) kernel and tile shape the library's own projections use for
  * this shape (row tiles, or the few-row kernel below), kernel 1 =
- * the CUDA-core kernel, kernel 2 + v = tensor-core tile variant v (0: 128x32 tiles, 10 stages;
- * 1: 128x64, 8; 2: 128x128, 3; 3: 128x128, 6; 4: 128x256, 4; then K split over a cluster of
- * CTAs with a shared-memory reduction: 5: 128x128 split 2; 6: 128x128 split 4; 7: 128x64
- * split 2; 8: 128x64 split 4), kernel 11 + s (M <= 64 only) = the few-row kernel with the
+ * the CUDA-core kernel, kernel 2 + v = tensor-core tile variant v (0: 128x32 tiles; 1: 128x64;
+ * 2: 128x128, two CTAs per SM; 3: 128x128; 4: 128x256; then K split over a cluster of CTAs
+ * with a shared-memory reduction: 5: 128x128 split 2; 6: 128x128 split 4; 7: 128x64 split 2;
+ * 8: 128x64 split 4), kernel 11 + s (M <= 64 only) = the few-row kernel with the
  * weights on the MMA's M side and K split over a cluster of (s = 0: chosen, 1: 1, 2: 2, 3: 4,
  * 4: 8) CTAs, kernel 16 (M <= 4, N a multiple of 32, K <= 6144) = the weight-streaming
  * CUDA-core kernel, kernel 17 = the persistent row-tile kernel (128x256 tiles, one CTA per SM
