@@ -23,10 +23,12 @@ constexpr int FM = 128;                      // weight rows (features) per CTA: 
 constexpr int KB = 64;                       // k-block: one 128-byte swizzle row
 constexpr int W_BYTES = FM * KB * 2;
 
-template <int NB, int STAGES, int SPLIT>
+// KA 64-wide k-atoms per pipeline stage: [KA weight atoms][KA activation atoms] (larger
+// stages shorten the k-loop: a stage is delivered at a nearly fixed rate, see gemm_tc.cu).
+template <int NB, int STAGES, int SPLIT, int KA = 1>
 struct SwShape {
-    static constexpr int X_BYTES = NB * KB * 2;
-    static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
+    static constexpr int X_BYTES = NB * KB * 2;          // one activation atom
+    static constexpr int STAGE_BYTES = KA * (W_BYTES + X_BYTES);
     static constexpr int TMEM_COLS = NB < 32 ? 32 : NB;
     static constexpr int ROWS_PER_OWNER = FM / SPLIT;
     // the owner's partials, batch-column-major per source rank: [SPLIT][NB][ROWS_PER_OWNER]
@@ -112,11 +114,11 @@ __device__ __forceinline__ void epilogue16_t(Epi epi, const EpiArgs& ea, int n, 
     }
 }
 
-template <int NB, int STAGES, int SPLIT>
+template <int NB, int STAGES, int SPLIT, int KA>
 __global__ void __launch_bounds__(128, 1)
 k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, int M, int N, int K,
             Epi epi, EpiArgs ea, DevHeader* hdr) {
-    using S = SwShape<NB, STAGES, SPLIT>;
+    using S = SwShape<NB, STAGES, SPLIT, KA>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* recv = reinterpret_cast<float*>(smem + STAGES * S::STAGE_BYTES);
@@ -129,7 +131,7 @@ k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int f0 = blockIdx.x * FM, b0 = blockIdx.y * NB;
-    const int nkb_all = (K + KB - 1) / KB;
+    const int nkb_all = (K + KB * KA - 1) / (KB * KA);          // stages of KA atoms
     const uint32_t rank = SPLIT > 1 ? cluster_rank() : 0;
     const int per = (nkb_all + SPLIT - 1) / SPLIT;
     const int kb0 = min(nkb_all, (int)rank * per);
@@ -163,16 +165,21 @@ k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmX) : "memory");
         // every CTA reads the same activation k-blocks: rotate the start (as in gemm_tc.cu)
         const int rot = nkb > 0 ? (int)(blockIdx.x % (unsigned)nkb) : 0;
-        auto kx = [&](int kb) { return (kb0 + (kb + rot) % nkb) * KB; };
+        // element offset of atom q of stage kb
+        auto kx = [&](int kb, int q) { return ((kb0 + (kb + rot) % nkb) * KA + q) * KB; };
         // the bounded-wait self-test (ea.no_loads) issues nothing
         const int pre = ea.no_loads ? 0 : (nkb < STAGES ? nkb : STAGES);
         for (int kb = 0; kb < pre; ++kb) {
             mbar_expect_tx(&full[kb], S::STAGE_BYTES);
-            tma_load_2d(smem + kb * S::STAGE_BYTES, &tmW, &full[kb], kx(kb), f0);
+#pragma unroll
+            for (int q = 0; q < KA; ++q)
+                tma_load_2d(smem + kb * S::STAGE_BYTES + q * W_BYTES, &tmW, &full[kb], kx(kb, q), f0);
         }
         pdl_wait();
         for (int kb = 0; kb < pre; ++kb)
-            tma_load_2d(smem + kb * S::STAGE_BYTES + W_BYTES, &tmX, &full[kb], kx(kb), b0);
+#pragma unroll
+            for (int q = 0; q < KA; ++q)
+                tma_load_2d(smem + kb * S::STAGE_BYTES + KA * W_BYTES + q * S::X_BYTES, &tmX, &full[kb], kx(kb, q), b0);
         armed = pre;
         for (int kb = pre; kb < nkb && !ea.no_loads; ++kb) {
             int s = kb % STAGES;
@@ -180,8 +187,11 @@ k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
             if (!mbar_wait(&empty[s], ph ^ 1, &abort_flag, lim)) { abort_flag = 1; break; }
             uint8_t* st = smem + s * S::STAGE_BYTES;
             mbar_expect_tx(&full[s], S::STAGE_BYTES);
-            tma_load_2d(st, &tmW, &full[s], kx(kb), f0);
-            tma_load_2d(st + W_BYTES, &tmX, &full[s], kx(kb), b0);
+#pragma unroll
+            for (int q = 0; q < KA; ++q) {
+                tma_load_2d(st + q * W_BYTES, &tmW, &full[s], kx(kb, q), f0);
+                tma_load_2d(st + KA * W_BYTES + q * S::X_BYTES, &tmX, &full[s], kx(kb, q), b0);
+            }
             armed = kb + 1;
         }
     } else if (warp == 1 && lane == 0) {
@@ -193,9 +203,12 @@ k_gemm_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
             if (!mbar_wait(&full[s], ph, &abort_flag, lim)) { abort_flag = 1; break; }
             tc_fence_after();
             uint8_t* st = smem + s * S::STAGE_BYTES;
-            uint64_t dw = sdesc_sw128(st), dx = sdesc_sw128(st + W_BYTES);
 #pragma unroll
-            for (int k = 0; k < KB / 16; ++k) umma(tmem, dw + 2 * k, dx + 2 * k, idesc, (kb | k) != 0);
+            for (int q = 0; q < KA; ++q) {
+                const uint64_t dw = sdesc_sw128(st + q * W_BYTES), dx = sdesc_sw128(st + KA * W_BYTES + q * S::X_BYTES);
+#pragma unroll
+                for (int k = 0; k < KB / 16; ++k) umma(tmem, dw + 2 * k, dx + 2 * k, idesc, (kb | q | k) != 0);
+            }
             umma_commit(&empty[s]);
         }
         if (nkb > 0) umma_commit(done);
@@ -294,13 +307,13 @@ bool map2d(CUtensorMap* map, const void* ptr, int rows, int cols, int ld, int bo
     return tma_map_bf16(map, ptr, 2, dims, strides, box);
 }
 
-template <int NB, int STAGES, int SPLIT>
+template <int NB, int STAGES, int SPLIT, int KA>
 cudaError_t run_swap(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K, const EpiArgs& ea,
                      DevHeader* hdr) {
-    using S = SwShape<NB, STAGES, SPLIT>;
+    using S = SwShape<NB, STAGES, SPLIT, KA>;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_gemm_swap<NB, STAGES, SPLIT>,
+        cudaError_t e = cudaFuncSetAttribute(k_gemm_swap<NB, STAGES, SPLIT, KA>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
         if (e != cudaSuccess) return e;
         attr_set = true;
@@ -328,19 +341,21 @@ cudaError_t run_swap(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, i
     cfg.attrs = attr;
     cfg.numAttrs = na;
     *L.count += 1;
-    return cudaLaunchKernelEx(&cfg, k_gemm_swap<NB, STAGES, SPLIT>, tw, tx, M, N, K, epi, ea, hdr);
+    return cudaLaunchKernelEx(&cfg, k_gemm_swap<NB, STAGES, SPLIT, KA>, tw, tx, M, N, K, epi, ea, hdr);
 }
 
 template <int NB>
 cudaError_t run_swap_split(int split, Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                            const EpiArgs& ea, DevHeader* hdr) {
-    // one CTA per SM: as many stages as fit next to the split partials (~200 KB)
-    constexpr int ST = NB == 16 ? 10 : (NB == 32 ? 9 : 7);
+    // one CTA per SM: as many stages of two k-atoms (measured faster than one at every few-row
+    // decode shape, e.g. 32 x 2048 x 5632 split 4: 10.85 -> 9.53 us) as fit next to the split
+    // partials (~200 KB)
+    constexpr int ST = NB == 64 ? 4 : 5;
     switch (split) {
-        case 1: return run_swap<NB, ST, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 2: return run_swap<NB, ST, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 4: return run_swap<NB, ST, 4>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 8: return run_swap<NB, ST, 8>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 1: return run_swap<NB, ST, 1, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 2: return run_swap<NB, ST, 2, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 4: return run_swap<NB, ST, 4, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 8: return run_swap<NB, ST, 8, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
     }
     return cudaErrorInvalidValue;
 }
