@@ -338,19 +338,20 @@ __device__ __forceinline__ void epilogue32_staged(Epi epi, const EpiArgs& ea, in
     }
 }
 
-// The epilogue of one accumulator row m (TMEM lanes at lane_base, columns n0 .. n0+BN-1 of
-// output column tile tn), through the warp's staging area stg where the chunk allows it.
-// Warp-collective (TMEM loads, staging).
+// The epilogue of one accumulator row m (TMEM lanes at lane_base, columns n0 + c_begin ..
+// n0 + c_end - 1 of output column tile tn; LsePart takes all BN columns), through the warp's
+// staging area stg where the chunk allows it.  Warp-collective (TMEM loads, staging).
 template <int BN>
 __device__ __forceinline__ void epilogue_row(Epi epi, const EpiArgs& ea, uint32_t lane_base, int m, int M, int n0,
-                                             int N, int tn, RowNorm& rn, uint8_t* stg) {
+                                             int N, int tn, RowNorm& rn, uint8_t* stg, int c_begin = 0,
+                                             int c_end = BN) {
     if (epi == Epi::LsePart) {
         lse_row<BN>(ea, lane_base, m, M, n0, N, tn);
         return;
     }
     const int row0 = m - (int)(threadIdx.x & 31);
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = c_begin; c < c_end; c += 32) {
         const int n = n0 + c;
         if (staged_ok(epi, ea, n, N)) {
             float v[32];
@@ -360,7 +361,7 @@ __device__ __forceinline__ void epilogue_row(Epi epi, const EpiArgs& ea, uint32_
             continue;
         }
 #pragma unroll 1
-        for (int h = c; h < c + 32 && h < BN; h += 16) {
+        for (int h = c; h < c + 32 && h < c_end; h += 16) {
             float v[16];
             tmem_ld16(lane_base + h, v);
             if (m < M && n0 + h < N) {
@@ -394,11 +395,14 @@ struct TcShape {
 // each column band of its partial tile (BN / SPLIT columns per rank) to the CTA that owns the
 // band through distributed shared memory; the owner adds the SPLIT partials in rank order (the
 // same order for every element and every run) and applies the epilogue with all 128 threads.
-template <int BN, int STAGES, int SPLIT, int KA>
-__global__ void __launch_bounds__(128, 1)
+// EW = 8 (wide tiles without a split): four more warps join the epilogue only, warps w and w + 4
+// sharing TMEM lane quadrant w and taking one half of the tile's columns each.
+template <int BN, int STAGES, int SPLIT, int KA, int EW>
+__global__ void __launch_bounds__(EW * 32, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW, int M, int N, int K,
           Epi epi, EpiArgs ea, DevHeader* hdr) {
     using S = TcShape<BN, STAGES, SPLIT, KA>;
+    static_assert(EW == 4 || (EW == 8 && SPLIT == 1 && BN >= 64), "eight epilogue warps: unsplit tiles");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* recv = reinterpret_cast<float*>(smem + STAGES * S::STAGE_BYTES);
@@ -496,20 +500,29 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     __syncwarp();
     pdl_wait();
 
-    // epilogue: thread owns output row m0 + 32*warp + lane (a split rank with no k-blocks has
-    // issued no MMA and contributes zeros)
+    // epilogue: thread owns output row m0 + 32 * (warp % 4) + lane (a split rank with no
+    // k-blocks has issued no MMA and contributes zeros)
+    const int qd = warp & 3, chalf = EW == 8 ? warp >> 2 : 0;
     RowNorm rn;
-    if (ea.ss_in && m0 + warp * 32 + lane < M) rn.rinv = deferred_rinv(ea, m0 + warp * 32 + lane);
+    if (ea.ss_in && m0 + qd * 32 + lane < M) rn.rinv = deferred_rinv(ea, m0 + qd * 32 + lane);
     bool ok = nkb == 0 ? true : mbar_wait(done, 0, nullptr, lim);
     // a producer or issuer that gave up raised abort_flag before this barrier: no thread then
     // stores a partial accumulator
     ok = __syncthreads_and(ok) && abort_flag == 0;
     tc_fence_after();
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
     if constexpr (SPLIT == 1) {
-        // every stage of the ring has been consumed: its first 16 KB are the warps' staging areas
-        if (ok) epilogue_row<BN>(epi, ea, lane_base, m0 + warp * 32 + lane, M, n0, N, blockIdx.x, rn,
+        // every stage of the ring has been consumed: its first EW * 4 KB are the warps' staging
+        // areas.  With eight warps each half of the columns has its own warp (the fused head's
+        // per-row reduction stays with the first four).
+        if (ok && (EW == 4 || epi == Epi::LsePart)) {
+            if (chalf == 0)
+                epilogue_row<BN>(epi, ea, lane_base, m0 + qd * 32 + lane, M, n0, N, blockIdx.x, rn,
                                  smem + warp * STG_BYTES);
+        } else if (ok) {
+            epilogue_row<BN>(epi, ea, lane_base, m0 + qd * 32 + lane, M, n0, N, blockIdx.x, rn, smem + warp * STG_BYTES,
+                             chalf * (BN / 2), (chalf + 1) * (BN / 2));
+        }
     } else {
         // Column bands: rank r owns output columns [r * BAND, (r + 1) * BAND) of the tile for
         // all 128 rows, so every thread keeps its row.  It sends each band of its partial row
@@ -752,14 +765,17 @@ k_gemm_tc_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 //   warp 1           allocates the 2 * BN TMEM columns; lane 0 issues the MMAs of tile i into
 //                    accumulator i % 2 once the epilogue has drained it (acc_empty), then
 //                    commits acc_full;
-//   warps 2-5        epilogue: warp w reads TMEM lanes 32 * (w % 4) .. +31, i.e. output rows
-//                    of that quadrant, with the fused epilogues of k_gemm_tc, then arrives on
-//                    acc_empty.
+//   warps 2-9        epilogue: warp w reads TMEM lanes 32 * (w % 4) .. +31, i.e. output rows
+//                    of that quadrant, and columns of half (w - 2) / 4 of the tile (the fused
+//                    head's per-row reduction: warps 2-5 over all columns), with the fused
+//                    epilogues of k_gemm_tc, then arrives on acc_empty.
 // Every wait is bounded; after a timeout every role stops, the MMA issuer still commits what it
 // issued, the CTA waits (bounded) for its loads in flight, latches ERR_TIMEOUT and stores
 // nothing more.
+constexpr int PERS_EPI_WARPS = 8;
+
 template <int BN, int STAGES>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__((2 + PERS_EPI_WARPS) * 32, 1)
 k_gemm_tc_pers(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW, int M, int N, int K,
                Epi epi, EpiArgs ea, DevHeader* hdr) {
     using S = TcShape<BN, STAGES, 1>;
@@ -790,7 +806,7 @@ k_gemm_tc_pers(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&acc_full[a], 1);
-            mbar_init(&acc_empty[a], 4);             // one arrival per epilogue warp
+            mbar_init(&acc_empty[a], PERS_EPI_WARPS);   // one arrival per epilogue warp
         }
         abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -859,7 +875,7 @@ k_gemm_tc_pers(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     } else {
         // epilogue warps: TMEM lane quadrant q = warp % 4 holds output rows 32q .. 32q+31
         pdl_wait();
-        const int q = warp & 3;
+        const int q = warp & 3, chalf = (warp - 2) / 4;
         int count = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++count) {
             const int a = count & 1, use = count >> 1;
@@ -873,7 +889,11 @@ k_gemm_tc_pers(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             if (!ok) { abort_flag = 1; break; }
             tc_fence_after();
             const uint32_t lane_base = tmem + a * BN + ((uint32_t)(q * 32) << 16);
-            epilogue_row<BN>(epi, ea, lane_base, m, M, n0, N, tn, rn, stg_all + q * STG_BYTES);
+            if (epi != Epi::LsePart)
+                epilogue_row<BN>(epi, ea, lane_base, m, M, n0, N, tn, rn, stg_all + (warp - 2) * STG_BYTES,
+                                 chalf * (BN / 2), (chalf + 1) * (BN / 2));
+            else if (chalf == 0)
+                epilogue_row<BN>(epi, ea, lane_base, m, M, n0, N, tn, rn, stg_all + (warp - 2) * STG_BYTES);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[a]);
@@ -1009,13 +1029,13 @@ bool tma_map_bf16(CUtensorMap* map, const void* ptr, int rank, const uint64_t* d
 
 namespace {
 
-template <int BN, int STAGES, int SPLIT, int KA = 1>
+template <int BN, int STAGES, int SPLIT, int KA = 1, int EW = 4>
 cudaError_t run_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K, const EpiArgs& ea,
                    DevHeader* hdr) {
     using S = TcShape<BN, STAGES, SPLIT, KA>;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN, STAGES, SPLIT, KA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN, STAGES, SPLIT, KA, EW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              S::SMEM);
         if (e != cudaSuccess) return e;
         attr_set = true;
@@ -1024,7 +1044,7 @@ cudaError_t run_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int
     if (!cached_map(&ta, A, M, K, lda, BM) || !cached_map(&tw, W, N, K, K, BN)) return cudaErrorInvalidValue;
     dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, SPLIT);
     if constexpr (SPLIT == 1) {
-        return launch_k(L, k_gemm_tc<BN, STAGES, 1, KA>, grid, 128, S::SMEM, ta, tw, M, N, K, epi, ea, hdr);
+        return launch_k(L, k_gemm_tc<BN, STAGES, 1, KA, EW>, grid, EW * 32, S::SMEM, ta, tw, M, N, K, epi, ea, hdr);
     } else {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = grid;
@@ -1041,7 +1061,7 @@ cudaError_t run_tc(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int
         cfg.attrs = attr;
         cfg.numAttrs = 2;
         *L.count += 1;
-        return cudaLaunchKernelEx(&cfg, k_gemm_tc<BN, STAGES, SPLIT, KA>, ta, tw, M, N, K, epi, ea, hdr);
+        return cudaLaunchKernelEx(&cfg, k_gemm_tc<BN, STAGES, SPLIT, KA, 4>, ta, tw, M, N, K, epi, ea, hdr);
     }
 }
 
@@ -1082,7 +1102,7 @@ template <int BN, int STAGES>
 cudaError_t run_tc_pers(Launch L, Epi epi, const bf16* A, int lda, const bf16* W, int M, int N, int K,
                         const EpiArgs& ea, DevHeader* hdr) {
     using S = TcShape<BN, STAGES, 1>;
-    constexpr int SMEM = STAGES * S::STAGE_BYTES + 1024 + 256 + 4 * STG_BYTES;   // + the epilogue staging
+    constexpr int SMEM = STAGES * S::STAGE_BYTES + 1024 + 256 + PERS_EPI_WARPS * STG_BYTES;   // + epilogue staging
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(k_gemm_tc_pers<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1094,10 +1114,11 @@ cudaError_t run_tc_pers(Launch L, Epi epi, const bf16* A, int lda, const bf16* W
     if (!cached_map(&ta, A, M, K, lda, BM) || !cached_map(&tw, W, N, K, K, BN)) return cudaErrorInvalidValue;
     const long long tiles = (long long)((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const unsigned grid = (unsigned)(tiles < sm_count() ? tiles : sm_count());
-    return launch_k(L, k_gemm_tc_pers<BN, STAGES>, grid, 192, SMEM, ta, tw, M, N, K, epi, ea, hdr);
+    return launch_k(L, k_gemm_tc_pers<BN, STAGES>, grid, (2 + PERS_EPI_WARPS) * 32, SMEM, ta, tw, M, N, K, epi, ea, hdr);
 }
 
-// Tile variants: (BN, stages, CTAs per SM, k-split over a cluster, 64-wide k-atoms per stage).
+// Tile variants: (BN, stages, CTAs per SM, k-split over a cluster, 64-wide k-atoms per stage);
+// the one-per-SM 128- and 256-wide unsplit tiles run their epilogue on eight warps.
 // Two atoms per stage where it measured faster at decode sizes (B200, 512 x 1024 x 1024:
 // 128x64 split 2 7.06 -> 6.28 us; 512 x 3072 x 1024: 128x128 9.85 -> 8.51 us; 64 x 2048 x 2048:
 // 128x64 split 4 7.35 -> 6.61 us); the 256-wide tile is bound by its MMAs and keeps one.
@@ -1124,8 +1145,8 @@ cudaError_t run_variant(int v, Launch L, Epi epi, const bf16* A, int lda, const 
         case 0: return run_tc<32, 5, 1, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
         case 1: return run_tc<64, 4, 1, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
         case 2: return run_tc<128, 3, 1, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 3: return run_tc<128, 3, 1, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
-        case 4: return run_tc<256, 4, 1, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 3: return run_tc<128, 3, 1, 2, 8>(L, epi, A, lda, W, M, N, K, ea, hdr);
+        case 4: return run_tc<256, 4, 1, 1, 8>(L, epi, A, lda, W, M, N, K, ea, hdr);
         case 5: return run_tc<128, 4, 2, 1>(L, epi, A, lda, W, M, N, K, ea, hdr);
         case 6: return run_tc<128, 2, 4, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
         case 7: return run_tc<64, 3, 2, 2>(L, epi, A, lda, W, M, N, K, ea, hdr);
