@@ -166,12 +166,21 @@ struct RowNorm {
     }
 };
 
-// Fused head (Epi::LsePart) for one row m over the BN accumulator columns at lane_base: the
-// row's (max, sum of exp) of z = acc * scale over the tile's columns n0 .. n0+BN-1 (those
-// below N) goes to lse_part[m * lse_ld + tn], and the tile that holds the row's target column
-// writes its z to z_tok[m].  Nothing is stored per logit.  Warp-collective (TMEM loads).
+// Fused head (Epi::LsePart): nothing is stored per logit.  For row m, lse_partial returns the
+// (max, sum of exp) of z = acc * scale over accumulator columns c_begin .. c_end - 1 of the tile
+// (those below N), and the thread whose columns hold the row's target writes its z to z_tok[m];
+// the tile's (max, sum) goes to lse_part[m * lse_ld + tn].  The exponentials use ex2.approx
+// (relative error near 2^-22): the log-sum-exp and the log-probs are outputs only, nothing of
+// the recurrent state depends on them.  Warp-collective (TMEM loads).
+constexpr float LOG2E_F = 1.4426950408889634f;
+__device__ __forceinline__ float exp_fast(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x * LOG2E_F));
+    return y;
+}
 template <int BN>
-__device__ __forceinline__ void lse_row(const EpiArgs& ea, uint32_t lane_base, int m, int M, int n0, int N, int tn) {
+__device__ __forceinline__ float2 lse_partial(const EpiArgs& ea, uint32_t lane_base, int m, int M, int n0, int N,
+                                              int c_begin, int c_end) {
     int tk = -1;
     if (m < M && ea.lse_tok) {
         tk = ea.lse_tok[(long long)m * ea.tok_stride];
@@ -179,7 +188,7 @@ __device__ __forceinline__ void lse_row(const EpiArgs& ea, uint32_t lane_base, i
     }
     float mx = -INFINITY, sm = 0.f;
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 16) {
+    for (int c = c_begin; c < c_end; c += 16) {
         float v[16];
         tmem_ld16(lane_base + c, v);
         const int n = n0 + c;
@@ -193,15 +202,39 @@ __device__ __forceinline__ void lse_row(const EpiArgs& ea, uint32_t lane_base, i
                 if (n + j == tk) ea.z_tok[m] = v[j];
             }
             if (cm > mx) {
-                sm *= expf(mx - cm);
+                sm *= exp_fast(mx - cm);
                 mx = cm;
             }
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-                if (j < cnt) sm += expf(v[j] - mx);
+                if (j < cnt) sm += exp_fast(v[j] - mx);
         }
     }
-    if (m < M) ea.lse_part[(long long)m * ea.lse_ld + tn] = make_float2(mx, sm);
+    return make_float2(mx, sm);
+}
+// (max, sum of exp) of two column ranges, a's first
+__device__ __forceinline__ float2 lse_merge(float2 a, float2 b) {
+    const float mx = fmaxf(a.x, b.x);
+    if (mx == -INFINITY) return make_float2(mx, 0.f);
+    return make_float2(mx, a.y * exp_fast(a.x - mx) + b.y * exp_fast(b.x - mx));
+}
+template <int BN>
+__device__ __forceinline__ void lse_row(const EpiArgs& ea, uint32_t lane_base, int m, int M, int n0, int N, int tn) {
+    const float2 p = lse_partial<BN>(ea, lane_base, m, M, n0, N, 0, BN);
+    if (m < M) ea.lse_part[(long long)m * ea.lse_ld + tn] = p;
+}
+// AND of v over the nthreads threads that meet at named barrier id (all of them must arrive).
+__device__ __forceinline__ bool bar_and(int id, int nthreads, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.cta.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
 }
 
 // ---- Staged epilogue.  A warp owns 32 consecutive output rows (lane = row).  Writing each
@@ -515,10 +548,17 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         // every stage of the ring has been consumed: its first EW * 4 KB are the warps' staging
         // areas.  With eight warps each half of the columns has its own warp (the fused head's
         // per-row reduction stays with the first four).
-        if (ok && (EW == 4 || epi == Epi::LsePart)) {
-            if (chalf == 0)
-                epilogue_row<BN>(epi, ea, lane_base, m0 + qd * 32 + lane, M, n0, N, blockIdx.x, rn,
-                                 smem + warp * STG_BYTES);
+        if (ok && EW == 8 && epi == Epi::LsePart) {
+            // each half reduces its columns; the second half's (max, sum) pass through shared
+            // memory (past the staging areas) to the first, which merges them in column order
+            const int m = m0 + qd * 32 + lane;
+            const float2 part = lse_partial<BN>(ea, lane_base, m, M, n0, N, chalf * (BN / 2), (chalf + 1) * (BN / 2));
+            float2* xbuf = reinterpret_cast<float2*>(smem + EW * STG_BYTES);
+            if (chalf == 1) xbuf[qd * 32 + lane] = part;
+            __syncthreads();
+            if (chalf == 0 && m < M) ea.lse_part[(long long)m * ea.lse_ld + blockIdx.x] = lse_merge(part, xbuf[qd * 32 + lane]);
+        } else if (ok && EW == 4) {
+            epilogue_row<BN>(epi, ea, lane_base, m0 + qd * 32 + lane, M, n0, N, blockIdx.x, rn, smem + warp * STG_BYTES);
         } else if (ok) {
             epilogue_row<BN>(epi, ea, lane_base, m0 + qd * 32 + lane, M, n0, N, blockIdx.x, rn, smem + warp * STG_BYTES,
                              chalf * (BN / 2), (chalf + 1) * (BN / 2));
@@ -886,14 +926,24 @@ k_gemm_tc_pers(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             if (ea.ss_in && m < M) rn.rinv = deferred_rinv(ea, m);
             bool ok = mbar_wait(&acc_full[a], use & 1, &abort_flag, lim);
             ok = __all_sync(0xffffffffu, ok) && abort_flag == 0;
+            // the fused head's halves meet at a named barrier below: all eight epilogue warps
+            // take the same decision (every one of them reaches this barrier: its wait is bounded)
+            if (epi == Epi::LsePart) ok = bar_and(1, PERS_EPI_WARPS * 32, ok);
             if (!ok) { abort_flag = 1; break; }
             tc_fence_after();
             const uint32_t lane_base = tmem + a * BN + ((uint32_t)(q * 32) << 16);
-            if (epi != Epi::LsePart)
+            if (epi != Epi::LsePart) {
                 epilogue_row<BN>(epi, ea, lane_base, m, M, n0, N, tn, rn, stg_all + (warp - 2) * STG_BYTES,
                                  chalf * (BN / 2), (chalf + 1) * (BN / 2));
-            else if (chalf == 0)
-                epilogue_row<BN>(epi, ea, lane_base, m, M, n0, N, tn, rn, stg_all + (warp - 2) * STG_BYTES);
+            } else {
+                // two halves of the columns, merged in column order through shared memory (two
+                // buffers by tile parity: a buffer is rewritten only after the next barrier)
+                const float2 part = lse_partial<BN>(ea, lane_base, m, M, n0, N, chalf * (BN / 2), (chalf + 1) * (BN / 2));
+                float2* xbuf = reinterpret_cast<float2*>(stg_all) + (count & 1) * BM;
+                if (chalf == 1) xbuf[q * 32 + lane] = part;
+                asm volatile("bar.sync 1, %0;" ::"r"(PERS_EPI_WARPS * 32) : "memory");
+                if (chalf == 0 && m < M) ea.lse_part[(long long)m * ea.lse_ld + tn] = lse_merge(part, xbuf[q * 32 + lane]);
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[a]);
