@@ -1,15 +1,19 @@
 // Tensor-core GEMM for sm_100a: C[M, N] = A[M, K] x W[N, K]^T with bf16 operands, float32
 // accumulation in tensor memory (TMEM) and the fused epilogues of the RLT path.
 //
-// One CTA computes one 128 x BN output tile with 4 warps:
+// One CTA computes one 128 x BN output tile with 4 warps (8 for the wide unsplit tiles):
 //   warp 0, lane 0  TMA producer: 2-D tiled loads (128-byte swizzle) of A and W k-blocks of
-//                   64 elements into a ring of STAGES shared-memory slots (mbarrier full[s]);
+//                   64 elements (KA of them per stage) into a ring of STAGES shared-memory
+//                   slots (mbarrier full[s]);
 //   warp 1, lane 0  MMA issuer: four tcgen05.mma (M=128, N=BN, K=16) per k-block into the
 //                   TMEM accumulator; tcgen05.commit frees the slot (empty[s]) and, after
 //                   the last block, signals the epilogue (done);
 //   warp 2          allocates / frees the TMEM columns;
-//   all 4 warps     epilogue: warp w reads TMEM lanes 32w..32w+31 (one output row per
-//                   thread) with tcgen05.ld and applies the fused epilogue.
+//   all warps       epilogue: warp w reads TMEM lanes 32(w%4)..32(w%4)+31 (one output row per
+//                   thread; with 8 warps, warps w and w+4 take one half of the columns each)
+//                   with tcgen05.ld and applies the fused epilogue, staged through shared
+//                   memory.
+// The file also holds the CTA-pair (cta_group::2) and the persistent variants.
 // No load uses multicast.  Every mbarrier wait is bounded by %globaltimer; on
 // expiry the CTA raises ERR_TIMEOUT, stops issuing work, frees its TMEM and returns.
 #include <cuda.h>
