@@ -90,3 +90,7 @@ def test_null_handles_are_rejected():
     assert L.rlt_sample(None, None, 1, None, 0, 1.0, None, 1, None, None) == 1
     assert L.rlt_set_option(None, b"row_groups", 1) == 1
     assert L.rlt_selftest_wait_timeout(None, None, None, None, 1, 1, 8, 2, 1000000, None) == 1
+    # the GEMM building block: every kernel id (0-20) and one past the last
+    for k in (0, 17, 18, 20, 21):
+        assert L.rlt_gemm_bf16(None, None, None, None, 8, 8, 8, k, None) == 1
+        assert L.rlt_selftest_wait_timeout(None, None, None, None, 8, 8, 8, k, 1000000, None) == 1
